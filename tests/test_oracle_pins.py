@@ -1,0 +1,446 @@
+"""Pins of the CPU oracle against what the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: closed forms,
+an independent library implementation (Hugging Face Llama for the causal
+decoder, scipy for entropy), brute force over small inputs, and decode traces
+worked out by hand from the rules (tests/golden/)."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import wedlm_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+PIN_DIMS = dict(L=2, d=64, hq=4, hkv=2, hd=16, F=96, V=50, theta=10000.0, eps=1e-6, mask_id=49)
+
+
+def pin_weights(dims, std=0.25, seed=7):
+    """Weights large enough that attention is sharp and every term matters."""
+    w = synth.model_weights(dims, seed=seed, dtype="f32")
+    scale = std / synth.WEIGHT_STD
+    for key in ("embed", "lm_head"):
+        w[key] = (w[key] * scale).astype(np.float32)
+    for lw in w["layers"]:
+        for k in ("wq", "wk", "wv", "wo", "wg", "wu", "wd"):
+            lw[k] = (lw[k] * scale).astype(np.float32)
+        # non-trivial norm gains so a dropped gain is visible
+        lw["attn_norm"] = (1.0 + 0.5 * synth.uniform01(seed, 900, dims["d"])).astype(np.float32)
+        lw["ffn_norm"] = (1.0 + 0.5 * synth.uniform01(seed, 901, dims["d"])).astype(np.float32)
+    w["final_norm"] = (1.0 + 0.5 * synth.uniform01(seed, 902, dims["d"])).astype(np.float32)
+    return w
+
+
+def hf_llama_logits(dims, w, tokens):
+    """Logits of the same decoder built with Hugging Face's Llama implementation."""
+    import torch
+    from transformers import LlamaConfig, LlamaForCausalLM
+    cfg = LlamaConfig(hidden_size=dims["d"], intermediate_size=dims["F"], num_hidden_layers=dims["L"],
+                      num_attention_heads=dims["hq"], num_key_value_heads=dims["hkv"], head_dim=dims["hd"],
+                      vocab_size=dims["V"], rope_theta=dims["theta"], rms_norm_eps=dims["eps"],
+                      attention_bias=False, mlp_bias=False, tie_word_embeddings=False,
+                      max_position_embeddings=4096)
+    cfg._attn_implementation = "eager"
+    model = LlamaForCausalLM(cfg).double().eval()
+    sd = {"model.embed_tokens.weight": w["embed"], "lm_head.weight": w["lm_head"],
+          "model.norm.weight": w["final_norm"]}
+    for l, lw in enumerate(w["layers"]):
+        p = f"model.layers.{l}."
+        sd.update({p + "self_attn.q_proj.weight": lw["wq"], p + "self_attn.k_proj.weight": lw["wk"],
+                   p + "self_attn.v_proj.weight": lw["wv"], p + "self_attn.o_proj.weight": lw["wo"],
+                   p + "mlp.gate_proj.weight": lw["wg"], p + "mlp.up_proj.weight": lw["wu"],
+                   p + "mlp.down_proj.weight": lw["wd"], p + "input_layernorm.weight": lw["attn_norm"],
+                   p + "post_attention_layernorm.weight": lw["ffn_norm"]})
+    model.load_state_dict({k: torch.tensor(np.asarray(v, np.float64)) for k, v in sd.items()}, strict=True)
+    with torch.no_grad():
+        out = model(torch.tensor(np.asarray(tokens, np.int64))[None]).logits[0]
+    return out.numpy()
+
+
+def oracle_causal_logits(dims, w, tokens):
+    m = O.Model(dims, w)
+    hidden, _, _ = O.forward_window(m, O.KVCache.empty(m), tokens, np.arange(len(tokens)))
+    return O.lm_logits(m, hidden, 1.0)
+
+
+# ------------------------------------------------------------ forward ----
+def test_forward_matches_independent_llama_implementation():
+    """A plain causal forward (all slots filled, empty cache) is a standard
+    RMSNorm/GQA/RoPE/SwiGLU decoder: compare with Hugging Face's Llama."""
+    w = pin_weights(PIN_DIMS)
+    toks = synth.token_ids(3, 0, PIN_DIMS["V"], 23, exclude=PIN_DIMS["mask_id"])
+    ref = hf_llama_logits(PIN_DIMS, w, toks)
+    got = oracle_causal_logits(PIN_DIMS, w, toks)
+    # the library keeps RMSNorm statistics and rotary tables in fp32: ~1e-6 rel
+    err = np.abs(got - ref).max() / np.abs(ref).max()
+    assert err < 2e-5, err
+    assert np.abs(ref).max() > 1.0  # a sharp, non-degenerate test model
+
+
+def test_forward_with_cache_equals_forward_without():
+    """Splitting a causal forward into a cached prefix and a window gives the same rows."""
+    w = pin_weights(PIN_DIMS)
+    m = O.Model(PIN_DIMS, w)
+    toks = synth.token_ids(4, 0, PIN_DIMS["V"], 17, exclude=PIN_DIMS["mask_id"])
+    full, fk, fv = O.forward_window(m, O.KVCache.empty(m), toks, np.arange(17))
+    cache = O.KVCache.empty(m)
+    _, k1, v1 = O.forward_window(m, cache, toks[:11], np.arange(11))
+    cache.append(k1, v1)
+    part, k2, v2 = O.forward_window(m, cache, toks[11:], np.arange(11, 17))
+    np.testing.assert_allclose(part, full[11:], rtol=1e-12, atol=1e-12)
+    for l in range(m.L):
+        np.testing.assert_allclose(k2[l], fk[l][11:], rtol=1e-12, atol=1e-13)
+
+
+def test_rms_norm_closed_form():
+    x = np.array([[3.0, 4.0]])
+    g = np.array([2.0, 0.5])
+    got = O.rms_norm(x, g, 0.0)
+    want = np.array([[3.0 / math.sqrt(12.5) * 2.0, 4.0 / math.sqrt(12.5) * 0.5]])
+    np.testing.assert_allclose(got, want, rtol=1e-15)
+
+
+def test_rope_two_dim_is_rotation_by_position_radians():
+    """hd = 2: a single pair rotated by pos * theta^0 = pos radians (counter-clockwise)."""
+    x = np.array([[[1.0, 0.5]]])
+    for p in (0.0, 1.0, 2.5, 7.0):
+        got = O.rope(x, np.array([p]), 10000.0)[0, 0]
+        want = [math.cos(p) * 1.0 - math.sin(p) * 0.5, math.sin(p) * 1.0 + math.cos(p) * 0.5]
+        np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-15)
+
+
+def test_rope_pairs_and_frequencies():
+    """hd = 4 with theta = 100: pair (0, 2) turns by p, pair (1, 3) by p / 10."""
+    x = np.array([[[1.0, 2.0, 3.0, 4.0]]])
+    p = 3.0
+    got = O.rope(x, np.array([p]), 100.0)[0, 0]
+    a0, a1 = p, p / 10.0
+    want = [1 * math.cos(a0) - 3 * math.sin(a0), 2 * math.cos(a1) - 4 * math.sin(a1),
+            3 * math.cos(a0) + 1 * math.sin(a0), 4 * math.cos(a1) + 2 * math.sin(a1)]
+    np.testing.assert_allclose(got, want, rtol=1e-13)
+
+
+def test_rope_scores_depend_only_on_relative_position():
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((1, 1, 32))
+    k = rng.standard_normal((1, 1, 32))
+    s = [float((O.rope(q, np.array([p + 5.0]), 1e4) * O.rope(k, np.array([p + 0.0]), 1e4)).sum())
+         for p in (0, 17, 400)]
+    np.testing.assert_allclose(s, s[0], rtol=1e-11)
+
+
+# ---------------------------------------------------- topological reorder --
+def brute_force_visibility_attention(q, kc, vc, kw, vw, filled):
+    """Attention by logical visibility (Summary/Method): a filled slot sees the
+    cache and filled slots at positions <= its own; a mask slot sees the cache,
+    all filled slots and mask slots at positions <= its own."""
+    n, hq, hd = q.shape
+    hkv = kw.shape[1]
+    g = hq // hkv
+    out = np.zeros_like(q)
+    for i in range(n):
+        vis = [j for j in range(n) if (filled[j] and j <= i) or (not filled[i] and (filled[j] or j <= i))]
+        for h in range(hq):
+            kv = h // g
+            keys = np.concatenate([kc[:, kv], kw[vis, kv]], 0)
+            vals = np.concatenate([vc[:, kv], vw[vis, kv]], 0)
+            s = keys @ q[i, h] / math.sqrt(hd)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            out[i, h] = p @ vals
+    return out
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_reordered_causal_attention_equals_logical_visibility(seed):
+    """Topological reordering under a plain causal mask gives every mask slot
+    all observed tokens (Summary/Method; Abstract)."""
+    rng = np.random.default_rng(seed)
+    W, S, hq, hkv, hd = 7, 5, 4, 2, 8
+    filled = list(rng.random(W) < 0.5)
+    q = rng.standard_normal((W, hq, hd))
+    kw = rng.standard_normal((W, hkv, hd))
+    vw = rng.standard_normal((W, hkv, hd))
+    kc = rng.standard_normal((S, hkv, hd))
+    vc = rng.standard_normal((S, hkv, hd))
+    perm = O.reorder(filled)
+    phys = O.window_attention(q[perm], kc, vc, kw[perm], vw[perm])
+    got = np.empty_like(phys)
+    got[perm] = phys
+    want = brute_force_visibility_attention(q, kc, vc, kw, vw, filled)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("W", range(0, 9))
+def test_reorder_is_stable_partition_exhaustive(W):
+    for bits in range(1 << W):
+        filled = [(bits >> j) & 1 == 1 for j in range(W)]
+        perm = O.reorder(filled)
+        assert sorted(perm) == list(range(W))
+        nf = sum(filled)
+        assert all(filled[j] for j in perm[:nf]) and not any(filled[j] for j in perm[nf:])
+        assert perm[:nf] == sorted(perm[:nf]) and perm[nf:] == sorted(perm[nf:])
+        k = O.leading_filled(filled)
+        assert perm[:k] == list(range(k))       # the commit run is the physical prefix
+        assert all(filled[:k]) and (k == W or not filled[k])
+
+
+def test_reorder_hand_example():
+    assert O.reorder([False, True, False, True, True]) == [1, 3, 4, 0, 2]
+    assert O.leading_filled([True, True, False, True]) == 2
+    assert O.leading_filled([False, True]) == 0
+
+
+# ------------------------------------------------------------- entropy ----
+def test_entropy_uniform_excludes_mask():
+    V, mask = 64, 63
+    H, a = O.entropy_argmax(np.zeros(V), mask)
+    assert abs(H - math.log(V - 1)) < 1e-13
+    assert a == 0
+
+
+def test_entropy_two_valued_closed_form():
+    V, mask, c = 100, 5, 2.75
+    z = np.zeros(V)
+    A = [3, 17, 40]
+    z[A] = c
+    H, a = O.entropy_argmax(z, mask)
+    Vp, na = V - 1, len(A)
+    Z = na * math.exp(c) + (Vp - na)
+    want = math.log(Z) - na * c * math.exp(c) / Z
+    assert abs(H - want) < 1e-12
+    assert a == 3   # lowest id among the maxima
+
+
+def test_entropy_matches_scipy_on_random_logits():
+    from scipy.stats import entropy as sp_entropy
+    rng = np.random.default_rng(1)
+    for s in (0.5, 4.0, 16.0):
+        z = rng.standard_normal(1000) * s
+        mask = 999
+        H, a = O.entropy_argmax(z, mask)
+        zz = z[:999]
+        p = np.exp(zz - zz.max())
+        assert abs(H - sp_entropy(p / p.sum())) < 1e-10
+        assert a == int(np.argmax(zz))
+
+
+def test_entropy_ignores_mask_logit():
+    rng = np.random.default_rng(2)
+    z = rng.standard_normal(50)
+    H1, a1 = O.entropy_argmax(z, 10)
+    z2 = z.copy()
+    z2[10] = 1e3
+    H2, a2 = O.entropy_argmax(z2, 10)
+    assert H1 == H2 and a1 == a2 and a1 != 10
+
+
+def test_entropy_one_hot_is_near_zero():
+    z = np.zeros(32)
+    z[4] = 60.0
+    H, a = O.entropy_argmax(z, 31)
+    assert a == 4 and 0 <= H < 1e-20
+
+
+# ----------------------------------------------------------- selection ----
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden("selection_cases.json")["cases"], ids=lambda c: c["name"])
+def test_selection_golden(case):
+    tau = math.inf if case["tau"] == "inf" else case["tau"]
+    Ht = {int(j): O.penalised_entropy(h, int(j), case["lambda"]) for j, h in case["H"].items()}
+    assert O.select_fills(Ht, tau, case["tau_none"]) == case["fills"]
+
+
+def test_selection_brute_force():
+    """Against a direct enumeration of the rule on random small H vectors."""
+    rng = np.random.default_rng(3)
+    for _ in range(2000):
+        n = int(rng.integers(0, 7))
+        offs = sorted(rng.choice(8, size=n, replace=False).tolist())
+        Ht = {j: float(rng.choice([0.1, 0.2, 0.3, 0.5, 0.9])) for j in offs}
+        tau = float(rng.choice([0.0, 0.25, 0.5, 1.0]))
+        none = bool(rng.integers(0, 2))
+        under = [] if none else [j for j in offs if Ht[j] < tau]
+        if under:
+            want = under
+        elif offs:
+            lo = min(Ht.values())
+            want = [min(j for j in offs if Ht[j] == lo)]
+        else:
+            want = []
+        assert O.select_fills(Ht, tau, none) == want
+
+
+# ------------------------------------------------------- decode loop -----
+def scripted_forward(case):
+    c = {int(p): v for p, v in case["c"].items()}
+    tok = {int(p): v for p, v in case["tok"].items()}
+    V = case["vocab"]
+
+    def fwd(m, cache, toks, pos):
+        rows = np.zeros((len(pos), V))
+        for r, p in enumerate(pos):
+            rows[r, tok[int(p)]] = c[int(p)]
+        return rows, [np.zeros((len(pos), 1, 1))], [np.zeros((len(pos), 1, 1))]
+    return fwd
+
+
+class _StubModel:
+    def __init__(self, mask_id):
+        self.mask_id = mask_id
+        self.L, self.hkv, self.hd = 1, 1, 1
+
+
+@pytest.mark.parametrize("case", _golden("scripted_traces.json")["cases"], ids=lambda c: c["name"])
+def test_decode_loop_matches_hand_trace(case):
+    m = _StubModel(case["mask_id"])
+    st = O.stream_decode(m, np.zeros(case["prompt_len"], np.int64), case["N"], case["W"],
+                         case["lambda"], case["tau"], forward=scripted_forward(case))
+    assert len(st.trace) == len(case["steps"])
+    for tr, want in zip(st.trace, case["steps"]):
+        assert (tr.S, tr.n, tr.k, tr.perm, tr.committed) == (want["S"], want["n"], want["k"], want["perm"],
+                                                            want["committed"])
+        assert [[j, tr.argmax[j]] for j in tr.fills] == want["fills"]
+    assert st.out == case["out"]
+    assert st.rows == case["rows"]
+    assert abs(O.p_cache(st) - case["p_cache"]) < 1e-15
+
+
+TINY = synth.CONFIGS["tiny_f32"]
+
+
+@pytest.fixture(scope="module")
+def tiny_model():
+    dims = TINY["model"]
+    return O.Model(dims, synth.model_weights(dims, seed=0, dtype="f32"))
+
+
+def test_window_one_no_penalty_is_greedy_autoregression(tiny_model):
+    """W=1, lambda=0: every step predicts exactly the next position with the
+    whole committed prefix visible, i.e. greedy AR decoding (Abstract)."""
+    prompt = synth.prompts(TINY)[0]
+    N = 12
+    st = O.stream_decode(tiny_model, prompt, N, 1, 0.0, 0.5, logit_scale=TINY["logit_scale"])
+    ar = O.ar_greedy_recompute(tiny_model, prompt, N, logit_scale=TINY["logit_scale"])
+    assert st.out == ar
+    assert st.steps == 2 * N
+    assert O.p_cache(st) == 0.5
+
+
+@pytest.mark.parametrize("cfg_name", ["tiny_f32", "tiny_f32_tau"])
+def test_committed_kv_equals_full_recompute(tiny_model, cfg_name):
+    """Prefix cacheability: committed K/V depend only on earlier tokens, so they
+    equal a from-scratch causal forward of the committed sequence (Summary/Method)."""
+    cfg = synth.CONFIGS[cfg_name]
+    prompt = synth.prompts(cfg)[0]
+    st = O.stream_decode(tiny_model, prompt, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"],
+                         logit_scale=cfg["logit_scale"])
+    seq = list(prompt) + st.out
+    assert len(st.out) == cfg["N"]
+    fk, fv = O.full_causal_kv(tiny_model, seq)
+    for l in range(tiny_model.L):
+        np.testing.assert_allclose(st.cache.k[l], fk[l], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(st.cache.v[l], fv[l], rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("cfg_name,W", [("tiny_f32", 4), ("tiny_f32_tau", 4), ("tiny_f32_tau", 7)])
+def test_progress_and_workload_invariants(tiny_model, cfg_name, W):
+    """Fixed parallel workload and progress (Summary/Key Contributions and Method)."""
+    cfg = synth.CONFIGS[cfg_name]
+    prompt = synth.prompts(cfg)[0]
+    N = cfg["N"]
+    st = O.stream_decode(tiny_model, prompt, N, W, cfg["lam"], cfg["tau"], logit_scale=cfg["logit_scale"])
+    end = len(prompt) + N
+    for tr in st.trace:
+        assert tr.n == min(W, end - tr.S)
+        if tr.masked:
+            assert len(tr.fills) >= 1
+    assert st.steps <= 2 * N
+    assert sum(tr.k for tr in st.trace) == N
+    assert 0 < O.p_cache(st) <= 0.5
+    if cfg_name == "tiny_f32_tau":
+        assert max(len(tr.fills) for tr in st.trace) >= 2   # the multi-fill branch runs
+
+
+def test_one_by_one_mode_fills_exactly_one(tiny_model):
+    cfg = synth.CONFIGS["tiny_f32_tau"]
+    prompt = synth.prompts(cfg)[0]
+    st = O.stream_decode(tiny_model, prompt, 10, 4, 0.0, 100.0, tau_none=True, logit_scale=8.0)
+    for tr in st.trace:
+        if tr.masked:
+            assert len(tr.fills) == 1
+            assert tr.fills[0] == min(tr.masked, key=lambda j: (tr.H[j], j))
+
+
+# ------------------------------------------ planted mistakes are caught --
+def _wrong_rope(x, pos, theta):
+    n, _, hd = x.shape
+    half = hd // 2
+    inv = theta ** (-(2.0 * np.arange(half)) / hd)
+    ang = np.asarray(pos, np.float64)[:, None] * inv[None, :]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)   # rotation sign flipped
+
+
+def _wrong_gqa(q, kc, vc, kw, vw):
+    hkv = kw.shape[1]
+    # heads paired with KV heads by h % hkv instead of h // group
+    n, hq, hd = q.shape
+    qq = q.reshape(n, hq // hkv, hkv, hd).transpose(0, 2, 1, 3).reshape(n, hq, hd)
+    out = _orig_attention(qq, kc, vc, kw, vw)
+    return out.reshape(n, hkv, hq // hkv, hd).transpose(0, 2, 1, 3).reshape(n, hq, hd)
+
+
+_orig_attention = O.window_attention
+
+
+@pytest.mark.parametrize("mutation", ["rope_sign", "gqa_mapping", "norm_gain", "no_ffn_residual"])
+def test_llama_pin_detects_planted_forward_mistakes(monkeypatch, mutation):
+    w = pin_weights(PIN_DIMS)
+    toks = synth.token_ids(3, 0, PIN_DIMS["V"], 23, exclude=PIN_DIMS["mask_id"])
+    ref = hf_llama_logits(PIN_DIMS, w, toks)
+    if mutation == "rope_sign":
+        monkeypatch.setattr(O, "rope", _wrong_rope)
+    elif mutation == "gqa_mapping":
+        monkeypatch.setattr(O, "window_attention", _wrong_gqa)
+    elif mutation == "norm_gain":
+        monkeypatch.setattr(O, "rms_norm", lambda x, g, eps: x / np.sqrt(np.mean(x * x, -1, keepdims=True) + eps))
+    elif mutation == "no_ffn_residual":
+        monkeypatch.setattr(O, "silu", lambda x: 0.0 * x)
+    got = oracle_causal_logits(PIN_DIMS, w, toks)
+    assert np.abs(got - ref).max() / np.abs(ref).max() > 1e-3
+
+
+@pytest.mark.parametrize("mutation", ["penalty_sign", "commit_all_filled", "non_strict_tau"])
+def test_hand_traces_detect_planted_loop_mistakes(monkeypatch, mutation):
+    if mutation == "penalty_sign":
+        monkeypatch.setattr(O, "penalised_entropy", lambda H, j, lam: H - lam * j)
+    elif mutation == "commit_all_filled":
+        monkeypatch.setattr(O, "leading_filled", lambda filled: sum(1 for f in filled if f))
+    elif mutation == "non_strict_tau":
+        orig = O.select_fills
+
+        def le(Ht, tau, none):
+            return orig(Ht, np.nextafter(tau, np.inf), none)
+        monkeypatch.setattr(O, "select_fills", le)
+    failures = 0
+    for case in _golden("scripted_traces.json")["cases"]:
+        try:
+            test_decode_loop_matches_hand_trace(case)
+        except (AssertionError, IndexError, KeyError):
+            failures += 1
+    sel_fail = 0
+    for case in _golden("selection_cases.json")["cases"]:
+        tau = math.inf if case["tau"] == "inf" else case["tau"]
+        Ht = {int(j): O.penalised_entropy(h, int(j), case["lambda"]) for j, h in case["H"].items()}
+        sel_fail += O.select_fills(Ht, tau, case["tau_none"]) != case["fills"]
+    assert failures + sel_fail > 0
