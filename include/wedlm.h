@@ -1,0 +1,281 @@
+/*
+ * wedlm.h -- C ABI of libwedlm, a B200 (sm_100a) implementation of WeDLM's
+ * Streaming Parallel Decoding step.
+ *
+ * Method (hyper.ai summary of arXiv 2512.22737, section "Method"; sai.science
+ * review "WeDLM: Reconciling Diffusion Language Models with Standard Causal
+ * Attention for Fast Inference", sections Summary and Recommended Changes):
+ * a sequence keeps a sliding window of W slots, each either filled (a
+ * predicted token) or a mask.  One decode step
+ *   1. refills the window with masks up to min(W, end - S) slots,
+ *   2. reorders it so filled slots physically precede masks, each slot keeping
+ *      its logical position S + offset (Topological Reordering),
+ *   3. runs a causal forward over the reordered window against the persistent
+ *      paged KV cache, with RoPE at logical positions,
+ *   4. commits the leftmost contiguous run of slots that were filled when the
+ *      step began: their K/V depend only on earlier tokens, so they join the
+ *      cache and their tokens are emitted,
+ *   5. fills masked slots by the distance-penalised entropy rule
+ *      H~_j = H_j + lambda * j (j = slot offset): every slot with H~_j < tau,
+ *      or the single argmin if none (one-by-one when tau_none is set), each
+ *      with its argmax token (the mask id is never predicted),
+ *   6. slides the window past the committed run.
+ *
+ * Conventions
+ *   - All functions return a wedlm_status (0 = success, < 0 = error).  No
+ *     function aborts the process or traps the GPU; device-side checks record a
+ *     code in a device error word that the host reads after each call.
+ *   - The library owns all device memory it allocates (weights, KV pages,
+ *     scratch).  Host buffers passed in are owned by the caller and are only
+ *     read or written during the call.
+ *   - A context is bound to the CUDA device current at wedlm_create and to the
+ *     stream given there (borrowed, not owned; NULL = legacy default stream).
+ *     Calls are synchronous on return unless the name ends in _async.
+ *   - A context is not thread-safe; use one context per host thread.
+ *   - Sequence slots are integers in [0, max_batch).
+ *   - KV pages hold WEDLM_PAGE_TOKENS tokens.  Pages for a sequence's whole
+ *     length (prompt + max_new_tokens) are reserved at prefill; running out of
+ *     pages returns WEDLM_ERR_OOM_PAGES and leaves the context unchanged.
+ */
+#ifndef WEDLM_H
+#define WEDLM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t wedlm_status;
+
+#define WEDLM_OK                  0
+#define WEDLM_ERR_INVALID_ARG    -1  /* bad pointer, size, slot or tensor id */
+#define WEDLM_ERR_OOM_PAGES      -2  /* KV page pool exhausted */
+#define WEDLM_ERR_OOM_DEVICE     -3  /* cudaMalloc failed */
+#define WEDLM_ERR_CUDA           -4  /* a CUDA runtime call failed */
+#define WEDLM_ERR_DEVICE_ASSERT  -5  /* a kernel's own bounds check fired */
+#define WEDLM_ERR_STATE          -6  /* call not valid in the current state */
+#define WEDLM_ERR_UNSUPPORTED    -7  /* shape or dtype this build does not run */
+#define WEDLM_ERR_TIMEOUT        -8  /* a bounded device wait gave up */
+
+#define WEDLM_DTYPE_F32   0
+#define WEDLM_DTYPE_BF16  1
+
+#define WEDLM_MEM_HOST    0
+#define WEDLM_MEM_DEVICE  1
+
+#define WEDLM_PAGE_TOKENS 16
+
+/* Model shape and capacity.  A causal decoder: token embedding, L blocks of
+ * [RMSNorm -> GQA attention with RoPE -> residual, RMSNorm -> SwiGLU FFN ->
+ * residual], final RMSNorm, untied LM head (the Qwen2.5-7B / Qwen3-8B
+ * backbones the review names, without biases or QK-norm).
+ * dtype selects the storage and arithmetic of weights, activations and KV:
+ *   WEDLM_DTYPE_F32  fp32 everywhere (SIMT kernels; the exact-parity mode),
+ *   WEDLM_DTYPE_BF16 bf16 storage, fp32 accumulation (tensor-core kernels).
+ * Logits, the residual stream and all softmax/entropy arithmetic are fp32. */
+typedef struct wedlm_model_cfg {
+    int32_t n_layers;
+    int32_t d_model;
+    int32_t n_heads;        /* query heads */
+    int32_t n_kv_heads;     /* KV heads; n_heads % n_kv_heads == 0 */
+    int32_t head_dim;       /* even; bf16 mode requires 128 */
+    int32_t ffn_dim;
+    int32_t vocab;
+    int32_t mask_id;        /* id of the mask token, in [0, vocab) */
+    double  rope_theta;
+    float   rms_eps;
+    int32_t dtype;          /* WEDLM_DTYPE_* */
+    int32_t max_batch;      /* sequence slots */
+    int32_t max_window;     /* largest W any sequence may use (<= 64) */
+    int32_t max_ctx;        /* largest prompt + max_new_tokens of a sequence */
+    int32_t num_pages;      /* KV pool size in pages; 0 = max_batch * ceil(max_ctx / 16) */
+    int32_t prefill_chunk;  /* prompt rows per prefill forward; 0 = 1024 */
+} wedlm_model_cfg;
+
+typedef struct wedlm_ctx wedlm_ctx;
+
+/* Create a context on the current CUDA device.  Allocates weights storage
+ * (uninitialised until wedlm_load_weights), the KV pool and scratch.
+ * cuda_stream: a cudaStream_t (borrowed) or NULL. */
+wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_ctx** out_ctx);
+
+/* Free everything the context owns.  NULL is accepted. */
+void wedlm_destroy(wedlm_ctx* ctx);
+
+/* Static description of a status code. */
+const char* wedlm_status_str(wedlm_status status);
+
+/* Human-readable detail of the context's most recent error ("" if none).
+ * The string is owned by the context and valid until its next call. */
+const char* wedlm_last_error(const wedlm_ctx* ctx);
+
+/* Weight tensors, all in nn.Linear layout [out_features][in_features],
+ * row-major, contiguous:
+ *   EMBED [vocab][d]       LM_HEAD [vocab][d]     FINAL_NORM [d]
+ *   ATTN_NORM [d]          WQ [n_heads*head_dim][d]
+ *   WK, WV [n_kv_heads*head_dim][d]               WO [d][n_heads*head_dim]
+ *   FFN_NORM [d]           WG, WU [ffn][d]        WD [d][ffn]
+ * (per-layer tensors take `layer` in [0, n_layers); others ignore it). */
+#define WEDLM_T_EMBED       0
+#define WEDLM_T_LM_HEAD     1
+#define WEDLM_T_FINAL_NORM  2
+#define WEDLM_T_ATTN_NORM   3
+#define WEDLM_T_WQ          4
+#define WEDLM_T_WK          5
+#define WEDLM_T_WV          6
+#define WEDLM_T_WO          7
+#define WEDLM_T_FFN_NORM    8
+#define WEDLM_T_WG          9
+#define WEDLM_T_WU         10
+#define WEDLM_T_WD         11
+
+/* Copy one weight tensor into the context.  src points to host or device
+ * memory (src_mem = WEDLM_MEM_*) holding the tensor in src_dtype.  Norm gains
+ * must be WEDLM_DTYPE_F32.  Matrices must be in the context's dtype (no
+ * conversion is performed).  The source is not retained.  Every tensor must be
+ * loaded once before the first prefill. */
+wedlm_status wedlm_load_weights(wedlm_ctx* ctx, int32_t tensor, int32_t layer,
+                                const void* src, int32_t src_dtype, int32_t src_mem);
+
+/* Admit a sequence into `slot`: reserve KV pages for prompt_len +
+ * max_new_tokens positions, run the causal prefill forward over the prompt
+ * (host int32 ids, caller-owned) and commit all of it to the cache.  The
+ * sequence then decodes with a window of `window` slots (1 <= window <=
+ * max_window).  The slot must be free (see wedlm_kv_reset).  The prefill
+ * produces no logits: the first window is all masks. */
+wedlm_status wedlm_prefill(wedlm_ctx* ctx, int32_t slot, const int32_t* prompt_ids,
+                           int32_t prompt_len, int32_t max_new_tokens, int32_t window);
+
+/* Release a slot's pages and window (slot = -1: every slot). */
+wedlm_status wedlm_kv_reset(wedlm_ctx* ctx, int32_t slot);
+
+/* Decode knobs (sai.science review, Recommended Changes: lambda = 0.10 and
+ * tau in {0.3, 0.5, 0.9}; Reproducibility & code: a threshold of None gives
+ * one-by-one decoding).  logit_scale multiplies the LM-head logits before
+ * entropy and argmax (an inverse temperature; 1 = the model as loaded). */
+typedef struct wedlm_step_params {
+    float   lambda;       /* distance penalty per slot offset (nats) */
+    float   tau;          /* fill threshold on H~ (nats), strict < */
+    int32_t tau_none;     /* nonzero: fill exactly the argmin each step */
+    float   logit_scale;  /* > 0 */
+} wedlm_step_params;
+
+/* Run one decode step for every active slot (a slot is active from prefill
+ * until its committed length reaches prompt_len + max_new_tokens).
+ * Outputs (host, caller-owned, may be NULL to skip):
+ *   out_committed [max_batch * max_window]: the tokens committed by slot b this
+ *                 step at out_committed[b * max_window + 0 .. count-1]
+ *   out_counts    [max_batch]: tokens committed by each slot this step
+ *   out_active    [1]: slots still decoding after this step
+ * Synchronises the context's stream before returning. */
+wedlm_status wedlm_stream_step(wedlm_ctx* ctx, const wedlm_step_params* params,
+                               int32_t* out_committed, int32_t* out_counts, int32_t* out_active);
+
+/* Enqueue `n_steps` decode steps on the context's stream and return without
+ * waiting or copying results to the host.  Committed tokens accumulate on the
+ * device (read them with wedlm_read_generated).  Slots that finish mid-way
+ * stop decoding; their remaining steps are no-ops. */
+wedlm_status wedlm_stream_step_async(wedlm_ctx* ctx, const wedlm_step_params* params, int32_t n_steps);
+
+/* Copy every token committed so far after the prompt of `slot` (in position
+ * order) to host `out_tokens` (capacity `cap`); *out_len receives the count.
+ * Synchronises the stream. */
+wedlm_status wedlm_read_generated(wedlm_ctx* ctx, int32_t slot, int32_t* out_tokens, int32_t cap,
+                                  int32_t* out_len);
+
+/* Per-slot counters (read from the device; synchronises the stream). */
+typedef struct wedlm_seq_stats {
+    int64_t steps;          /* decode steps run while active */
+    int64_t forward_rows;   /* window rows forwarded by those steps */
+    int64_t committed;      /* generated tokens committed */
+    int64_t fills;          /* mask slots filled */
+    int32_t committed_len;  /* S: prompt + committed tokens */
+    int32_t end;            /* prompt_len + max_new_tokens */
+    int32_t window;         /* W */
+    int32_t active;         /* 1 while S < end */
+} wedlm_seq_stats;
+
+wedlm_status wedlm_get_stats(wedlm_ctx* ctx, int32_t slot, wedlm_seq_stats* out);
+
+/* Number of kernels this context has launched since creation (each launch
+ * counted once; a captured graph counts its kernels at every replay). */
+wedlm_status wedlm_kernel_launches(const wedlm_ctx* ctx, int64_t* out);
+
+/* ---------------------------------------------------------------------
+ * Test hooks.  They expose intermediate state of the most recent step so the
+ * tests can compare each stage with an independent CPU implementation.
+ * ------------------------------------------------------------------- */
+
+/* Items readable with wedlm_debug_read.  The last decode step ran `rows` =
+ * (1 + highest active slot) * Ws physical rows, Ws = the largest window among
+ * active slots; row b * Ws + r is physical row r of slot b. */
+#define WEDLM_DBG_PERM     0  /* int32 [rows]: slot offset at each physical row (-1 = padding) */
+#define WEDLM_DBG_POS      1  /* int32 [rows]: logical position at each row */
+#define WEDLM_DBG_ROWTOK   2  /* int32 [rows]: token fed at each row */
+#define WEDLM_DBG_LOGITS   3  /* float [rows][vocab]: unscaled LM-head logits per row */
+#define WEDLM_DBG_HTILDE   4  /* float [max_batch][max_window]: H~ per slot offset (NaN if not masked) */
+#define WEDLM_DBG_ARGMAX   5  /* int32 [max_batch][max_window]: argmax token per masked slot offset */
+#define WEDLM_DBG_FILL     6  /* uint8 [max_batch][max_window]: 1 where the slot was filled this step */
+#define WEDLM_DBG_KN       7  /* int32 [max_batch][3]: (k, rows n, filled count) of the step */
+#define WEDLM_DBG_ROWSTRIDE 8 /* int32 [2]: (Ws, rows) of the last step */
+
+/* Copy `bytes` of a debug item to host memory.  Synchronises the stream. */
+wedlm_status wedlm_debug_read(wedlm_ctx* ctx, int32_t item, void* host_dst, int64_t bytes);
+
+/* Read cached K and V of `slot`, `layer`, positions [pos0, pos0 + n), widened
+ * to fp32, into host arrays of [n][n_kv_heads][head_dim] each. */
+wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t pos0, int32_t n,
+                            float* host_k, float* host_v);
+
+/* Read / replace a slot's window (host arrays of `n` entries; replacing is
+ * used to drive both implementations from the same state). */
+wedlm_status wedlm_debug_get_window(wedlm_ctx* ctx, int32_t slot, uint8_t* filled, int32_t* tokens,
+                                    int32_t cap, int32_t* n);
+wedlm_status wedlm_debug_set_window(wedlm_ctx* ctx, int32_t slot, const uint8_t* filled,
+                                    const int32_t* tokens, int32_t n);
+
+/* Stand-alone launches of single stages on caller-provided DEVICE buffers
+ * (no context; the caller owns all memory; stream may be NULL).
+ *
+ * Topological reordering (summary, section Method): for each of n_seq windows
+ * of n[b] <= stride slots with flags filled[b*stride + j] (1 = filled):
+ *   k[b]    = length of the leftmost run of filled slots,
+ *   nf[b]   = number of filled slots,
+ *   perm[b*stride + r] = slot offset at physical row r (filled slots in
+ *             ascending order, then masks in ascending order; rows >= n[b]
+ *             get -1),
+ *   pos[b*stride + r]  = S[b] + perm (logical position; -1 past n[b]).
+ * Bit-exact integer work. */
+wedlm_status wedlm_reorder_window(const uint8_t* filled, const int32_t* n, const int32_t* S,
+                                  int32_t n_seq, int32_t stride,
+                                  int32_t* perm, int32_t* pos, int32_t* k, int32_t* nf, void* stream);
+
+/* Distance-penalised entropy selection (summary, section Method; review,
+ * Weaknesses: the functional form is not printed, read here as
+ * H~ = H + lambda * offset).  For each of n_seq windows of n[b] <= stride slots:
+ * logits[(b*stride + j) * vocab + v] (fp32, unscaled) are the logits of slot j;
+ * only slots with filled == 0 are read.  For each such slot:
+ *   H_j = entropy (nats) of softmax(logit_scale * logits) over ids != mask_id,
+ *   argmax_j = lowest id attaining the max (never mask_id),
+ *   htilde[b*stride+j] = H_j + lambda * j  (NaN for filled slots or j >= n[b]).
+ * fill[b*stride+j] = 1 for slots chosen by the threshold / argmin rule, else 0;
+ * argmax[b*stride+j] = argmax_j (or -1).  Device buffers, caller-owned. */
+wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t mask_id,
+                                  const uint8_t* filled, const int32_t* n, int32_t n_seq, int32_t stride,
+                                  const wedlm_step_params* params,
+                                  float* htilde, int32_t* argmax, uint8_t* fill, void* stream);
+
+/* Dense projection on the bf16 tensor-core path: Y = X * W^T with X bf16
+ * [M][K], W bf16 [N][K] (nn.Linear layout), Y fp32 [M][N], all DEVICE
+ * pointers owned by the caller (16-byte aligned; K % 8 == 0).  This is the
+ * kernel every QKV, O, gate/up, down and LM-head projection of the step runs
+ * (split-K partial planes are summed before returning). */
+wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                               void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WEDLM_H */

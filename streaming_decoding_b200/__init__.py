@@ -1,0 +1,5 @@
+"""B200 (sm_100a) implementation of WeDLM Streaming Parallel Decoding.
+
+The decode step runs in libwedlm.so (CUDA kernels behind the C ABI declared in
+include/wedlm.h); ``api`` is its Python binding."""
+from .api import Engine, step_params, reorder_window, entropy_select, linear_bf16  # noqa: F401

@@ -1,0 +1,217 @@
+"""Python binding of libwedlm: the C-ABI calls under the same names, with
+argument marshalling only.  Every step of the decode path runs in the CUDA
+library; this module never computes any part of it.
+
+Host arrays are numpy; device buffers are torch CUDA tensors (PyTorch supplies
+device memory and streams)."""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import _lib
+from ._lib import ModelCfg, SeqStats, StepParams, WedlmError
+
+C = _lib.header_constants()
+DTYPE = {"f32": C["WEDLM_DTYPE_F32"], "bf16": C["WEDLM_DTYPE_BF16"]}
+
+
+def _ptr(a) -> int:
+    if a is None:
+        return 0
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return int(a.data_ptr())  # torch tensor
+
+
+def _check(st: int, where: str, ctx=None):
+    if st != 0:
+        detail = _lib.load().wedlm_last_error(ctx).decode() if ctx else ""
+        raise WedlmError(st, where, detail)
+
+
+def step_params(lam: float, tau: float, tau_none: bool = False, logit_scale: float = 1.0) -> StepParams:
+    return StepParams(float(lam), float(tau), 1 if tau_none else 0, float(logit_scale))
+
+
+class Engine:
+    """One libwedlm context (one model, a batch of sequence slots)."""
+
+    def __init__(self, dims: dict, max_batch: int, max_window: int, max_ctx: int, dtype: str | None = None,
+                 num_pages: int = 0, prefill_chunk: int = 0, stream=None):
+        self.lib = _lib.load()
+        self.dims = dict(dims)
+        dtype = dtype or dims.get("dtype", "f32")
+        self.dtype = dtype
+        cfg = ModelCfg(dims["L"], dims["d"], dims["hq"], dims["hkv"], dims["hd"], dims["F"], dims["V"],
+                       dims["mask_id"], float(dims["theta"]), float(dims["eps"]), DTYPE[dtype], max_batch,
+                       max_window, max_ctx, num_pages, prefill_chunk)
+        self.max_batch, self.max_window, self.max_ctx = max_batch, max_window, max_ctx
+        self.stream = stream
+        h = ctypes.c_void_p()
+        _check(self.lib.wedlm_create(ctypes.byref(cfg), ctypes.c_void_p(_stream_handle(stream)), ctypes.byref(h)),
+               "wedlm_create")
+        self.ctx = h
+
+    # -- lifetime ---------------------------------------------------------
+    def close(self):
+        if getattr(self, "ctx", None):
+            self.lib.wedlm_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+    # -- weights ------------------------------------------------------------
+    def load_weights(self, kind: int, layer: int, src):
+        """src: numpy array (host) or torch CUDA tensor (device); float32 or bf16 (uint16 bits / torch.bfloat16)."""
+        if isinstance(src, np.ndarray):
+            src = np.ascontiguousarray(src)
+            dt = C["WEDLM_DTYPE_BF16"] if src.dtype == np.uint16 else C["WEDLM_DTYPE_F32"]
+            if src.dtype not in (np.uint16, np.float32):
+                raise TypeError(src.dtype)
+            mem = C["WEDLM_MEM_HOST"]
+        else:
+            import torch
+            dt = C["WEDLM_DTYPE_BF16"] if src.dtype in (torch.bfloat16, torch.int16) else C["WEDLM_DTYPE_F32"]
+            mem = C["WEDLM_MEM_DEVICE"] if src.is_cuda else C["WEDLM_MEM_HOST"]
+            src = src.contiguous()
+        _check(self.lib.wedlm_load_weights(self.ctx, kind, layer, _ptr(src), dt, mem), "wedlm_load_weights",
+               self.ctx)
+
+    def load_model(self, weight_iter):
+        for kind, layer, arr in weight_iter:
+            self.load_weights(kind, layer, arr)
+
+    # -- sequences -----------------------------------------------------------
+    def prefill(self, slot: int, prompt, max_new_tokens: int, window: int):
+        p = np.ascontiguousarray(np.asarray(prompt, dtype=np.int32))
+        _check(self.lib.wedlm_prefill(self.ctx, slot, p.ctypes.data if len(p) else None, len(p), max_new_tokens,
+                                      window), "wedlm_prefill", self.ctx)
+
+    def kv_reset(self, slot: int = -1):
+        _check(self.lib.wedlm_kv_reset(self.ctx, slot), "wedlm_kv_reset", self.ctx)
+
+    def stream_step(self, params: StepParams):
+        """One decode step: returns (committed tokens per slot, counts, active)."""
+        committed = np.zeros((self.max_batch, self.max_window), np.int32)
+        counts = np.zeros(self.max_batch, np.int32)
+        active = np.zeros(1, np.int32)
+        _check(self.lib.wedlm_stream_step(self.ctx, ctypes.byref(params), committed.ctypes.data, counts.ctypes.data,
+                                          active.ctypes.data), "wedlm_stream_step", self.ctx)
+        return [committed[b, :counts[b]].tolist() for b in range(self.max_batch)], counts, int(active[0])
+
+    def stream_step_into(self, params: StepParams, committed: np.ndarray, counts: np.ndarray, active: np.ndarray):
+        """Same as stream_step with caller-provided (e.g. pinned) host buffers."""
+        _check(self.lib.wedlm_stream_step(self.ctx, ctypes.byref(params), _ptr(committed), _ptr(counts),
+                                          _ptr(active)), "wedlm_stream_step", self.ctx)
+
+    def stream_step_async(self, params: StepParams, n_steps: int = 1):
+        _check(self.lib.wedlm_stream_step_async(self.ctx, ctypes.byref(params), n_steps), "wedlm_stream_step_async",
+               self.ctx)
+
+    def read_generated(self, slot: int) -> list:
+        buf = np.zeros(self.max_ctx, np.int32)
+        n = ctypes.c_int32()
+        _check(self.lib.wedlm_read_generated(self.ctx, slot, buf.ctypes.data, len(buf), ctypes.byref(n)),
+               "wedlm_read_generated", self.ctx)
+        return buf[:n.value].tolist()
+
+    def stats(self, slot: int) -> dict:
+        s = SeqStats()
+        _check(self.lib.wedlm_get_stats(self.ctx, slot, ctypes.byref(s)), "wedlm_get_stats", self.ctx)
+        return {f: getattr(s, f) for f, _ in SeqStats._fields_}
+
+    def kernel_launches(self) -> int:
+        n = ctypes.c_int64()
+        _check(self.lib.wedlm_kernel_launches(self.ctx, ctypes.byref(n)), "wedlm_kernel_launches")
+        return n.value
+
+    # -- test hooks ---------------------------------------------------------
+    def debug_read(self, item: str, shape, dtype):
+        out = np.zeros(shape, dtype)
+        _check(self.lib.wedlm_debug_read(self.ctx, C["WEDLM_DBG_" + item], out.ctypes.data, out.nbytes),
+               "wedlm_debug_read", self.ctx)
+        return out
+
+    def last_rows(self):
+        v = self.debug_read("ROWSTRIDE", 2, np.int32)
+        return int(v[0]), int(v[1])
+
+    def debug_kv(self, slot: int, layer: int, pos0: int, n: int):
+        hkv, hd = self.dims["hkv"], self.dims["hd"]
+        k = np.zeros((n, hkv, hd), np.float32)
+        v = np.zeros((n, hkv, hd), np.float32)
+        _check(self.lib.wedlm_debug_kv(self.ctx, slot, layer, pos0, n, k.ctypes.data, v.ctypes.data),
+               "wedlm_debug_kv", self.ctx)
+        return k, v
+
+    def get_window(self, slot: int):
+        f = np.zeros(self.max_window, np.uint8)
+        t = np.zeros(self.max_window, np.int32)
+        n = ctypes.c_int32()
+        _check(self.lib.wedlm_debug_get_window(self.ctx, slot, f.ctypes.data, t.ctypes.data, self.max_window,
+                                               ctypes.byref(n)), "wedlm_debug_get_window", self.ctx)
+        return f[:n.value].copy(), t[:n.value].copy()
+
+    def set_window(self, slot: int, filled, tokens):
+        f = np.ascontiguousarray(np.asarray(filled, np.uint8))
+        t = np.ascontiguousarray(np.asarray(tokens, np.int32))
+        _check(self.lib.wedlm_debug_set_window(self.ctx, slot, f.ctypes.data, t.ctypes.data, len(f)),
+               "wedlm_debug_set_window", self.ctx)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return 0
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+# -- stand-alone stage launches (device buffers are torch CUDA tensors) -----
+def reorder_window(filled, n, S, stride: int, stream=None):
+    import torch
+    n_seq = filled.shape[0]
+    dev = filled.device
+    perm = torch.empty((n_seq, stride), dtype=torch.int32, device=dev)
+    pos = torch.empty_like(perm)
+    k = torch.empty(n_seq, dtype=torch.int32, device=dev)
+    nf = torch.empty_like(k)
+    _check(_lib.load().wedlm_reorder_window(_ptr(filled), _ptr(n), _ptr(S), n_seq, stride, _ptr(perm), _ptr(pos),
+                                            _ptr(k), _ptr(nf), _stream_handle(stream)), "wedlm_reorder_window")
+    return perm, pos, k, nf
+
+
+def entropy_select(logits, vocab: int, mask_id: int, filled, n, stride: int, params: StepParams, stream=None):
+    import torch
+    n_seq = filled.shape[0]
+    dev = logits.device
+    ht = torch.empty((n_seq, stride), dtype=torch.float32, device=dev)
+    am = torch.empty((n_seq, stride), dtype=torch.int32, device=dev)
+    fill = torch.empty((n_seq, stride), dtype=torch.uint8, device=dev)
+    _check(_lib.load().wedlm_entropy_select(_ptr(logits), vocab, mask_id, _ptr(filled), _ptr(n), n_seq, stride,
+                                            ctypes.byref(params), _ptr(ht), _ptr(am), _ptr(fill),
+                                            _stream_handle(stream)), "wedlm_entropy_select")
+    return ht, am, fill
+
+
+def linear_bf16(X, W, stream=None):
+    """Y = X W^T (fp32) on the tcgen05 GEMM; X [M][K], W [N][K] torch.bfloat16 CUDA tensors."""
+    import torch
+    M, K = X.shape
+    N = W.shape[0]
+    Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    _check(_lib.load().wedlm_linear_bf16(_ptr(X.contiguous()), _ptr(W.contiguous()), _ptr(Y), M, N, K,
+                                         _stream_handle(stream)), "wedlm_linear_bf16")
+    return Y

@@ -1,0 +1,737 @@
+// Window, epilogue, fp32 and selection kernels of libwedlm.
+//
+// Method references (by page and section):
+//   [Method]  hyper.ai summary of arXiv 2512.22737, section "Method":
+//             Topological Reordering, Streaming Parallel Decoding,
+//             distance-penalised entropy selection.
+//   [Review]  sai.science review "WeDLM: Reconciling Diffusion Language Models
+//             with Standard Causal Attention for Fast Inference".
+#include <cfloat>
+#include <cmath>
+
+#include "kernels.cuh"
+
+namespace wedlm {
+
+// ---------------------------------------------------------------------------
+// Embedding gather + RMSNorm of one row: x = E[tok] (fp32), h = x / rms * g.
+template <typename T>
+__device__ void embed_norm_row(const T* __restrict__ E, int d, int tok, const float* __restrict__ g,
+                               float eps, float* __restrict__ x, T* __restrict__ h, float* red) {
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        const float v = to_f32<T>(E[(int64_t)tok * d + c]);
+        x[c] = v;
+        ss += v * v;
+    }
+    ss = block_sum(ss, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    for (int c = threadIdx.x; c < d; c += blockDim.x) h[c] = from_f32<T>(x[c] * inv * g[c]);
+}
+
+// Decode step window preparation, one CTA per batch entry [Method]:
+//   refill with masks to min(W, end - S) slots; k = leftmost filled run;
+//   stable partition (filled ascending, then masks ascending); logical
+//   position S + offset per physical row; embed + first RMSNorm.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_prepare_kernel(const T* __restrict__ embed, const float* __restrict__ g,
+                                                             float eps, int d, int mask_id, SlotState ss, RowState rs,
+                                                             uint8_t* __restrict__ rowmask, int stride,
+                                                             float* __restrict__ x, T* __restrict__ h) {
+    __shared__ float red[32];
+    __shared__ int s_n;
+    const int slot = blockIdx.x;
+    const int base = slot * stride;
+    if (threadIdx.x == 0) {
+        int n = 0;
+        const int W = ss.W[slot];
+        const int S = ss.S[slot];
+        const int end = ss.end[slot];
+        uint8_t* f = ss.filled + (int64_t)slot * ss.maxW;
+        int32_t* t = ss.token + (int64_t)slot * ss.maxW;
+        if (W > 0 && S < end) {
+            n = min(min(W, end - S), stride);
+            for (int j = ss.wlen[slot]; j < n; ++j) {  // refill
+                f[j] = 0;
+                t[j] = mask_id;
+            }
+            ss.wlen[slot] = n;
+        }
+        int k = 0;
+        while (k < n && f[k]) ++k;
+        int nf = 0;
+        for (int j = 0; j < n; ++j)
+            if (f[j]) {
+                rs.perm[base + nf] = j;
+                ++nf;
+            }
+        int m = nf;
+        for (int j = 0; j < n; ++j)
+            if (!f[j]) rs.perm[base + m++] = j;
+        for (int r = 0; r < stride; ++r) {
+            if (r < n) {
+                const int j = rs.perm[base + r];
+                rs.pos[base + r] = S + j;
+                rs.tok[base + r] = f[j] ? t[j] : mask_id;
+                rowmask[base + r] = f[j] ? 0 : 1;
+            } else {
+                rs.perm[base + r] = -1;
+                rs.pos[base + r] = -1;
+                rs.tok[base + r] = -1;
+                rowmask[base + r] = 0;
+            }
+        }
+        ss.n[slot] = n;
+        ss.k[slot] = k;
+        ss.nf[slot] = nf;
+        s_n = n;
+    }
+    __syncthreads();
+    const int n = s_n;
+    for (int r = 0; r < stride; ++r) {
+        float* xr = x + (int64_t)(base + r) * d;
+        T* hr = h + (int64_t)(base + r) * d;
+        if (r < n) {
+            embed_norm_row<T>(embed, d, rs.tok[base + r], g, eps, xr, hr, red);
+        } else {
+            for (int c = threadIdx.x; c < d; c += blockDim.x) {
+                xr[c] = 0.f;
+                hr[c] = from_f32<T>(0.f);
+            }
+        }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) prefill_prepare_kernel(const T* __restrict__ embed, const float* __restrict__ g,
+                                                              float eps, int d, const int32_t* __restrict__ ids,
+                                                              int slot, int S0, int n, SlotState ss, RowState rs,
+                                                              float* __restrict__ x, T* __restrict__ h) {
+    __shared__ float red[32];
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        ss.S[slot] = S0;
+        ss.n[slot] = n;
+    }
+    for (int r = blockIdx.x; r < n; r += gridDim.x) {
+        if (threadIdx.x == 0) {
+            rs.pos[r] = S0 + r;
+            rs.tok[r] = ids[r];
+            rs.perm[r] = r;
+        }
+        embed_norm_row<T>(embed, d, ids[r], g, eps, x + (int64_t)r * d, h + (int64_t)r * d, red);
+    }
+}
+
+__global__ void slot_admit_kernel(SlotState ss, int slot, int P, int end, int W) {
+    ss.S[slot] = P;
+    ss.P[slot] = P;
+    ss.end[slot] = end;
+    ss.W[slot] = W;
+    ss.wlen[slot] = 0;
+    ss.n[slot] = 0;
+    ss.k[slot] = 0;
+    ss.nf[slot] = 0;
+    for (int j = 0; j < ss.maxW; ++j) {
+        ss.filled[(int64_t)slot * ss.maxW + j] = 0;
+        ss.token[(int64_t)slot * ss.maxW + j] = 0;
+    }
+    for (int c = 0; c < 4; ++c) ss.counters[slot * 4 + c] = 0;
+    ss.out_count[slot] = 0;
+}
+
+__global__ void prefill_finish_kernel(SlotState ss, int slot, int P) {
+    ss.S[slot] = P;
+    ss.n[slot] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// fp32 SIMT GEMM (exact-parity mode): C[M][N] = X[M][K] * W[N][K]^T, fp32 FMA
+// accumulation in ascending k.  64x64 tiles, 16-deep k slabs, 4x4 per thread.
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ X, const float* __restrict__ Wt,
+                                                       float* __restrict__ C, int M, int N, int K) {
+    __shared__ float Xs[16][64 + 1];
+    __shared__ float Ws[16][64 + 1];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        for (int i = tid; i < 64 * 16; i += 256) {
+            const int rr = i / 16, kk = i % 16;
+            const int m = m0 + rr, n = n0 + rr, k = k0 + kk;
+            Xs[kk][rr] = (m < M && k < K) ? X[(int64_t)m * K + k] : 0.f;
+            Ws[kk][rr] = (n < N && k < K) ? Wt[(int64_t)n * K + k] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = Xs[kk][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = Ws[kk][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+            if (m < M && n < N) C[(int64_t)m * N + n] = acc[i][j];
+        }
+}
+
+// ---------------------------------------------------------------------------
+// QKV epilogue: sum split-K partials, rotate q and k at the row's logical
+// position (rotate-half pairs (i, i + hd/2); [Method]: RoPE keeps logical
+// positions through the reordering), write q to q_out[row][hq][hd] and k, v to
+// the paged cache at physical index S + r of the row's sequence (rows 0..k-1
+// of the window are the committed run, so their K/V land at their final
+// cache positions without a copy).
+template <typename T>
+__global__ void __launch_bounds__(256) qkv_rope_kernel(const float* __restrict__ ws, int splits, int64_t sstride,
+                                                       int hq, int hkv, int hd, T* __restrict__ q_out,
+                                                       T* __restrict__ kv_pool, KVLayout kvl, int layer,
+                                                       const float2* __restrict__ rope_cs, int rope_max_pos,
+                                                       RowState rs, SlotState ss, RowMap rm, int* err) {
+    const int row = blockIdx.x;
+    int slot, r;
+    if (!rm.live(row, slot, r)) return;
+    const int pos = rs.pos[row];
+    const int p = ss.S[slot] + r;
+    const int pidx = p / kPage, off = p % kPage;
+    if (pidx >= ss.pages_per_seq || pos < 0 || pos >= rope_max_pos) {
+        if (threadIdx.x == 0) set_error(err, kErrBounds);
+        return;
+    }
+    const int page = ss.page_table[(int64_t)slot * ss.pages_per_seq + pidx];
+    if (page < 0 || page >= kvl.num_pages) {
+        if (threadIdx.x == 0) set_error(err, kErrBounds);
+        return;
+    }
+    const int half = hd / 2;
+    const int ncols = (hq + 2 * hkv) * hd;
+    const int npairs = (hq + 2 * hkv) * half;
+    for (int pr = threadIdx.x; pr < npairs; pr += blockDim.x) {
+        const int head = pr / half, i = pr - head * half;
+        const int col = head * hd + i;
+        float a = 0.f, b = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float* w = ws + s * sstride + (int64_t)row * ncols;
+            a += w[col];
+            b += w[col + half];
+        }
+        if (head < hq + hkv) {
+            const float2 cs = rope_cs[(int64_t)pos * half + i];
+            const float a2 = a * cs.x - b * cs.y;
+            const float b2 = b * cs.x + a * cs.y;
+            a = a2;
+            b = b2;
+        }
+        if (head < hq) {
+            T* qo = q_out + (int64_t)row * hq * hd + head * hd;
+            qo[i] = from_f32<T>(a);
+            qo[i + half] = from_f32<T>(b);
+        } else {
+            const int kv = head < hq + hkv ? 0 : 1;
+            const int h = head - hq - kv * hkv;
+            T* dst = kv_pool + kvl.page_base(layer, page, kv, h) + (int64_t)off * hd;
+            dst[i] = from_f32<T>(a);
+            dst[i + half] = from_f32<T>(b);
+        }
+    }
+}
+
+// fp32 attention (exact-parity mode): one warp per (row, query head).  Row r
+// of a sequence with committed length S attends to cache positions 0..S+r
+// (the window rows before it in physical order, then itself) [Method].
+__global__ void __launch_bounds__(128) attn_f32_kernel(const float* __restrict__ q, const float* __restrict__ kv_pool,
+                                                       KVLayout kvl, int layer, int hq, int hkv, int hd,
+                                                       float* __restrict__ out, SlotState ss, RowMap rm, int* err) {
+    const int row = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int head = blockIdx.y * 4 + warp;
+    if (head >= hq) return;
+    int slot, r;
+    float* o = out + (int64_t)row * hq * hd + head * hd;
+    if (!rm.live(row, slot, r)) {
+        for (int c = lane; c < hd; c += 32) o[c] = 0.f;
+        return;
+    }
+    const int kvh = head / (hq / hkv);
+    const int T = ss.S[slot] + r + 1;
+    const float* qr = q + (int64_t)row * hq * hd + head * hd;
+    constexpr int MAXD = 4;  // head_dim <= 128
+    float qv[MAXD], acc[MAXD];
+    const int nd = hd / 32;
+#pragma unroll
+    for (int j = 0; j < MAXD; ++j) {
+        qv[j] = (j < nd) ? qr[lane + 32 * j] : 0.f;
+        acc[j] = 0.f;
+    }
+    const float scale = 1.0f / sqrtf((float)hd);
+    float m = -INFINITY, l = 0.f;
+    const int32_t* pt = ss.page_table + (int64_t)slot * ss.pages_per_seq;
+    for (int t = 0; t < T; ++t) {
+        const int pidx = t / kPage;
+        const int page = (pidx < ss.pages_per_seq) ? pt[pidx] : -1;
+        if (page < 0 || page >= kvl.num_pages) {
+            if (lane == 0) set_error(err, kErrBounds);
+            break;
+        }
+        const float* kp = kv_pool + kvl.page_base(layer, page, 0, kvh) + (int64_t)(t % kPage) * hd;
+        const float* vp = kv_pool + kvl.page_base(layer, page, 1, kvh) + (int64_t)(t % kPage) * hd;
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < MAXD; ++j)
+            if (j < nd) s = fmaf(qv[j], kp[lane + 32 * j], s);
+        s = warp_sum(s) * scale;
+        const float mn = fmaxf(m, s);
+        const float c = expf(m - mn);
+        const float pe = expf(s - mn);
+        l = l * c + pe;
+#pragma unroll
+        for (int j = 0; j < MAXD; ++j)
+            if (j < nd) acc[j] = acc[j] * c + pe * vp[lane + 32 * j];
+        m = mn;
+    }
+    const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+#pragma unroll
+    for (int j = 0; j < MAXD; ++j)
+        if (j < nd) o[lane + 32 * j] = acc[j] * inv;
+}
+
+// Residual add of the summed split-K partials, then RMSNorm with gain g:
+// x += sum_s ws[s]; h = x / rms(x) * g.
+template <typename T>
+__global__ void __launch_bounds__(256) residual_norm_kernel(const float* __restrict__ ws, int splits, int64_t sstride,
+                                                            int d, float* __restrict__ x, T* __restrict__ h,
+                                                            const float* __restrict__ g, float eps, RowMap rm) {
+    __shared__ float red[32];
+    const int row = blockIdx.x;
+    int slot, r;
+    if (!rm.live(row, slot, r)) return;
+    float* xr = x + (int64_t)row * d;
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        float v = xr[c];
+        for (int s = 0; s < splits; ++s) v += ws[s * sstride + (int64_t)row * d + c];
+        xr[c] = v;
+        ss += v * v;
+    }
+    ss = block_sum(ss, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    T* hr = h + (int64_t)row * d;
+    for (int c = threadIdx.x; c < d; c += blockDim.x) hr[c] = from_f32<T>(xr[c] * inv * g[c]);
+}
+
+// SwiGLU: act = silu(gate) * up, gate = columns [0, F), up = [F, 2F).
+template <typename T>
+__global__ void __launch_bounds__(256) swiglu_kernel(const float* __restrict__ ws, int splits, int64_t sstride, int F,
+                                                     T* __restrict__ act, RowMap rm) {
+    const int row = blockIdx.x;
+    int slot, r;
+    if (!rm.live(row, slot, r)) return;
+    for (int c = threadIdx.x; c < F; c += blockDim.x) {
+        float gv = 0.f, uv = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            const float* w = ws + s * sstride + (int64_t)row * 2 * F;
+            gv += w[c];
+            uv += w[F + c];
+        }
+        act[(int64_t)row * F + c] = from_f32<T>(gv / (1.0f + expf(-gv)) * uv);
+    }
+}
+
+__global__ void rope_table_kernel(float2* cs, int max_pos, int half, int hd, double theta) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)max_pos * half) return;
+    const int pos = (int)(idx / half), i = (int)(idx % half);
+    const double inv = pow(theta, -2.0 * (double)i / (double)hd);
+    const double ang = (double)pos * inv;
+    cs[idx] = make_float2((float)cos(ang), (float)sin(ang));
+}
+
+// ---------------------------------------------------------------------------
+// Entropy and argmax of softmax(scale * z) over ids != mask_id, as one
+// streaming pass [Method; Review, Weaknesses]: per chunk of the vocabulary a
+// running (M, s, t, amax) with M = max, s = sum e^(z-M), t = sum e^(z-M)(z-M);
+// then H = log s - t/s.  Probabilities are never stored.
+struct EntAcc {
+    float m, s, t;
+    int a;
+};
+
+__device__ __forceinline__ void ent_push(EntAcc& e, float z, int idx) {
+    if (z > e.m) {
+        if (e.s > 0.f) {
+            const float al = expf(e.m - z);
+            e.t = al * (e.t + (e.m - z) * e.s);
+            e.s = al * e.s;
+        }
+        e.s += 1.f;
+        e.m = z;
+        e.a = idx;
+    } else {
+        const float ex = expf(z - e.m);
+        e.s += ex;
+        e.t += ex * (z - e.m);
+    }
+}
+
+__device__ __forceinline__ EntAcc ent_merge(const EntAcc& x, const EntAcc& y) {
+    if (y.s == 0.f) return x;
+    if (x.s == 0.f) return y;
+    EntAcc o;
+    o.m = fmaxf(x.m, y.m);
+    const float ax = expf(x.m - o.m), ay = expf(y.m - o.m);
+    o.s = ax * x.s + ay * y.s;
+    o.t = ax * (x.t + (x.m - o.m) * x.s) + ay * (y.t + (y.m - o.m) * y.s);
+    o.a = (x.m > y.m) ? x.a : (y.m > x.m) ? y.a : min(x.a, y.a);
+    return o;
+}
+
+__device__ __forceinline__ EntAcc ent_shfl_merge(EntAcc e, int o) {
+    EntAcc y;
+    y.m = __shfl_xor_sync(0xffffffffu, e.m, o);
+    y.s = __shfl_xor_sync(0xffffffffu, e.s, o);
+    y.t = __shfl_xor_sync(0xffffffffu, e.t, o);
+    y.a = __shfl_xor_sync(0xffffffffu, e.a, o);
+    return ent_merge(e, y);
+}
+
+__global__ void __launch_bounds__(256) entropy_partial_kernel(const float* __restrict__ logits, int splits,
+                                                              int64_t sstride, int64_t ld, int V, int mask_id,
+                                                              float scale, const uint8_t* __restrict__ rowmask,
+                                                              int chunks, float4* __restrict__ part) {
+    const int row = blockIdx.y, c = blockIdx.x;
+    if (!rowmask[row]) return;
+    const int csz = ((V + chunks - 1) / chunks + 3) & ~3;
+    const int v0 = c * csz, v1 = min(V, v0 + csz);
+    EntAcc e{-INFINITY, 0.f, 0.f, INT_MAX};
+    const float* zr = logits + (int64_t)row * ld;
+    if (splits == 1 && (ld & 3) == 0) {
+        const int nvec = (v1 - v0) >> 2;
+        const float4* z4 = reinterpret_cast<const float4*>(zr + v0);
+        for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+            const float4 q = __ldg(z4 + i);
+            const int id = v0 + 4 * i;
+            if (id != mask_id) ent_push(e, scale * q.x, id);
+            if (id + 1 != mask_id) ent_push(e, scale * q.y, id + 1);
+            if (id + 2 != mask_id) ent_push(e, scale * q.z, id + 2);
+            if (id + 3 != mask_id) ent_push(e, scale * q.w, id + 3);
+        }
+        for (int id = v0 + 4 * nvec + threadIdx.x; id < v1; id += blockDim.x)
+            if (id != mask_id) ent_push(e, scale * zr[id], id);
+    } else {
+        for (int id = v0 + threadIdx.x; id < v1; id += blockDim.x) {
+            if (id == mask_id) continue;
+            float z = 0.f;
+            for (int s = 0; s < splits; ++s) z += logits[s * sstride + (int64_t)row * ld + id];
+            ent_push(e, scale * z, id);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e = ent_shfl_merge(e, o);
+    __shared__ EntAcc sh[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) sh[warp] = e;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        EntAcc t = sh[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) t = ent_merge(t, sh[w]);
+        part[(int64_t)row * chunks + c] = make_float4(t.m, t.s, t.t, __int_as_float(t.a));
+    }
+}
+
+__device__ __forceinline__ void combine_entropy(const float4* part, int chunks, int row, float& H, int& a) {
+    EntAcc e{-INFINITY, 0.f, 0.f, INT_MAX};
+    for (int c = 0; c < chunks; ++c) {
+        const float4 q = part[(int64_t)row * chunks + c];
+        EntAcc y{q.x, q.y, q.z, __float_as_int(q.w)};
+        e = ent_merge(e, y);
+    }
+    H = (e.s > 0.f) ? logf(e.s) - e.t / e.s : 0.f;
+    a = e.a;
+}
+
+// Fill decisions for one window from H~ of its masked slots (R5): every
+// masked slot with H~ < tau; if none (or tau_none) the argmin, lowest offset
+// on ties.  ht[j] is NaN for non-masked slots.
+__device__ __forceinline__ int choose_fills(const float* ht, const uint8_t* masked, int n, StepKnobs kn,
+                                            uint8_t* fill) {
+    int count = 0;
+    for (int j = 0; j < n; ++j) {
+        fill[j] = 0;
+        if (!kn.tau_none && masked[j] && ht[j] < kn.tau) {
+            fill[j] = 1;
+            ++count;
+        }
+    }
+    if (count == 0) {
+        int best = -1;
+        for (int j = 0; j < n; ++j)
+            if (masked[j] && (best < 0 || ht[j] < ht[best])) best = j;
+        if (best >= 0) {
+            fill[best] = 1;
+            count = 1;
+        }
+    }
+    return count;
+}
+
+// Selection, commit and slide for one decode step, one CTA per batch entry
+// [Method]: H~_j = H_j + lambda * j over masked slots; commit the k slots of
+// the leftmost filled run (their K/V already sit at cache positions S..S+k-1);
+// fill the chosen masks with their argmax tokens; slide the window by k.
+__global__ void __launch_bounds__(64) select_commit_kernel(const float4* __restrict__ part, int chunks, SlotState ss,
+                                                           RowState rs, int stride, StepKnobs kn, int* err) {
+    const int slot = blockIdx.x;
+    const int n = ss.n[slot];
+    __shared__ float sh[kMaxWindow];
+    __shared__ int sa[kMaxWindow];
+    __shared__ uint8_t smask[kMaxWindow];
+    __shared__ uint8_t sfill[kMaxWindow];
+    const int maxW = ss.maxW;
+    if (n == 0) {
+        if (threadIdx.x == 0) ss.out_count[slot] = 0;
+        for (int j = threadIdx.x; j < maxW; j += blockDim.x) {
+            ss.htilde[(int64_t)slot * maxW + j] = NAN;
+            ss.amax[(int64_t)slot * maxW + j] = -1;
+            ss.fillflag[(int64_t)slot * maxW + j] = 0;
+        }
+        return;
+    }
+    const int k = ss.k[slot], nf = ss.nf[slot];
+    const uint8_t* f = ss.filled + (int64_t)slot * maxW;
+    for (int j = threadIdx.x; j < kMaxWindow; j += blockDim.x) {
+        sh[j] = NAN;
+        sa[j] = -1;
+        smask[j] = (j < n && !f[j]) ? 1 : 0;
+    }
+    __syncthreads();
+    for (int r = nf + threadIdx.x; r < n; r += blockDim.x) {
+        const int row = slot * stride + r;
+        const int j = rs.perm[row];
+        float H;
+        int a;
+        combine_entropy(part, chunks, row, H, a);
+        if (j >= 0 && j < n) {
+            sh[j] = H + kn.lambda * (float)j;
+            sa[j] = a;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int nfill = choose_fills(sh, smask, n, kn, sfill);
+        int32_t* tok = ss.token + (int64_t)slot * maxW;
+        uint8_t* fl = ss.filled + (int64_t)slot * maxW;
+        const int S = ss.S[slot], P = ss.P[slot];
+        for (int j = 0; j < k; ++j) {
+            ss.out_tokens[(int64_t)slot * maxW + j] = tok[j];
+            const int gi = S - P + j;
+            if (gi >= 0 && gi < ss.gen_cap) ss.gen[(int64_t)slot * ss.gen_cap + gi] = tok[j];
+            else set_error(err, kErrBounds);
+        }
+        for (int j = 0; j < n; ++j) {
+            ss.htilde[(int64_t)slot * maxW + j] = sh[j];
+            ss.amax[(int64_t)slot * maxW + j] = sa[j];
+            ss.fillflag[(int64_t)slot * maxW + j] = sfill[j];
+            if (sfill[j]) {
+                fl[j] = 1;
+                tok[j] = sa[j];
+            }
+        }
+        for (int j = n; j < maxW; ++j) {
+            ss.htilde[(int64_t)slot * maxW + j] = NAN;
+            ss.amax[(int64_t)slot * maxW + j] = -1;
+            ss.fillflag[(int64_t)slot * maxW + j] = 0;
+        }
+        for (int j = k; j < n; ++j) {  // slide
+            fl[j - k] = fl[j];
+            tok[j - k] = tok[j];
+        }
+        ss.wlen[slot] = n - k;
+        ss.S[slot] = S + k;
+        int64_t* cnt = ss.counters + (int64_t)slot * 4;
+        cnt[0] += 1;
+        cnt[1] += n;
+        cnt[2] += k;
+        cnt[3] += nfill;
+        ss.out_count[slot] = k;
+    }
+}
+
+// Stand-alone stages (test hooks) ------------------------------------------
+__global__ void reorder_only_kernel(const uint8_t* __restrict__ filled, const int32_t* __restrict__ n,
+                                    const int32_t* __restrict__ S, int n_seq, int stride, int32_t* perm,
+                                    int32_t* pos, int32_t* kout, int32_t* nfout) {
+    const int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= n_seq) return;
+    const uint8_t* f = filled + (int64_t)b * stride;
+    const int nb = min(n[b], stride);
+    int k = 0;
+    while (k < nb && f[k]) ++k;
+    int nf = 0;
+    for (int j = 0; j < nb; ++j)
+        if (f[j]) perm[(int64_t)b * stride + nf++] = j;
+    int m = nf;
+    for (int j = 0; j < nb; ++j)
+        if (!f[j]) perm[(int64_t)b * stride + m++] = j;
+    for (int r = 0; r < stride; ++r) {
+        if (r < nb) pos[(int64_t)b * stride + r] = S[b] + perm[(int64_t)b * stride + r];
+        else {
+            perm[(int64_t)b * stride + r] = -1;
+            pos[(int64_t)b * stride + r] = -1;
+        }
+    }
+    kout[b] = k;
+    nfout[b] = nf;
+}
+
+__global__ void rowmask_kernel(const uint8_t* filled, const int32_t* n, int n_seq, int stride, uint8_t* rowmask) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n_seq * stride) return;
+    const int b = i / stride, j = i % stride;
+    rowmask[i] = (j < n[b] && !filled[i]) ? 1 : 0;
+}
+
+__global__ void __launch_bounds__(64) select_only_kernel(const float4* __restrict__ part, int chunks,
+                                                         const uint8_t* __restrict__ filled, const int32_t* __restrict__ n,
+                                                         int stride, StepKnobs kn, float* htilde, int32_t* amax,
+                                                         uint8_t* fill) {
+    const int b = blockIdx.x;
+    const int nb = min(n[b], min(stride, kMaxWindow));
+    __shared__ float sh[kMaxWindow];
+    __shared__ uint8_t smask[kMaxWindow];
+    __shared__ uint8_t sfill[kMaxWindow];
+    __shared__ int sa[kMaxWindow];
+    for (int j = threadIdx.x; j < kMaxWindow; j += blockDim.x) {
+        const bool m = j < nb && !filled[(int64_t)b * stride + j];
+        smask[j] = m ? 1 : 0;
+        sh[j] = NAN;
+        sa[j] = -1;
+        if (m) {
+            float H;
+            int a;
+            combine_entropy(part, chunks, b * stride + j, H, a);
+            sh[j] = H + kn.lambda * (float)j;
+            sa[j] = a;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) choose_fills(sh, smask, nb, kn, sfill);
+    __syncthreads();
+    for (int j = threadIdx.x; j < stride; j += blockDim.x) {
+        const bool in = j < kMaxWindow;
+        htilde[(int64_t)b * stride + j] = in ? sh[j] : NAN;
+        amax[(int64_t)b * stride + j] = in ? sa[j] : -1;
+        fill[(int64_t)b * stride + j] = in ? sfill[j] : 0;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host launch wrappers.
+template <typename T>
+void launch_decode_prepare(const T* embed, const float* g, float eps, int d, int mask_id, SlotState ss, RowState rs,
+                           uint8_t* rowmask, int n_entries, int stride, float* x, T* h, cudaStream_t st) {
+    decode_prepare_kernel<T><<<n_entries, 256, 0, st>>>(embed, g, eps, d, mask_id, ss, rs, rowmask, stride, x, h);
+}
+
+template <typename T>
+void launch_prefill_prepare(const T* embed, const float* g, float eps, int d, const int32_t* ids, int slot, int S0,
+                            int n, SlotState ss, RowState rs, float* x, T* h, cudaStream_t st) {
+    const int grid = n < 592 ? n : 592;
+    prefill_prepare_kernel<T><<<grid > 0 ? grid : 1, 256, 0, st>>>(embed, g, eps, d, ids, slot, S0, n, ss, rs, x, h);
+}
+
+void launch_slot_admit(SlotState ss, int slot, int P, int end, int W, cudaStream_t st) {
+    slot_admit_kernel<<<1, 1, 0, st>>>(ss, slot, P, end, W);
+}
+
+void launch_prefill_finish(SlotState ss, int slot, int P, cudaStream_t st) {
+    prefill_finish_kernel<<<1, 1, 0, st>>>(ss, slot, P);
+}
+
+void launch_gemm_f32(const float* X, const float* W, float* C, int M, int N, int K, cudaStream_t st) {
+    dim3 grid((N + 63) / 64, (M + 63) / 64);
+    gemm_f32_kernel<<<grid, 256, 0, st>>>(X, W, C, M, N, K);
+}
+
+template <typename T>
+void launch_qkv_rope(const float* ws, int splits, int64_t sstride, int M, int hq, int hkv, int hd, T* q_out,
+                     T* kv_pool, KVLayout kvl, int layer, const float2* rope_cs, int rope_max_pos, RowState rs,
+                     SlotState ss, RowMap rm, int* err, cudaStream_t st) {
+    qkv_rope_kernel<T><<<M, 256, 0, st>>>(ws, splits, sstride, hq, hkv, hd, q_out, kv_pool, kvl, layer, rope_cs,
+                                          rope_max_pos, rs, ss, rm, err);
+}
+
+void launch_attn_f32(const float* q, const float* kv_pool, KVLayout kvl, int layer, int hq, int hkv, int hd,
+                     float* out, int M, SlotState ss, RowMap rm, int* err, cudaStream_t st) {
+    dim3 grid(M, (hq + 3) / 4);
+    attn_f32_kernel<<<grid, 128, 0, st>>>(q, kv_pool, kvl, layer, hq, hkv, hd, out, ss, rm, err);
+}
+
+template <typename T>
+void launch_residual_norm(const float* ws, int splits, int64_t sstride, int M, int d, float* x, T* h, const float* g,
+                          float eps, RowMap rm, cudaStream_t st) {
+    residual_norm_kernel<T><<<M, 256, 0, st>>>(ws, splits, sstride, d, x, h, g, eps, rm);
+}
+
+template <typename T>
+void launch_swiglu(const float* ws, int splits, int64_t sstride, int M, int F, T* act, RowMap rm, cudaStream_t st) {
+    swiglu_kernel<T><<<M, 256, 0, st>>>(ws, splits, sstride, F, act, rm);
+}
+
+void launch_rope_table(float2* cs, int max_pos, int half, int hd, double theta, cudaStream_t st) {
+    const int64_t n = (int64_t)max_pos * half;
+    rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(cs, max_pos, half, hd, theta);
+}
+
+void launch_entropy_partials(const float* logits, int splits, int64_t sstride, int64_t ld, int V, int mask_id,
+                             float scale, const uint8_t* rowmask, int rows, int chunks, float4* part, cudaStream_t st) {
+    dim3 grid(chunks, rows);
+    entropy_partial_kernel<<<grid, 256, 0, st>>>(logits, splits, sstride, ld, V, mask_id, scale, rowmask, chunks, part);
+}
+
+void launch_select_commit(const float4* part, int chunks, SlotState ss, RowState rs, int n_entries, int stride,
+                          StepKnobs kn, int* err, cudaStream_t st) {
+    select_commit_kernel<<<n_entries, 64, 0, st>>>(part, chunks, ss, rs, stride, kn, err);
+}
+
+void launch_reorder_only(const uint8_t* filled, const int32_t* n, const int32_t* S, int n_seq, int stride,
+                         int32_t* perm, int32_t* pos, int32_t* k, int32_t* nf, cudaStream_t st) {
+    reorder_only_kernel<<<(n_seq + 63) / 64, 64, 0, st>>>(filled, n, S, n_seq, stride, perm, pos, k, nf);
+}
+
+void launch_select_only(const float4* part, int chunks, const uint8_t* filled, const int32_t* n, int n_seq,
+                        int stride, StepKnobs kn, float* htilde, int32_t* argmax, uint8_t* fill, cudaStream_t st) {
+    select_only_kernel<<<n_seq, 64, 0, st>>>(part, chunks, filled, n, stride, kn, htilde, argmax, fill);
+}
+
+void launch_rowmask_from_filled(const uint8_t* filled, const int32_t* n, int n_seq, int stride, uint8_t* rowmask,
+                                cudaStream_t st) {
+    const int tot = n_seq * stride;
+    rowmask_kernel<<<(tot + 255) / 256, 256, 0, st>>>(filled, n, n_seq, stride, rowmask);
+}
+
+// Explicit instantiations.
+#define WEDLM_INST(T)                                                                                             \
+    template void launch_decode_prepare<T>(const T*, const float*, float, int, int, SlotState, RowState, uint8_t*, \
+                                           int, int, float*, T*, cudaStream_t);                                   \
+    template void launch_prefill_prepare<T>(const T*, const float*, float, int, const int32_t*, int, int, int,     \
+                                            SlotState, RowState, float*, T*, cudaStream_t);                       \
+    template void launch_qkv_rope<T>(const float*, int, int64_t, int, int, int, int, T*, T*, KVLayout, int,        \
+                                     const float2*, int, RowState, SlotState, RowMap, int*, cudaStream_t);        \
+    template void launch_residual_norm<T>(const float*, int, int64_t, int, int, float*, T*, const float*, float,  \
+                                          RowMap, cudaStream_t);                                                  \
+    template void launch_swiglu<T>(const float*, int, int64_t, int, int, T*, RowMap, cudaStream_t);
+WEDLM_INST(float)
+WEDLM_INST(bf16)
+#undef WEDLM_INST
+
+}  // namespace wedlm

@@ -1,0 +1,89 @@
+// Kernel launch interface of libwedlm (host-callable wrappers).
+#pragma once
+
+#include "common.cuh"
+
+namespace wedlm {
+
+// Which rows of a forward belong to which slot: row = entry * stride + r,
+// slot = slot_base + entry, row is live iff r < n[slot].
+struct RowMap {
+    int slot_base;
+    int stride;
+    const int32_t* n;
+    __device__ __forceinline__ bool live(int row, int& slot, int& r) const {
+        const int e = row / stride;
+        r = row - e * stride;
+        slot = slot_base + e;
+        return r < n[slot];
+    }
+};
+
+struct StepKnobs {
+    float lambda, tau, logit_scale;
+    int tau_none;
+};
+
+// Window prepare for a decode step: refill, reorder, embed, first RMSNorm.
+template <typename T>
+void launch_decode_prepare(const T* embed, const float* norm_g, float eps, int d, int mask_id,
+                           SlotState ss, RowState rs, uint8_t* rowmask, int n_entries, int stride,
+                           float* x, T* h, cudaStream_t st);
+// Prefill rows: tokens from `ids` (device), logical positions S0 + r.
+template <typename T>
+void launch_prefill_prepare(const T* embed, const float* norm_g, float eps, int d, const int32_t* ids,
+                            int slot, int S0, int n, SlotState ss, RowState rs, float* x, T* h,
+                            cudaStream_t st);
+void launch_slot_admit(SlotState ss, int slot, int P, int end, int W, cudaStream_t st);
+void launch_prefill_finish(SlotState ss, int slot, int P, cudaStream_t st);
+
+// fp32 SIMT GEMM: C[M][N] = X[M][K] * W[N][K]^T.
+void launch_gemm_f32(const float* X, const float* W, float* C, int M, int N, int K, cudaStream_t st);
+
+template <typename T>
+void launch_qkv_rope(const float* ws, int splits, int64_t split_stride, int M, int hq, int hkv, int hd,
+                     T* q_out, T* kv_pool, KVLayout kvl, int layer, const float2* rope_cs, int rope_max_pos,
+                     RowState rs, SlotState ss, RowMap rm, int* err, cudaStream_t st);
+
+void launch_attn_f32(const float* q, const float* kv_pool, KVLayout kvl, int layer, int hq, int hkv, int hd,
+                     float* out, int M, SlotState ss, RowMap rm, int* err, cudaStream_t st);
+
+template <typename T>
+void launch_residual_norm(const float* ws, int splits, int64_t split_stride, int M, int d, float* x, T* h,
+                          const float* g, float eps, RowMap rm, cudaStream_t st);
+
+template <typename T>
+void launch_swiglu(const float* ws, int splits, int64_t split_stride, int M, int F, T* act, RowMap rm,
+                   cudaStream_t st);
+
+void launch_rope_table(float2* cs, int max_pos, int half, int hd, double theta, cudaStream_t st);
+
+// Entropy / argmax partials over vocabulary chunks for rows with rowmask[row] != 0.
+void launch_entropy_partials(const float* logits, int splits, int64_t split_stride, int64_t ld, int V,
+                             int mask_id, float scale, const uint8_t* rowmask, int rows, int chunks,
+                             float4* part, cudaStream_t st);
+
+void launch_select_commit(const float4* part, int chunks, SlotState ss, RowState rs, int n_entries,
+                          int stride, StepKnobs knobs, int* err, cudaStream_t st);
+
+void launch_reorder_only(const uint8_t* filled, const int32_t* n, const int32_t* S, int n_seq, int stride,
+                         int32_t* perm, int32_t* pos, int32_t* k, int32_t* nf, cudaStream_t st);
+
+void launch_select_only(const float4* part, int chunks, const uint8_t* filled, const int32_t* n, int n_seq,
+                        int stride, StepKnobs knobs, float* htilde, int32_t* argmax, uint8_t* fill,
+                        cudaStream_t st);
+
+void launch_rowmask_from_filled(const uint8_t* filled, const int32_t* n, int n_seq, int stride,
+                                uint8_t* rowmask, cudaStream_t st);
+
+// bf16 tensor-core paths (gemm_tc.cu, attn_mma.cu).
+struct TmaDesc;
+void launch_attn_bf16(const bf16* q, const bf16* kv_pool, KVLayout kvl, int layer, int hq, int hkv, int hd,
+                      bf16* out, float* part_o, float2* part_ml, int n_entries, int stride, int kv_chunk,
+                      int max_splits, SlotState ss, RowMap rm, int* err, cudaStream_t st);
+void launch_attn_combine(const float* part_o, const float2* part_ml, bf16* out, int M, int hq, int hd,
+                         int kv_chunk, int max_splits, int rows_per_tile, SlotState ss, RowMap rm,
+                         cudaStream_t st);
+int attn_rows_per_tile(int group);
+
+}  // namespace wedlm

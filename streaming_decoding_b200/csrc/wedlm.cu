@@ -1,0 +1,958 @@
+// libwedlm: context, weights, prefill and the Streaming Parallel Decoding step
+// behind the C ABI declared in include/wedlm.h.
+//
+// One decode step (hyper.ai summary of arXiv 2512.22737, section "Method") is
+// a fixed sequence of kernel launches on the context's stream:
+//   decode_prepare      refill + topological reorder + embed + RMSNorm
+//   per layer (x L):    QKV GEMM -> qkv_rope (RoPE at logical positions,
+//                       K/V into the paged cache) -> attention (+ combine)
+//                       -> O GEMM -> residual+RMSNorm -> gate/up GEMM
+//                       -> SwiGLU -> down GEMM -> residual+RMSNorm
+//   LM-head GEMM        (all window rows; only masked rows are read)
+//   entropy_partials    online (max, sum e, sum e*z, argmax) per vocab chunk
+//   select_commit       H~ = H + lambda*j, threshold/argmin fills, commit run,
+//                       slide
+// followed by one device->host copy of the per-slot results.  Every size a
+// kernel needs per step lives in device memory, so a step is replayable
+// without host involvement.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <deque>
+#include <string>
+#include <vector>
+
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+using namespace wedlm;
+
+namespace {
+
+constexpr int kEntropyChunks = 16;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Arena {
+    // One cudaMalloc carved into 256-byte aligned pieces.
+    char* base = nullptr;
+    size_t size = 0, used = 0;
+    std::vector<std::pair<void**, size_t>> plan;
+    void add(void** p, size_t bytes) { plan.emplace_back(p, align_up(bytes ? bytes : 1, 256)); }
+    cudaError_t commit() {
+        size = 0;
+        for (auto& e : plan) size += e.second;
+        cudaError_t err = cudaMalloc(&base, size);
+        if (err != cudaSuccess) return err;
+        size_t off = 0;
+        for (auto& e : plan) {
+            *e.first = base + off;
+            off += e.second;
+        }
+        return cudaMemsetAsync(base, 0, size, 0);
+    }
+    void release() {
+        if (base) cudaFree(base);
+        base = nullptr;
+    }
+};
+
+}  // namespace
+
+struct wedlm_ctx {
+    wedlm_model_cfg cfg{};
+    int device = 0;
+    int num_sms = 148;
+    cudaStream_t stream = nullptr;
+    bool bf16 = false;
+    size_t elt = 4;
+    std::string last_error;
+    int64_t launches = 0;
+
+    int L, d, hq, hkv, hd, F, V, Nqkv;
+    int maxB, maxW, max_ctx, num_pages, pages_per_seq, chunk;
+    int Mdec, Mmax;
+
+    Arena weights_arena, state_arena, scratch_arena;
+    // weights
+    void* embed = nullptr;
+    void* lm_head = nullptr;
+    float* final_norm = nullptr;
+    std::vector<float*> attn_norm, ffn_norm;
+    std::vector<void*> wqkv, wo, wgu, wd;
+    std::vector<uint8_t> loaded;  // per tensor slot
+    bool weights_ready = false;
+    // bf16 tensor maps of the weights (box 128 rows)
+    std::vector<CUtensorMap> tm_qkv, tm_o, tm_gu, tm_d;
+    CUtensorMap tm_lm{};
+    bool maps_ready = false;
+    // KV pool
+    void* kv_pool = nullptr;
+    KVLayout kvl{};
+    float2* rope_cs = nullptr;
+    // slot state (device)
+    SlotState ss{};
+    RowState rs{};
+    uint8_t* rowmask = nullptr;
+    int* err = nullptr;
+    // scratch
+    float* x = nullptr;
+    void* h = nullptr;
+    void* q = nullptr;
+    void* attn_out = nullptr;
+    void* act = nullptr;
+    float* ws = nullptr;
+    size_t ws_floats = 0;
+    float* logits = nullptr;
+    size_t logits_floats = 0;
+    float4* ent_part = nullptr;
+    float* attn_po = nullptr;
+    float2* attn_pml = nullptr;
+    int attn_kv_chunk = 1 << 30, attn_max_splits = 1;
+    int32_t* ids_dev = nullptr;
+    // step results block for one device->host copy: counts[B], S[B], tokens[B][maxW], err
+    int32_t* res_dev = nullptr;
+    int32_t* res_host = nullptr;  // pinned
+    // activation tensor maps keyed by (buffer, rows, cols, box)
+    struct XMap {
+        const void* p;
+        uint64_t rows, cols;
+        uint32_t box;
+        CUtensorMap tm;
+    };
+    std::deque<XMap> xmaps;
+    // host mirrors
+    std::vector<int> h_W, h_S, h_end, h_P;
+    std::vector<std::vector<int>> h_pages;
+    std::vector<int> free_pages;
+    int last_stride = 0;
+    int logits_splits_last = 1;
+    int last_M = 0;
+};
+
+namespace {
+
+wedlm_status fail(wedlm_ctx* c, wedlm_status s, const std::string& msg) {
+    if (c) c->last_error = msg;
+    return s;
+}
+
+#define CK(call)                                                                                  \
+    do {                                                                                          \
+        cudaError_t e_ = (call);                                                                  \
+        if (e_ != cudaSuccess)                                                                    \
+            return fail(ctx, WEDLM_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+    } while (0)
+
+int tensor_slot(const wedlm_ctx* c, int tensor, int layer) {
+    switch (tensor) {
+        case WEDLM_T_EMBED: return 0;
+        case WEDLM_T_LM_HEAD: return 1;
+        case WEDLM_T_FINAL_NORM: return 2;
+        default: break;
+    }
+    if (tensor < WEDLM_T_ATTN_NORM || tensor > WEDLM_T_WD || layer < 0 || layer >= c->L) return -1;
+    return 3 + layer * 9 + (tensor - WEDLM_T_ATTN_NORM);
+}
+
+const CUtensorMap* xmap(wedlm_ctx* c, const void* p, uint64_t rows, uint64_t cols, uint32_t box) {
+    for (auto& m : c->xmaps)
+        if (m.p == p && m.rows == rows && m.cols == cols && m.box == box) return &m.tm;
+    wedlm_ctx::XMap m{p, rows, cols, box, {}};
+    if (!make_tmap_bf16(&m.tm, p, rows, cols, box)) return nullptr;
+    c->xmaps.push_back(m);
+    return &c->xmaps.back().tm;
+}
+
+// Y[M][N] (fp32 partial planes in ws or `out`) = X[M][K] * W[N][K]^T.
+wedlm_status gemm(wedlm_ctx* ctx, const void* X, const void* W, const CUtensorMap* tmW, int M, int N, int K,
+                  float* out, size_t out_cap_floats, int* splits_out, int max_splits = 32) {
+    if (!ctx->bf16) {
+        if ((size_t)M * N > out_cap_floats) return fail(ctx, WEDLM_ERR_STATE, "gemm workspace too small");
+        launch_gemm_f32((const float*)X, (const float*)W, out, M, N, K, ctx->stream);
+        ctx->launches++;
+        *splits_out = 1;
+        return WEDLM_OK;
+    }
+    GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms);
+    // cap the K splits by the caller's limit and by the partial-plane capacity
+    const size_t plane = (size_t)M * N;
+    const int cap = (int)std::min<size_t>((size_t)max_splits, out_cap_floats / plane);
+    if (cap < 1) return fail(ctx, WEDLM_ERR_STATE, "gemm workspace too small");
+    if (p.splits > cap) {
+        const int KB = (K + 63) / 64;
+        p.kb_per_split = (KB + cap - 1) / cap;
+        p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;
+    }
+    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
+    if (!tx) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for activations");
+    cudaError_t e = launch_gemm_bf16(*tmW, *tx, out, M, N, K, p, ctx->err, ctx->stream);
+    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("gemm launch: ") + cudaGetErrorString(e));
+    ctx->launches++;
+    *splits_out = p.splits;
+    return WEDLM_OK;
+}
+
+size_t gemm_ws_need(const wedlm_ctx* c, int M, int N, int K) {
+    if (!c->bf16) return (size_t)M * N;
+    GemmPlan p = plan_gemm_bf16(M, N, K, c->num_sms);
+    return (size_t)p.splits * M * N;
+}
+
+wedlm_status build_weight_maps(wedlm_ctx* ctx) {
+    if (!ctx->bf16 || ctx->maps_ready) return WEDLM_OK;
+    ctx->tm_qkv.resize(ctx->L);
+    ctx->tm_o.resize(ctx->L);
+    ctx->tm_gu.resize(ctx->L);
+    ctx->tm_d.resize(ctx->L);
+    bool ok = true;
+    for (int l = 0; l < ctx->L; ++l) {
+        ok &= make_tmap_bf16(&ctx->tm_qkv[l], ctx->wqkv[l], ctx->Nqkv, ctx->d, 128);
+        ok &= make_tmap_bf16(&ctx->tm_o[l], ctx->wo[l], ctx->d, (uint64_t)ctx->hq * ctx->hd, 128);
+        ok &= make_tmap_bf16(&ctx->tm_gu[l], ctx->wgu[l], 2 * (uint64_t)ctx->F, ctx->d, 128);
+        ok &= make_tmap_bf16(&ctx->tm_d[l], ctx->wd[l], ctx->d, ctx->F, 128);
+    }
+    ok &= make_tmap_bf16(&ctx->tm_lm, ctx->lm_head, ctx->V, ctx->d, 128);
+    if (!ok) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for weights");
+    ctx->maps_ready = true;
+    return WEDLM_OK;
+}
+
+wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
+    if (code == 0) return WEDLM_OK;
+    CK(cudaMemsetAsync(ctx->err, 0, sizeof(int), ctx->stream));
+    if (code == kErrTimeout) return fail(ctx, WEDLM_ERR_TIMEOUT, "a bounded device wait timed out");
+    return fail(ctx, WEDLM_ERR_DEVICE_ASSERT, "a device bounds check fired");
+}
+
+// The transformer stack over rows [entry * stride + r] of slots slot_base +
+// entry.  On entry x holds the embeddings and h the first RMSNorm; on exit h
+// holds the final-normed hidden states.
+template <typename T>
+wedlm_status forward_layers(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
+    const int M = n_entries * stride;
+    RowMap rm{slot_base, stride, ctx->ss.n};
+    const float eps = ctx->cfg.rms_eps;
+    T* h = (T*)ctx->h;
+    T* qb = (T*)ctx->q;
+    T* ao = (T*)ctx->attn_out;
+    T* act = (T*)ctx->act;
+    const int rt = ctx->bf16 ? attn_rows_per_tile(ctx->hq / ctx->hkv) : 1;
+    for (int l = 0; l < ctx->L; ++l) {
+        int sp = 1;
+        wedlm_status s;
+        s = gemm(ctx, h, ctx->wqkv[l], ctx->bf16 ? &ctx->tm_qkv[l] : nullptr, M, ctx->Nqkv, ctx->d, ctx->ws,
+                 ctx->ws_floats, &sp);
+        if (s) return s;
+        launch_qkv_rope<T>(ctx->ws, sp, (int64_t)M * ctx->Nqkv, M, ctx->hq, ctx->hkv, ctx->hd, qb, (T*)ctx->kv_pool,
+                           ctx->kvl, l, ctx->rope_cs, ctx->max_ctx, ctx->rs, ctx->ss, rm, ctx->err, ctx->stream);
+        ctx->launches++;
+        if (ctx->bf16) {
+            const int kc = decode ? ctx->attn_kv_chunk : (1 << 30);
+            const int ms = decode ? ctx->attn_max_splits : 1;
+            launch_attn_bf16((const bf16*)qb, (const bf16*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd,
+                             (bf16*)ao, ctx->attn_po, ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss, rm, ctx->err,
+                             ctx->stream);
+            ctx->launches++;
+            if (ms > 1) {
+                launch_attn_combine(ctx->attn_po, ctx->attn_pml, (bf16*)ao, M, ctx->hq, ctx->hd, kc, ms, rt, ctx->ss,
+                                    rm, ctx->stream);
+                ctx->launches++;
+            }
+        } else {
+            launch_attn_f32((const float*)qb, (const float*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd,
+                            (float*)ao, M, ctx->ss, rm, ctx->err, ctx->stream);
+            ctx->launches++;
+        }
+        s = gemm(ctx, ao, ctx->wo[l], ctx->bf16 ? &ctx->tm_o[l] : nullptr, M, ctx->d, ctx->hq * ctx->hd, ctx->ws,
+                 ctx->ws_floats, &sp);
+        if (s) return s;
+        launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, ctx->ffn_norm[l], eps, rm,
+                                ctx->stream);
+        ctx->launches++;
+        s = gemm(ctx, h, ctx->wgu[l], ctx->bf16 ? &ctx->tm_gu[l] : nullptr, M, 2 * ctx->F, ctx->d, ctx->ws,
+                 ctx->ws_floats, &sp);
+        if (s) return s;
+        launch_swiglu<T>(ctx->ws, sp, (int64_t)M * 2 * ctx->F, M, ctx->F, act, rm, ctx->stream);
+        ctx->launches++;
+        s = gemm(ctx, act, ctx->wd[l], ctx->bf16 ? &ctx->tm_d[l] : nullptr, M, ctx->d, ctx->F, ctx->ws,
+                 ctx->ws_floats, &sp);
+        if (s) return s;
+        const float* gnext = (l + 1 < ctx->L) ? ctx->attn_norm[l + 1] : ctx->final_norm;
+        launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, gnext, eps, rm, ctx->stream);
+        ctx->launches++;
+    }
+    return WEDLM_OK;
+}
+
+wedlm_status run_forward(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
+    return ctx->bf16 ? forward_layers<bf16>(ctx, slot_base, n_entries, stride, decode)
+                     : forward_layers<float>(ctx, slot_base, n_entries, stride, decode);
+}
+
+int max_active_window(const wedlm_ctx* c, int* n_entries) {
+    int w = 0, last = -1;
+    for (int b = 0; b < c->maxB; ++b)
+        if (c->h_W[b] > 0 && c->h_S[b] < c->h_end[b]) {
+            w = std::max(w, c->h_W[b]);
+            last = b;
+        }
+    *n_entries = last + 1;
+    return w;
+}
+
+// Enqueue one decode step over slots [0, n_entries) with row stride `stride`.
+wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_entries, int stride) {
+    const int M = n_entries * stride;
+    if (ctx->bf16)
+        launch_decode_prepare<bf16>((const bf16*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
+                                    ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
+                                    (bf16*)ctx->h, ctx->stream);
+    else
+        launch_decode_prepare<float>((const float*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
+                                     ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
+                                     (float*)ctx->h, ctx->stream);
+    ctx->launches++;
+    wedlm_status s = run_forward(ctx, 0, n_entries, stride, true);
+    if (s) return s;
+    int lsp = 1;
+    s = gemm(ctx, ctx->h, ctx->lm_head, ctx->bf16 ? &ctx->tm_lm : nullptr, M, ctx->V, ctx->d, ctx->logits,
+             ctx->logits_floats, &lsp, 4);
+    if (s) return s;
+    launch_entropy_partials(ctx->logits, lsp, (int64_t)M * ctx->V, ctx->V, ctx->V, ctx->cfg.mask_id, prm->logit_scale,
+                            ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream);
+    ctx->launches++;
+    StepKnobs kn{prm->lambda, prm->tau, prm->logit_scale, prm->tau_none};
+    launch_select_commit(ctx->ent_part, kEntropyChunks, ctx->ss, ctx->rs, n_entries, stride, kn, ctx->err,
+                         ctx->stream);
+    ctx->launches++;
+    ctx->last_stride = stride;
+    ctx->last_M = M;
+    ctx->logits_splits_last = lsp;
+    return WEDLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wedlm_status_str(wedlm_status s) {
+    switch (s) {
+        case WEDLM_OK: return "ok";
+        case WEDLM_ERR_INVALID_ARG: return "invalid argument";
+        case WEDLM_ERR_OOM_PAGES: return "KV page pool exhausted";
+        case WEDLM_ERR_OOM_DEVICE: return "device out of memory";
+        case WEDLM_ERR_CUDA: return "CUDA error";
+        case WEDLM_ERR_DEVICE_ASSERT: return "device bounds check fired";
+        case WEDLM_ERR_STATE: return "invalid state for this call";
+        case WEDLM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case WEDLM_ERR_TIMEOUT: return "bounded device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char* wedlm_last_error(const wedlm_ctx* ctx) { return ctx ? ctx->last_error.c_str() : ""; }
+
+}  // extern "C"
+
+// ===========================================================================
+// Context lifetime, weights, sequences, decode step.
+namespace {
+
+bool valid_cfg(const wedlm_model_cfg* c, std::string* why) {
+    auto bad = [&](const char* m) {
+        *why = m;
+        return false;
+    };
+    if (c->n_layers <= 0 || c->d_model <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+        c->ffn_dim <= 0 || c->vocab <= 1)
+        return bad("model dimensions must be positive");
+    if (c->n_heads % c->n_kv_heads) return bad("n_heads must be a multiple of n_kv_heads");
+    if (c->head_dim % 2) return bad("head_dim must be even");
+    if (c->mask_id < 0 || c->mask_id >= c->vocab) return bad("mask_id out of range");
+    if (!(c->rope_theta > 0.0) || !(c->rms_eps >= 0.f)) return bad("rope_theta must be > 0 and rms_eps >= 0");
+    if (c->max_batch <= 0 || c->max_batch > 4096) return bad("max_batch must be in [1, 4096]");
+    if (c->max_window <= 0 || c->max_window > kMaxWindow) return bad("max_window must be in [1, 64]");
+    if (c->max_ctx <= 0) return bad("max_ctx must be positive");
+    if (c->num_pages < 0 || c->prefill_chunk < 0) return bad("num_pages / prefill_chunk must be >= 0");
+    if (c->dtype == WEDLM_DTYPE_F32) {
+        if (c->head_dim % 32 || c->head_dim > 128) return bad("fp32 mode needs head_dim a multiple of 32, <= 128");
+    } else if (c->dtype == WEDLM_DTYPE_BF16) {
+        if (c->head_dim != 128) return bad("bf16 mode needs head_dim 128");
+        if (c->d_model % 8 || c->ffn_dim % 8) return bad("bf16 mode needs d_model and ffn_dim multiples of 8");
+    } else {
+        return bad("unknown dtype");
+    }
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_ctx** out_ctx) {
+    if (!cfg || !out_ctx) return WEDLM_ERR_INVALID_ARG;
+    *out_ctx = nullptr;
+    std::string why;
+    if (!valid_cfg(cfg, &why)) return WEDLM_ERR_INVALID_ARG;
+    wedlm_ctx* ctx = new wedlm_ctx();
+    ctx->cfg = *cfg;
+    ctx->stream = (cudaStream_t)cuda_stream;
+    ctx->bf16 = cfg->dtype == WEDLM_DTYPE_BF16;
+    ctx->elt = ctx->bf16 ? 2 : 4;
+    auto bail = [&](wedlm_status s) {
+        ctx->weights_arena.release();
+        ctx->state_arena.release();
+        ctx->scratch_arena.release();
+        if (ctx->res_host) cudaFreeHost(ctx->res_host);
+        delete ctx;
+        return s;
+    };
+    if (cudaGetDevice(&ctx->device) != cudaSuccess) return bail(WEDLM_ERR_CUDA);
+    cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
+    ctx->L = cfg->n_layers;
+    ctx->d = cfg->d_model;
+    ctx->hq = cfg->n_heads;
+    ctx->hkv = cfg->n_kv_heads;
+    ctx->hd = cfg->head_dim;
+    ctx->F = cfg->ffn_dim;
+    ctx->V = cfg->vocab;
+    ctx->Nqkv = (ctx->hq + 2 * ctx->hkv) * ctx->hd;
+    ctx->maxB = cfg->max_batch;
+    ctx->maxW = cfg->max_window;
+    ctx->max_ctx = cfg->max_ctx;
+    ctx->pages_per_seq = (cfg->max_ctx + kPage - 1) / kPage;
+    ctx->num_pages = cfg->num_pages ? cfg->num_pages : ctx->maxB * ctx->pages_per_seq;
+    ctx->chunk = cfg->prefill_chunk ? cfg->prefill_chunk : 1024;
+    ctx->Mdec = ctx->maxB * ctx->maxW;
+    ctx->Mmax = std::max(ctx->Mdec, ctx->chunk);
+    const size_t elt = ctx->elt;
+    const int L = ctx->L, d = ctx->d, F = ctx->F, V = ctx->V;
+    const int B = ctx->maxB, maxW = ctx->maxW, Mmax = ctx->Mmax;
+
+    // Weights.
+    Arena& wa = ctx->weights_arena;
+    ctx->attn_norm.assign(L, nullptr);
+    ctx->ffn_norm.assign(L, nullptr);
+    ctx->wqkv.assign(L, nullptr);
+    ctx->wo.assign(L, nullptr);
+    ctx->wgu.assign(L, nullptr);
+    ctx->wd.assign(L, nullptr);
+    wa.add(&ctx->embed, (size_t)V * d * elt);
+    wa.add(&ctx->lm_head, (size_t)V * d * elt);
+    wa.add((void**)&ctx->final_norm, (size_t)d * 4);
+    for (int l = 0; l < L; ++l) {
+        wa.add((void**)&ctx->attn_norm[l], (size_t)d * 4);
+        wa.add((void**)&ctx->ffn_norm[l], (size_t)d * 4);
+        wa.add(&ctx->wqkv[l], (size_t)ctx->Nqkv * d * elt);
+        wa.add(&ctx->wo[l], (size_t)d * ctx->hq * ctx->hd * elt);
+        wa.add(&ctx->wgu[l], (size_t)2 * F * d * elt);
+        wa.add(&ctx->wd[l], (size_t)d * F * elt);
+    }
+    if (wa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+    ctx->loaded.assign(3 + 9 * L, 0);
+
+    // KV pool, rope table, slot and row state, step-result block.
+    const int64_t page_elems = (int64_t)2 * ctx->hkv * kPage * ctx->hd;
+    ctx->kvl.layer_stride = (int64_t)ctx->num_pages * page_elems;
+    ctx->kvl.hkv = ctx->hkv;
+    ctx->kvl.hd = ctx->hd;
+    ctx->kvl.num_pages = ctx->num_pages;
+    Arena& sa = ctx->state_arena;
+    sa.add(&ctx->kv_pool, (size_t)L * ctx->kvl.layer_stride * elt);
+    sa.add((void**)&ctx->rope_cs, (size_t)ctx->max_ctx * (ctx->hd / 2) * sizeof(float2));
+    SlotState& ss = ctx->ss;
+    const size_t res_ints = (size_t)2 * B + (size_t)B * maxW + 1;
+    sa.add((void**)&ctx->res_dev, res_ints * 4);
+    sa.add((void**)&ss.end, B * 4);
+    sa.add((void**)&ss.P, B * 4);
+    sa.add((void**)&ss.W, B * 4);
+    sa.add((void**)&ss.wlen, B * 4);
+    sa.add((void**)&ss.n, B * 4);
+    sa.add((void**)&ss.k, B * 4);
+    sa.add((void**)&ss.nf, B * 4);
+    sa.add((void**)&ss.filled, (size_t)B * maxW);
+    sa.add((void**)&ss.token, (size_t)B * maxW * 4);
+    sa.add((void**)&ss.page_table, (size_t)B * ctx->pages_per_seq * 4);
+    sa.add((void**)&ss.counters, (size_t)B * 4 * 8);
+    sa.add((void**)&ss.gen, (size_t)B * ctx->max_ctx * 4);
+    sa.add((void**)&ss.htilde, (size_t)B * maxW * 4);
+    sa.add((void**)&ss.amax, (size_t)B * maxW * 4);
+    sa.add((void**)&ss.fillflag, (size_t)B * maxW);
+    sa.add((void**)&ctx->rs.pos, (size_t)Mmax * 4);
+    sa.add((void**)&ctx->rs.tok, (size_t)Mmax * 4);
+    sa.add((void**)&ctx->rs.perm, (size_t)Mmax * 4);
+    sa.add((void**)&ctx->rowmask, (size_t)Mmax);
+    sa.add((void**)&ctx->ids_dev, (size_t)ctx->chunk * 4);
+    if (sa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+    ss.out_count = ctx->res_dev;
+    ss.S = ctx->res_dev + B;
+    ss.out_tokens = ctx->res_dev + 2 * B;
+    ctx->err = ctx->res_dev + 2 * B + (size_t)B * maxW;
+    ss.pages_per_seq = ctx->pages_per_seq;
+    ss.maxW = maxW;
+    ss.gen_cap = ctx->max_ctx;
+    if (cudaMallocHost((void**)&ctx->res_host, res_ints * 4) != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+
+    // Attention key splits for decode (fixed per context so a sequence's
+    // result does not depend on its batch neighbours).
+    if (ctx->bf16) {
+        const int g = ctx->hq / ctx->hkv;
+        const int rt = attn_rows_per_tile(g);
+        const int tiles = (maxW + rt - 1) / rt;
+        const int base = B * tiles * ctx->hkv;
+        int splits = (2 * ctx->num_sms + base - 1) / base;
+        splits = std::max(1, std::min(splits, (ctx->max_ctx + 255) / 256));
+        ctx->attn_kv_chunk = (int)align_up((size_t)((ctx->max_ctx + splits - 1) / splits), 64);
+        ctx->attn_max_splits = (ctx->max_ctx + ctx->attn_kv_chunk - 1) / ctx->attn_kv_chunk;
+    }
+
+    // Scratch.
+    Arena& xa = ctx->scratch_arena;
+    xa.add((void**)&ctx->x, (size_t)Mmax * d * 4);
+    xa.add(&ctx->h, (size_t)Mmax * d * elt);
+    xa.add(&ctx->q, (size_t)Mmax * ctx->hq * ctx->hd * elt);
+    xa.add(&ctx->attn_out, (size_t)Mmax * ctx->hq * ctx->hd * elt);
+    xa.add(&ctx->act, (size_t)Mmax * F * elt);
+    size_t need = 0;
+    for (int M : {ctx->Mdec, ctx->chunk}) {
+        need = std::max(need, gemm_ws_need(ctx, M, ctx->Nqkv, d));
+        need = std::max(need, gemm_ws_need(ctx, M, d, ctx->hq * ctx->hd));
+        need = std::max(need, gemm_ws_need(ctx, M, 2 * F, d));
+        need = std::max(need, gemm_ws_need(ctx, M, d, F));
+    }
+    ctx->ws_floats = need;
+    xa.add((void**)&ctx->ws, need * 4);
+    const size_t lsp = ctx->bf16 ? (size_t)std::min(4, plan_gemm_bf16(ctx->Mdec, V, d, ctx->num_sms).splits) : 1;
+    ctx->logits_floats = lsp * ctx->Mdec * (size_t)V;
+    xa.add((void**)&ctx->logits, ctx->logits_floats * 4);
+    xa.add((void**)&ctx->ent_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float4));
+    if (ctx->bf16 && ctx->attn_max_splits > 1) {
+        const size_t pairs = (size_t)ctx->Mdec * ctx->hq * ctx->attn_max_splits;
+        xa.add((void**)&ctx->attn_po, pairs * ctx->hd * 4);
+        xa.add((void**)&ctx->attn_pml, pairs * sizeof(float2));
+    }
+    if (xa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+
+    launch_rope_table(ctx->rope_cs, ctx->max_ctx, ctx->hd / 2, ctx->hd, cfg->rope_theta, ctx->stream);
+    std::vector<int32_t> pt((size_t)B * ctx->pages_per_seq, -1);
+    if (cudaMemcpy(ss.page_table, pt.data(), pt.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+        return bail(WEDLM_ERR_CUDA);
+    if (cudaDeviceSynchronize() != cudaSuccess) return bail(WEDLM_ERR_CUDA);
+    ctx->h_W.assign(B, 0);
+    ctx->h_S.assign(B, 0);
+    ctx->h_end.assign(B, 0);
+    ctx->h_P.assign(B, 0);
+    ctx->h_pages.assign(B, {});
+    ctx->free_pages.resize(ctx->num_pages);
+    for (int i = 0; i < ctx->num_pages; ++i) ctx->free_pages[i] = ctx->num_pages - 1 - i;
+    *out_ctx = ctx;
+    return WEDLM_OK;
+}
+
+void wedlm_destroy(wedlm_ctx* ctx) {
+    if (!ctx) return;
+    if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+    else cudaDeviceSynchronize();
+    ctx->weights_arena.release();
+    ctx->state_arena.release();
+    ctx->scratch_arena.release();
+    if (ctx->res_host) cudaFreeHost(ctx->res_host);
+    delete ctx;
+}
+
+wedlm_status wedlm_load_weights(wedlm_ctx* ctx, int32_t tensor, int32_t layer, const void* src, int32_t src_dtype,
+                                int32_t src_mem) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (!src) return fail(ctx, WEDLM_ERR_INVALID_ARG, "null source");
+    if (src_mem != WEDLM_MEM_HOST && src_mem != WEDLM_MEM_DEVICE)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad src_mem");
+    const int slot = tensor_slot(ctx, tensor, layer);
+    if (slot < 0) return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad tensor id or layer");
+    const bool norm = tensor == WEDLM_T_FINAL_NORM || tensor == WEDLM_T_ATTN_NORM || tensor == WEDLM_T_FFN_NORM;
+    const int want = norm ? WEDLM_DTYPE_F32 : ctx->cfg.dtype;
+    if (src_dtype != want) return fail(ctx, WEDLM_ERR_INVALID_ARG, "source dtype does not match the tensor's dtype");
+    const size_t elt = ctx->elt;
+    const size_t d = ctx->d, qd = (size_t)ctx->hq * ctx->hd, kd = (size_t)ctx->hkv * ctx->hd, F = ctx->F;
+    char* dst = nullptr;
+    size_t bytes = 0;
+    switch (tensor) {
+        case WEDLM_T_EMBED: dst = (char*)ctx->embed; bytes = (size_t)ctx->V * d * elt; break;
+        case WEDLM_T_LM_HEAD: dst = (char*)ctx->lm_head; bytes = (size_t)ctx->V * d * elt; break;
+        case WEDLM_T_FINAL_NORM: dst = (char*)ctx->final_norm; bytes = d * 4; break;
+        case WEDLM_T_ATTN_NORM: dst = (char*)ctx->attn_norm[layer]; bytes = d * 4; break;
+        case WEDLM_T_FFN_NORM: dst = (char*)ctx->ffn_norm[layer]; bytes = d * 4; break;
+        case WEDLM_T_WQ: dst = (char*)ctx->wqkv[layer]; bytes = qd * d * elt; break;
+        case WEDLM_T_WK: dst = (char*)ctx->wqkv[layer] + qd * d * elt; bytes = kd * d * elt; break;
+        case WEDLM_T_WV: dst = (char*)ctx->wqkv[layer] + (qd + kd) * d * elt; bytes = kd * d * elt; break;
+        case WEDLM_T_WO: dst = (char*)ctx->wo[layer]; bytes = d * qd * elt; break;
+        case WEDLM_T_WG: dst = (char*)ctx->wgu[layer]; bytes = F * d * elt; break;
+        case WEDLM_T_WU: dst = (char*)ctx->wgu[layer] + F * d * elt; bytes = F * d * elt; break;
+        case WEDLM_T_WD: dst = (char*)ctx->wd[layer]; bytes = d * F * elt; break;
+        default: return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad tensor id");
+    }
+    CK(cudaMemcpyAsync(dst, src, bytes, src_mem == WEDLM_MEM_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice,
+                       ctx->stream));
+    CK(cudaStreamSynchronize(ctx->stream));
+    ctx->loaded[slot] = 1;
+    bool all = true;
+    for (uint8_t f : ctx->loaded) all &= f != 0;
+    ctx->weights_ready = all;
+    ctx->maps_ready = false;
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_prefill(wedlm_ctx* ctx, int32_t slot, const int32_t* prompt_ids, int32_t prompt_len,
+                           int32_t max_new_tokens, int32_t window) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB) return fail(ctx, WEDLM_ERR_INVALID_ARG, "slot out of range");
+    if (prompt_len < 0 || (prompt_len > 0 && !prompt_ids)) return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad prompt");
+    if (max_new_tokens < 1 || (int64_t)prompt_len + max_new_tokens > ctx->max_ctx)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "prompt_len + max_new_tokens must be in [1, max_ctx]");
+    if (window < 1 || window > ctx->maxW) return fail(ctx, WEDLM_ERR_INVALID_ARG, "window out of range");
+    if (!ctx->weights_ready) return fail(ctx, WEDLM_ERR_STATE, "weights not fully loaded");
+    if (ctx->h_W[slot] != 0) return fail(ctx, WEDLM_ERR_STATE, "slot is in use (call wedlm_kv_reset)");
+    for (int i = 0; i < prompt_len; ++i)
+        if (prompt_ids[i] < 0 || prompt_ids[i] >= ctx->V)
+            return fail(ctx, WEDLM_ERR_INVALID_ARG, "prompt id out of range");
+    const int end = prompt_len + max_new_tokens;
+    const int need = (end + kPage - 1) / kPage;
+    if ((int)ctx->free_pages.size() < need) return fail(ctx, WEDLM_ERR_OOM_PAGES, "KV page pool exhausted");
+    wedlm_status s = build_weight_maps(ctx);
+    if (s) return s;
+    std::vector<int32_t> row(ctx->pages_per_seq, -1);
+    std::vector<int> taken;
+    for (int i = 0; i < need; ++i) {
+        taken.push_back(ctx->free_pages.back());
+        ctx->free_pages.pop_back();
+        row[i] = taken.back();
+    }
+    auto give_back = [&]() {
+        for (int p : taken) ctx->free_pages.push_back(p);
+    };
+    cudaError_t e = cudaMemcpyAsync(ctx->ss.page_table + (size_t)slot * ctx->pages_per_seq, row.data(),
+                                    row.size() * 4, cudaMemcpyHostToDevice, ctx->stream);
+    if (e != cudaSuccess) {
+        give_back();
+        return fail(ctx, WEDLM_ERR_CUDA, cudaGetErrorString(e));
+    }
+    launch_slot_admit(ctx->ss, slot, prompt_len, end, window, ctx->stream);
+    ctx->launches++;
+    for (int c0 = 0; c0 < prompt_len; c0 += ctx->chunk) {
+        const int n = std::min(ctx->chunk, prompt_len - c0);
+        e = cudaMemcpyAsync(ctx->ids_dev, prompt_ids + c0, (size_t)n * 4, cudaMemcpyHostToDevice, ctx->stream);
+        if (e != cudaSuccess) {
+            give_back();
+            return fail(ctx, WEDLM_ERR_CUDA, cudaGetErrorString(e));
+        }
+        if (ctx->bf16)
+            launch_prefill_prepare<bf16>((const bf16*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
+                                         ctx->ids_dev, slot, c0, n, ctx->ss, ctx->rs, ctx->x, (bf16*)ctx->h,
+                                         ctx->stream);
+        else
+            launch_prefill_prepare<float>((const float*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
+                                          ctx->ids_dev, slot, c0, n, ctx->ss, ctx->rs, ctx->x, (float*)ctx->h,
+                                          ctx->stream);
+        ctx->launches++;
+        s = run_forward(ctx, slot, 1, n, false);
+        if (s) {
+            give_back();
+            return s;
+        }
+        // the ids buffer is reused by the next chunk: wait for this one
+        e = cudaStreamSynchronize(ctx->stream);
+        if (e != cudaSuccess) {
+            give_back();
+            return fail(ctx, WEDLM_ERR_CUDA, cudaGetErrorString(e));
+        }
+    }
+    launch_prefill_finish(ctx->ss, slot, prompt_len, ctx->stream);
+    ctx->launches++;
+    int errw = 0;
+    CK(cudaMemcpyAsync(&errw, ctx->err, 4, cudaMemcpyDeviceToHost, ctx->stream));
+    CK(cudaStreamSynchronize(ctx->stream));
+    s = check_device_error(ctx, errw);
+    if (s) {
+        give_back();
+        launch_slot_admit(ctx->ss, slot, 0, 0, 0, ctx->stream);
+        return s;
+    }
+    ctx->h_pages[slot] = taken;
+    ctx->h_W[slot] = window;
+    ctx->h_S[slot] = prompt_len;
+    ctx->h_end[slot] = end;
+    ctx->h_P[slot] = prompt_len;
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_kv_reset(wedlm_ctx* ctx, int32_t slot) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < -1 || slot >= ctx->maxB) return fail(ctx, WEDLM_ERR_INVALID_ARG, "slot out of range");
+    CK(cudaStreamSynchronize(ctx->stream));
+    for (int b = 0; b < ctx->maxB; ++b) {
+        if (slot != -1 && b != slot) continue;
+        for (int p : ctx->h_pages[b]) ctx->free_pages.push_back(p);
+        ctx->h_pages[b].clear();
+        ctx->h_W[b] = ctx->h_S[b] = ctx->h_end[b] = ctx->h_P[b] = 0;
+        launch_slot_admit(ctx->ss, b, 0, 0, 0, ctx->stream);
+        ctx->launches++;
+        std::vector<int32_t> row(ctx->pages_per_seq, -1);
+        CK(cudaMemcpyAsync(ctx->ss.page_table + (size_t)b * ctx->pages_per_seq, row.data(), row.size() * 4,
+                           cudaMemcpyHostToDevice, ctx->stream));
+        CK(cudaStreamSynchronize(ctx->stream));
+    }
+    return WEDLM_OK;
+}
+
+static wedlm_status check_params(wedlm_ctx* ctx, const wedlm_step_params* p) {
+    if (!p) return fail(ctx, WEDLM_ERR_INVALID_ARG, "null params");
+    if (!(p->logit_scale > 0.f) || !std::isfinite(p->logit_scale) || std::isnan(p->lambda) || std::isnan(p->tau))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "logit_scale must be finite and > 0; lambda, tau not NaN");
+    if (!ctx->weights_ready) return fail(ctx, WEDLM_ERR_STATE, "weights not fully loaded");
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_stream_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int32_t* out_committed,
+                               int32_t* out_counts, int32_t* out_active) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    wedlm_status s = check_params(ctx, prm);
+    if (s) return s;
+    const int B = ctx->maxB, maxW = ctx->maxW;
+    int n_entries = 0;
+    const int stride = max_active_window(ctx, &n_entries);
+    if (n_entries == 0) {
+        if (out_counts) std::memset(out_counts, 0, B * 4);
+        if (out_active) *out_active = 0;
+        return WEDLM_OK;
+    }
+    s = enqueue_step(ctx, prm, n_entries, stride);
+    if (s) return s;
+    const size_t res_ints = (size_t)2 * B + (size_t)B * maxW + 1;
+    CK(cudaMemcpyAsync(ctx->res_host, ctx->res_dev, res_ints * 4, cudaMemcpyDeviceToHost, ctx->stream));
+    CK(cudaStreamSynchronize(ctx->stream));
+    const int32_t* counts = ctx->res_host;
+    const int32_t* S = ctx->res_host + B;
+    const int32_t* toks = ctx->res_host + 2 * B;
+    const int errw = ctx->res_host[res_ints - 1];
+    s = check_device_error(ctx, errw);
+    if (s) return s;
+    int active = 0;
+    for (int b = 0; b < B; ++b) {
+        if (ctx->h_W[b] > 0) {
+            ctx->h_S[b] = S[b];
+            if (S[b] < ctx->h_end[b]) ++active;
+        }
+    }
+    if (out_counts) std::memcpy(out_counts, counts, (size_t)B * 4);
+    if (out_committed) std::memcpy(out_committed, toks, (size_t)B * maxW * 4);
+    if (out_active) *out_active = active;
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_stream_step_async(wedlm_ctx* ctx, const wedlm_step_params* prm, int32_t n_steps) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    wedlm_status s = check_params(ctx, prm);
+    if (s) return s;
+    if (n_steps < 0) return fail(ctx, WEDLM_ERR_INVALID_ARG, "n_steps < 0");
+    int n_entries = 0;
+    const int stride = max_active_window(ctx, &n_entries);
+    if (n_entries == 0) return WEDLM_OK;
+    for (int i = 0; i < n_steps; ++i) {
+        s = enqueue_step(ctx, prm, n_entries, stride);
+        if (s) return s;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, cudaGetErrorString(e));
+    return WEDLM_OK;
+}
+
+static wedlm_status refresh_mirrors(wedlm_ctx* ctx) {
+    const int B = ctx->maxB, maxW = ctx->maxW;
+    const size_t res_ints = (size_t)2 * B + (size_t)B * maxW + 1;
+    CK(cudaMemcpyAsync(ctx->res_host, ctx->res_dev, res_ints * 4, cudaMemcpyDeviceToHost, ctx->stream));
+    CK(cudaStreamSynchronize(ctx->stream));
+    for (int b = 0; b < B; ++b)
+        if (ctx->h_W[b] > 0) ctx->h_S[b] = ctx->res_host[B + b];
+    return check_device_error(ctx, ctx->res_host[res_ints - 1]);
+}
+
+wedlm_status wedlm_read_generated(wedlm_ctx* ctx, int32_t slot, int32_t* out_tokens, int32_t cap, int32_t* out_len) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB || !out_len || cap < 0 || (cap > 0 && !out_tokens))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad slot or buffer");
+    wedlm_status s = refresh_mirrors(ctx);
+    if (s) return s;
+    const int len = ctx->h_W[slot] > 0 ? ctx->h_S[slot] - ctx->h_P[slot] : 0;
+    *out_len = len;
+    const int n = std::min(len, cap);
+    if (n > 0) {
+        CK(cudaMemcpy(out_tokens, ctx->ss.gen + (size_t)slot * ctx->max_ctx, (size_t)n * 4, cudaMemcpyDeviceToHost));
+    }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_get_stats(wedlm_ctx* ctx, int32_t slot, wedlm_seq_stats* out) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB || !out) return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad slot or output");
+    wedlm_status s = refresh_mirrors(ctx);
+    if (s) return s;
+    int64_t c[4];
+    CK(cudaMemcpy(c, ctx->ss.counters + (size_t)slot * 4, sizeof(c), cudaMemcpyDeviceToHost));
+    out->steps = c[0];
+    out->forward_rows = c[1];
+    out->committed = c[2];
+    out->fills = c[3];
+    out->committed_len = ctx->h_S[slot];
+    out->end = ctx->h_end[slot];
+    out->window = ctx->h_W[slot];
+    out->active = (ctx->h_W[slot] > 0 && ctx->h_S[slot] < ctx->h_end[slot]) ? 1 : 0;
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_kernel_launches(const wedlm_ctx* ctx, int64_t* out) {
+    if (!ctx || !out) return WEDLM_ERR_INVALID_ARG;
+    *out = ctx->launches;
+    return WEDLM_OK;
+}
+
+// ------------------------------------------------------------- test hooks --
+static float bf16_bits_to_float(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    std::memcpy(&f, &u, 4);
+    return f;
+}
+
+wedlm_status wedlm_debug_read(wedlm_ctx* ctx, int32_t item, void* host_dst, int64_t bytes) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (!host_dst || bytes < 0) return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad destination");
+    CK(cudaStreamSynchronize(ctx->stream));
+    const int B = ctx->maxB, maxW = ctx->maxW;
+    const void* src = nullptr;
+    size_t avail = 0;
+    switch (item) {
+        case WEDLM_DBG_PERM: src = ctx->rs.perm; avail = (size_t)ctx->Mmax * 4; break;
+        case WEDLM_DBG_POS: src = ctx->rs.pos; avail = (size_t)ctx->Mmax * 4; break;
+        case WEDLM_DBG_ROWTOK: src = ctx->rs.tok; avail = (size_t)ctx->Mmax * 4; break;
+        case WEDLM_DBG_HTILDE: src = ctx->ss.htilde; avail = (size_t)B * maxW * 4; break;
+        case WEDLM_DBG_ARGMAX: src = ctx->ss.amax; avail = (size_t)B * maxW * 4; break;
+        case WEDLM_DBG_FILL: src = ctx->ss.fillflag; avail = (size_t)B * maxW; break;
+        case WEDLM_DBG_ROWSTRIDE: {
+            if (bytes < 8) return fail(ctx, WEDLM_ERR_INVALID_ARG, "need 8 bytes");
+            const int32_t v[2] = {ctx->last_stride, ctx->last_M};
+            std::memcpy(host_dst, v, 8);
+            return WEDLM_OK;
+        }
+        case WEDLM_DBG_KN: {
+            if ((size_t)bytes > (size_t)B * 3 * 4) return fail(ctx, WEDLM_ERR_INVALID_ARG, "too many bytes");
+            std::vector<int32_t> k(B), n(B), nf(B), outv((size_t)B * 3);
+            CK(cudaMemcpy(k.data(), ctx->ss.k, B * 4, cudaMemcpyDeviceToHost));
+            CK(cudaMemcpy(n.data(), ctx->ss.n, B * 4, cudaMemcpyDeviceToHost));
+            CK(cudaMemcpy(nf.data(), ctx->ss.nf, B * 4, cudaMemcpyDeviceToHost));
+            for (int b = 0; b < B; ++b) {
+                outv[3 * b] = k[b];
+                outv[3 * b + 1] = n[b];
+                outv[3 * b + 2] = nf[b];
+            }
+            std::memcpy(host_dst, outv.data(), (size_t)bytes);
+            return WEDLM_OK;
+        }
+        case WEDLM_DBG_LOGITS: {
+            const size_t plane = (size_t)ctx->last_M * ctx->V;
+            if ((size_t)bytes > plane * 4) return fail(ctx, WEDLM_ERR_INVALID_ARG, "too many bytes");
+            const size_t nf = (size_t)bytes / 4;
+            float* dst = (float*)host_dst;
+            CK(cudaMemcpy(dst, ctx->logits, nf * 4, cudaMemcpyDeviceToHost));
+            if (ctx->logits_splits_last > 1) {
+                std::vector<float> tmp(nf);
+                for (int sp = 1; sp < ctx->logits_splits_last; ++sp) {
+                    CK(cudaMemcpy(tmp.data(), ctx->logits + sp * plane, nf * 4, cudaMemcpyDeviceToHost));
+                    for (size_t i = 0; i < nf; ++i) dst[i] += tmp[i];
+                }
+            }
+            return WEDLM_OK;
+        }
+        default: return fail(ctx, WEDLM_ERR_INVALID_ARG, "unknown debug item");
+    }
+    if ((size_t)bytes > avail) return fail(ctx, WEDLM_ERR_INVALID_ARG, "too many bytes for this item");
+    CK(cudaMemcpy(host_dst, src, (size_t)bytes, cudaMemcpyDeviceToHost));
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t pos0, int32_t n, float* host_k,
+                            float* host_v) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB || layer < 0 || layer >= ctx->L || pos0 < 0 || n < 0 || !host_k || !host_v)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad arguments");
+    if ((int64_t)pos0 + n > (int64_t)ctx->h_pages[slot].size() * kPage)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "positions beyond the slot's pages");
+    CK(cudaStreamSynchronize(ctx->stream));
+    const int hkv = ctx->hkv, hd = ctx->hd;
+    const size_t page_elems = (size_t)2 * hkv * kPage * hd;
+    std::vector<uint8_t> buf(page_elems * ctx->elt);
+    int cur = -1;
+    for (int i = 0; i < n; ++i) {
+        const int p = pos0 + i;
+        const int pidx = p / kPage;
+        if (pidx != cur) {
+            const int page = ctx->h_pages[slot][pidx];
+            const char* src = (const char*)ctx->kv_pool +
+                              ((size_t)layer * ctx->kvl.layer_stride + (size_t)page * page_elems) * ctx->elt;
+            CK(cudaMemcpy(buf.data(), src, buf.size(), cudaMemcpyDeviceToHost));
+            cur = pidx;
+        }
+        for (int kv = 0; kv < 2; ++kv)
+            for (int hh = 0; hh < hkv; ++hh)
+                for (int c = 0; c < hd; ++c) {
+                    const size_t idx = (((size_t)kv * hkv + hh) * kPage + (p % kPage)) * hd + c;
+                    const float v = ctx->bf16 ? bf16_bits_to_float(((const uint16_t*)buf.data())[idx])
+                                              : ((const float*)buf.data())[idx];
+                    (kv ? host_v : host_k)[((size_t)i * hkv + hh) * hd + c] = v;
+                }
+    }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_get_window(wedlm_ctx* ctx, int32_t slot, uint8_t* filled, int32_t* tokens, int32_t cap,
+                                    int32_t* n) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB || !filled || !tokens || !n || cap < 0)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad arguments");
+    CK(cudaStreamSynchronize(ctx->stream));
+    int32_t w = 0;
+    CK(cudaMemcpy(&w, ctx->ss.wlen + slot, 4, cudaMemcpyDeviceToHost));
+    *n = w;
+    const int m = std::min(w, cap);
+    if (m > 0) {
+        CK(cudaMemcpy(filled, ctx->ss.filled + (size_t)slot * ctx->maxW, m, cudaMemcpyDeviceToHost));
+        CK(cudaMemcpy(tokens, ctx->ss.token + (size_t)slot * ctx->maxW, (size_t)m * 4, cudaMemcpyDeviceToHost));
+    }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_set_window(wedlm_ctx* ctx, int32_t slot, const uint8_t* filled, const int32_t* tokens,
+                                    int32_t n) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB || n < 0 || n > ctx->maxW || (n > 0 && (!filled || !tokens)))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad arguments");
+    if (ctx->h_W[slot] == 0) return fail(ctx, WEDLM_ERR_STATE, "slot not in use");
+    if (n > ctx->h_W[slot] || n > ctx->h_end[slot] - ctx->h_S[slot])
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "window longer than W or than the remaining positions");
+    for (int j = 0; j < n; ++j)
+        if (filled[j] && (tokens[j] < 0 || tokens[j] >= ctx->V || tokens[j] == ctx->cfg.mask_id))
+            return fail(ctx, WEDLM_ERR_INVALID_ARG, "filled slot with an invalid token");
+    CK(cudaStreamSynchronize(ctx->stream));
+    std::vector<uint8_t> f(ctx->maxW, 0);
+    std::vector<int32_t> t(ctx->maxW, ctx->cfg.mask_id);
+    for (int j = 0; j < n; ++j) {
+        f[j] = filled[j] ? 1 : 0;
+        t[j] = filled[j] ? tokens[j] : ctx->cfg.mask_id;
+    }
+    CK(cudaMemcpy(ctx->ss.filled + (size_t)slot * ctx->maxW, f.data(), ctx->maxW, cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(ctx->ss.token + (size_t)slot * ctx->maxW, t.data(), (size_t)ctx->maxW * 4, cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(ctx->ss.wlen + slot, &n, 4, cudaMemcpyHostToDevice));
+    return WEDLM_OK;
+}
+
+}  // extern "C"
