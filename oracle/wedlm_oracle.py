@@ -292,13 +292,16 @@ def prefill(m: Model, prompt, N: int, W: int) -> SeqState:
 
 
 def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
-                logit_scale: float, forward=None, keep_trace: bool = True) -> StepTrace | None:
+                logit_scale: float, forward=None, keep_trace: bool = True, choose=None) -> StepTrace | None:
     """One Streaming Parallel Decoding step (Summary/Method), in the pages' order:
     refill the window with masks, reorder, causal forward, commit the leftmost
     filled run, then fill selected masks (distance-penalised entropy rule).
 
     ``forward(m, cache, toks, pos) -> (logits rows [n, V] or None, wk, wv)`` may
-    replace the model forward (used by tests with a scripted predictor)."""
+    replace the model forward (used by tests with a scripted predictor).
+    ``choose(step_index, Ht, fills) -> fills`` lets a test make the oracle follow
+    another implementation's fill decision where floating point leaves it open;
+    it does not change how anything is computed."""
     if st.done:
         return None
     # refill: masks appended so the window holds min(W, end - S) slots (R12)
@@ -329,6 +332,8 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
         H[j], amax[j] = entropy_argmax(logits[j], m.mask_id)
         Ht[j] = penalised_entropy(H[j], j, lam)
     fills = select_fills(Ht, tau, tau_none)
+    if choose is not None:
+        fills = list(choose(st.steps, Ht, fills))
     for j in fills:
         st.filled[j] = True
         st.token[j] = amax[j]
@@ -348,14 +353,14 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
 
 def stream_decode(m: Model, prompt, N: int, W: int, lam: float, tau: float,
                   tau_none: bool = False, logit_scale: float = 1.0, max_steps: int | None = None,
-                  forward=None) -> SeqState:
+                  forward=None, choose=None) -> SeqState:
     """Decode N tokens after ``prompt`` with Streaming Parallel Decoding."""
     st = prefill(m, prompt, N, W) if forward is None else SeqState(
         prompt=np.asarray(prompt), N=N, W=W, cache=KVCache.empty(m), S=len(prompt), end=len(prompt) + N)
     while not st.done:
         if max_steps is not None and st.steps >= max_steps:
             break
-        stream_step(m, st, lam, tau, tau_none, logit_scale, forward=forward)
+        stream_step(m, st, lam, tau, tau_none, logit_scale, forward=forward, choose=choose)
     return st
 
 

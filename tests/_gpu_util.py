@@ -41,3 +41,23 @@ def oracle_select(logits_rows: dict, mask_id: int, lam: float, tau: float, tau_n
         Ht[j] = O.penalised_entropy(H, j, lam)
         am[j] = a
     return Ht, am, O.select_fills(Ht, tau, tau_none)
+
+
+def valid_fill_decision(Ht: dict, tau: float, tau_none: bool, fills) -> bool:
+    """Is `fills` a decision the rule allows once every H~ may be off by MARGIN?
+
+    Slots with H~ < tau - MARGIN must be filled and slots with H~ > tau + MARGIN
+    must not (threshold branch); a single fill is also valid as the fallback if
+    no slot is certainly under tau and the slot is within MARGIN of the minimum."""
+    fills = sorted(fills)
+    if not Ht:
+        return fills == []
+    under = {j for j, v in Ht.items() if v < tau - MARGIN}
+    over = {j for j, v in Ht.items() if v > tau + MARGIN}
+    lo = min(Ht.values())
+    if len(fills) == 1 and not (under and not tau_none) and Ht.get(fills[0], float("inf")) <= lo + MARGIN:
+        return True
+    if tau_none or not fills:
+        return False
+    F = set(fills)
+    return F.issubset(Ht) and under.issubset(F) and not (F & over)

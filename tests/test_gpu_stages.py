@@ -66,8 +66,9 @@ def test_entropy_select_matches_oracle(V, logit_std, lam, tau, tau_none, scale):
     filled, _ = synth.window_state(2000 + V % 97, 0, n_seq, stride, None, V, mask_id)
     n = np.array([16, 16, 9, 1, 13, 16], np.int32)
     logits = synth.normal(2100, int(logit_std * 10), logit_std, (n_seq, stride, V), "f32")
-    # a few exact ties for the argmax rule
-    logits[0, 1, 7] = logits[0, 1, 9] = logits[0, 1].max() + 1.0
+    # an exact tie for the argmax rule in the first masked slot of sequence 0
+    j0 = int(np.nonzero(filled[0, :n[0]] == 0)[0][0])
+    logits[0, j0, 7] = logits[0, j0, 9] = logits[0, j0].max() + 1.0
     prm = step_params(lam, tau, tau_none, scale)
     ht, am, fill = entropy_select(_dev(logits, torch.float32), V, mask_id, _dev(filled, torch.uint8),
                                   _dev(n, torch.int32), stride, prm)
@@ -86,7 +87,7 @@ def test_entropy_select_matches_oracle(V, logit_std, lam, tau, tau_none, scale):
             assert sorted(np.nonzero(fill[b])[0].tolist()) == fills
             n_compared += 1
     assert n_compared >= n_seq - 1
-    assert am[0, 1] == 7  # lowest id among tied maxima
+    assert am[0, j0] == 7  # lowest id among tied maxima
 
 
 @pytest.mark.parametrize("M,N,K", [(16, 6144, 4096), (1, 300, 64), (37, 1000, 520), (128, 4096, 4096),

@@ -5,7 +5,7 @@ import pytest
 
 import synth
 from oracle import wedlm_oracle as O
-from _gpu_util import MARGIN, comparable, make_engine, oracle_model
+from _gpu_util import MARGIN, comparable, make_engine, oracle_model, valid_fill_decision
 
 pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -49,15 +49,34 @@ def run_gpu_traced(eng, slot_prompts, N, W, lam, tau, tau_none, scale):
     return out, traces
 
 
-def compare_traces(st, gtrace, tau, tau_none):
-    """Step-by-step equality while decisions are comparable; returns steps compared."""
+def lockstep_oracle(model, prompt, N, W, lam, tau, tau_none, scale, gtrace):
+    """Run the oracle alongside a recorded GPU trace.  Where the oracle's H~
+    leave the decision open within MARGIN, the GPU's decision must be a valid
+    one and the oracle then follows it; elsewhere decisions must be equal.
+    Returns (oracle state, number of near-tie steps)."""
+    near = [0]
+
+    def choose(t, Ht, fills):
+        g = gtrace[t]["fills"]
+        if comparable(Ht, tau, tau_none):
+            assert g == fills, (t, g, fills, Ht)
+        else:
+            assert valid_fill_decision(Ht, tau, tau_none, g), (t, g, fills, Ht)
+            near[0] += 1
+        return g
+
+    st = O.stream_decode(model, prompt, N, W, lam, tau, tau_none=tau_none, logit_scale=scale, choose=choose)
+    return st, near[0]
+
+
+def compare_traces(st, gtrace):
+    """Per-step equality of the commit run, window size, physical order and H~."""
     assert len(st.trace) == len(gtrace)
     for t_or, t_gpu in zip(st.trace, gtrace):
         assert (t_gpu["k"], t_gpu["n"], t_gpu["perm"]) == (t_or.k, t_or.n, t_or.perm)
         assert set(t_gpu["Ht"]) == set(t_or.Ht)
         for j, v in t_or.Ht.items():
             assert abs(t_gpu["Ht"][j] - v) < MARGIN, (j, t_gpu["Ht"][j], v)
-        assert comparable(t_or.Ht, tau, tau_none), "near-tie: pick another seed"
         assert t_gpu["fills"] == t_or.fills
     return len(st.trace)
 
@@ -69,9 +88,10 @@ def test_token_stream_and_decisions_match_oracle(model, cfg_name):
     eng = make_engine(DIMS, max_batch=1, max_window=cfg["W"], max_ctx=64)
     out, tr = run_gpu_traced(eng, {0: prompt}, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"], False,
                              cfg["logit_scale"])
-    st = O.stream_decode(model, prompt, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"],
-                         logit_scale=cfg["logit_scale"])
-    compare_traces(st, tr[0], cfg["tau"], False)
+    st, near = lockstep_oracle(model, prompt, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"], False,
+                               cfg["logit_scale"], tr[0])
+    compare_traces(st, tr[0])
+    assert near <= 2
     assert out[0] == st.out
     assert eng.read_generated(0) == st.out
     s = eng.stats(0)
@@ -131,8 +151,9 @@ def test_batch_of_ragged_sequences_matches_independent_decodes(model):
     eng = make_engine(DIMS, max_batch=4, max_window=4, max_ctx=64)
     out, tr = run_gpu_traced(eng, prompts, N, W, cfg["lam"], cfg["tau"], False, cfg["logit_scale"])
     for b, p in prompts.items():
-        st = O.stream_decode(model, p, N, W[b], cfg["lam"], cfg["tau"], logit_scale=cfg["logit_scale"])
-        compare_traces(st, tr[b], cfg["tau"], False)
+        st, near = lockstep_oracle(model, p, N, W[b], cfg["lam"], cfg["tau"], False, cfg["logit_scale"], tr[b])
+        compare_traces(st, tr[b])
+        assert near <= 2
         assert out[b] == st.out
 
 
