@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Committed tokens/s of Streaming Parallel Decoding on B200.
+
+Default workload: the Qwen3-8B-shaped bf16 model (36 layers, d 4096, 32/8
+heads, head_dim 128, FFN 12288, vocab 151936) at batch 16, prompts of
+U[128, 1024] uniform-random tokens, 1024 tokens to generate, window 16,
+lambda 0.1, tau 0.3, LM-head logit scale x4 (the medium-entropy regime).
+Batch 1 (prompt 256) and the x16 / x1 regimes are reported under "extra".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Sequences are independent, so
+ranks are replicas with their own prompts and no data-path collective
+("scaling": "weak"); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "committed tokens/s"
+UNIT = "tok/s"
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_8b_b16")
+    ap.add_argument("--no-extra", action="store_true", help="skip the batch-1 and regime sweeps")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="headline measurement only (for profiler runs)")
+    return ap.parse_args()
+
+
+def workload_desc(cfg: dict, name: str) -> str:
+    m = cfg["model"]
+    P = cfg["P"]
+    ps = f"U[{P[0]}, {P[1]}]" if isinstance(P, (tuple, list)) else str(P)
+    return (f"{name}: random-init bf16 model L{m['L']} d{m['d']} heads {m['hq']}/{m['hkv']} hd{m['hd']} "
+            f"ffn {m['F']} vocab {m['V']}; batch {cfg['B']}, prompts {ps} uniform ids, {cfg['N']} new tokens, "
+            f"W {cfg['W']}, lambda {cfg['lam']}, tau {cfg['tau']}, logit scale x{cfg['logit_scale']:g}")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], tc=p["bf16_tflops"], tc_sus=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, tc=1590.0, tc_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], cap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        load = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("cap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load),
+                "power_w_median": statistics.median(r["power"] for r in load)}
+
+
+# ------------------------------------------------------------- our arm ---
+class Replica:
+    """One engine holding the Qwen3-8B-shaped model with max batch 16."""
+
+    def __init__(self, cfg: dict, device: int, seed: int):
+        import torch
+        from streaming_decoding_b200 import Engine
+        self.torch = torch
+        self.cfg = cfg
+        self.dims = cfg["model"]
+        torch.cuda.set_device(device)
+        self.stream = torch.cuda.Stream()
+        Pmax = max(cfg["P"]) if isinstance(cfg["P"], (tuple, list)) else cfg["P"]
+        self.max_ctx = max(Pmax, 256) + cfg["N"]
+        t0 = time.perf_counter()
+        self.eng = Engine(self.dims, max_batch=cfg["B"], max_window=cfg["W"], max_ctx=self.max_ctx,
+                          stream=self.stream)
+        for kind, layer, arr in synth.iter_weights(self.dims, seed=0, dtype="bf16"):
+            self.eng.load_weights(kind, layer, arr)
+        self.load_s = time.perf_counter() - t0
+        self.seed = seed
+
+    def admit(self, prompts, N, W):
+        self.eng.kv_reset(-1)
+        t0 = time.perf_counter()
+        for b, p in enumerate(prompts):
+            self.eng.prefill(b, p, N, W)
+        self.prefill_s = time.perf_counter() - t0
+        self.prefill_tokens = int(sum(len(p) for p in prompts))
+
+    def committed(self, B):
+        return sum(self.eng.stats(b)["committed"] for b in range(B))
+
+    def timed_async(self, params, steps, B):
+        """Device time of `steps` back-to-back steps (no host sync inside)."""
+        torch = self.torch
+        c0 = self.committed(B)
+        l0 = self.eng.kernel_launches()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(self.stream)
+        self.eng.stream_step_async(params, steps)
+        end.record(self.stream)
+        end.synchronize()
+        ms = start.elapsed_time(end)
+        return ms, self.committed(B) - c0, self.eng.kernel_launches() - l0
+
+    def timed_e2e(self, params, steps):
+        """Same metric through the synchronous public call with pinned host buffers."""
+        torch = self.torch
+        B, W = self.cfg["B"], self.cfg["W"]
+        committed = torch.zeros((B, W), dtype=torch.int32).pin_memory().numpy()
+        counts = torch.zeros(B, dtype=torch.int32).pin_memory().numpy()
+        active = torch.zeros(1, dtype=torch.int32).pin_memory().numpy()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        total = 0
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        start.record(self.stream)
+        for _ in range(steps):
+            self.eng.stream_step_into(params, committed, counts, active)
+            total += int(counts.sum())
+        end.record(self.stream)
+        end.synchronize()
+        wall = time.perf_counter() - t0
+        d2h = (2 * B + B * W + 1) * 4
+        return start.elapsed_time(end), wall, total, d2h
+
+    def profile(self, params, steps):
+        self.eng.profile_enable(True)
+        self.eng.stream_step_async(params, steps)
+        prof = self.eng.profile_read()
+        self.eng.profile_enable(False)
+        return prof
+
+
+def gemm_shapes(dims, M):
+    d, hq, hkv, hd, F, V = dims["d"], dims["hq"], dims["hkv"], dims["hd"], dims["F"], dims["V"]
+    L = dims["L"]
+    return {"gemm_qkv": (L, M, (hq + 2 * hkv) * hd, d), "gemm_o": (L, M, d, hq * hd),
+            "gemm_gate_up": (L, M, 2 * F, d), "gemm_down": (L, M, d, F), "gemm_lm_head": (1, M, V, d)}
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "streaming_decoding_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current source."""
+    path = os.path.join(PROFILES, f"{kernel_file}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        p = json.load(f)
+    if p.get("source_hash") != src_hash(*p.get("sources", [])) or p.get("workload") != workload:
+        return None
+    return p.get("dram_bytes_per_launch")
+
+
+def roofline(prof, dims, M, pk, workload):
+    """Dominant kernel: the tcgen05 GEMM over all projections of the step."""
+    shapes = gemm_shapes(dims, M)
+    bytes_tot = flops_tot = ms_tot = 0.0
+    launches = 0
+    for kind, (count, m, n, k) in shapes.items():
+        ms, nl = prof.get(kind, (0.0, 0))
+        if nl == 0:
+            continue
+        per = nl / count  # profiled steps
+        bytes_tot += per * count * (2.0 * n * k + 2.0 * m * k + 4.0 * m * n)
+        flops_tot += per * count * 2.0 * m * n * k
+        ms_tot += ms
+        launches += nl
+    t_hbm = bytes_tot / (pk["hbm"] * 1e9)
+    t_tc = flops_tot / (pk["tc_sus"] * 1e12)
+    sec = ms_tot / 1e3
+    traffic = measured_traffic("gemm_bf16_tc", workload)
+    if t_hbm >= t_tc:
+        ach = bytes_tot / sec / 1e9
+        out = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
+               "frac": round(ach / pk["hbm"], 4)}
+    else:
+        ach = flops_tot / sec / 1e12
+        out = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["tc_sus"], "unit": "TFLOP/s",
+               "frac": round(ach / pk["tc_sus"], 4)}
+    out.update({"traffic": traffic, "kernel": "gemm_bf16_tc_kernel (all projections and LM head)",
+                "launches_profiled": launches, "avg_launch_us": round(ms_tot * 1e3 / max(1, launches), 2),
+                "algorithmic_bytes_per_launch": round(bytes_tot / max(1, launches)),
+                "peak_source": f"{pk['src']} ({'hbm_gbs' if out['bound'] == 'hbm' else 'bf16_tflops_sustained'})"})
+    return out, bytes_tot, flops_tot
+
+
+def step_bytes_flops(dims, B, W, S_mean):
+    """Algorithmic bytes and flops of one decode step (weights once, committed KV
+    once per sequence and layer, logits once)."""
+    d, hq, hkv, hd, F, V, L = (dims[k] for k in ("d", "hq", "hkv", "hd", "F", "V", "L"))
+    params = L * ((hq + 2 * hkv) * hd * d + d * hq * hd + 3 * F * d) + V * d
+    M = B * W
+    byt = 2.0 * params + B * S_mean * L * 2 * hkv * hd * 2 + M * V * 4
+    fl = 2.0 * M * (params - V * d) + 2.0 * M * V * d + 4.0 * M * hq * hd * (S_mean + W / 2) * L
+    return byt, fl
+
+
+def run_ours(a):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        from datetime import timedelta
+        dist = dist_mod
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    cfg = dict(synth.CONFIGS[a.workload])
+    dims = cfg["model"]
+    pk = peaks()
+    rep = Replica(cfg, local, seed=rank)
+    prompts = synth.prompts(cfg, seed=cfg["prompt_seed"] + 100 * rank)
+    B, W, N = cfg["B"], cfg["W"], cfg["N"]
+    from streaming_decoding_b200 import step_params
+    prm = step_params(cfg["lam"], cfg["tau"], False, cfg["logit_scale"])
+
+    # headline: device-resident steps, CUDA events on the library's stream
+    rep.admit(prompts, N, W)
+    rep.eng.stream_step_async(prm, a.warmup)
+    torch.cuda.synchronize()
+    S0 = np.mean([rep.eng.stats(b)["committed_len"] for b in range(B)])
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms, committed, launches = rep.timed_async(prm, a.steps, B)
+    ms_all = ms
+    tok_all = committed
+    if dist:
+        t = torch.tensor([ms, committed], dtype=torch.float64, device="cuda")
+        mx = t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        ms_all, tok_all = float(mx[0]), float(t[1])
+    value = tok_all / (ms_all / 1e3)
+    S1 = np.mean([rep.eng.stats(b)["committed_len"] for b in range(B)])
+
+    # per-kernel profile (separate pass; event gaps do not touch the headline)
+    prof = rep.profile(prm, 10)
+    M = B * W
+    roof, gb, gf = roofline(prof, dims, M, pk, a.workload)
+    sb, sf = step_bytes_flops(dims, B, W, (S0 + S1) / 2)
+    step_floor_ms = max(sb / (pk["hbm"] * 1e9), sf / (pk["tc_sus"] * 1e12)) * 1e3
+
+    # end to end through the public synchronous call
+    e2e_steps = max(20, a.steps // 3)
+    e_ms, e_wall, e_tok, d2h = rep.timed_e2e(prm, e2e_steps)
+    e2e_val = e_tok / (e_ms / 1e3)
+    if dist:
+        t = torch.tensor([e_ms, e_tok], dtype=torch.float64, device="cuda")
+        mx = t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        e2e_val = float(t[1]) / (float(mx[0]) / 1e3)
+
+    extra = {"prefill": {"tokens": rep.prefill_tokens, "seconds": round(rep.prefill_s, 3),
+                         "tok_per_s": round(rep.prefill_tokens / rep.prefill_s, 1)},
+             "weights_load_s": round(rep.load_s, 2),
+             "committed_per_step": round(committed / a.steps, 3),
+             "mean_committed_len": [round(S0, 1), round(S1, 1)],
+             "step_ms_floor_algorithmic": round(step_floor_ms, 3),
+             "step_roofline_frac": round(step_floor_ms / (ms / a.steps), 4),
+             "profile_ms_per_step": {k: round(v[0] / 10, 4) for k, v in prof.items() if v[1]},
+             "e2e_wall_s": round(e_wall, 3)}
+    if not a.quick and not a.no_extra and world == 1:
+        extra.update(sweeps(rep, cfg, a))
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.quick:
+        cpu = cpu_baseline(cfg, budget_s=25.0)
+        cpu.pop("steps_timed", None)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(ms_all / a.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded random-init weights, uniform-random prompt ids)",
+            "config": {"workload": workload_desc(cfg, a.workload), "batch_per_gpu": B, "window": W,
+                       "global_batch": B * world, "l2": "inputs larger than L2 (15.1 GB of weights read per step)",
+                       "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": d2h,
+                    "api": "wedlm_stream_step (synchronous), pinned host outputs",
+                    "note": "decode steps take no host input (window and KV state stay on the device)"},
+            "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "extra": extra}
+    print(json.dumps(line))
+
+
+def sweeps(rep, cfg, a):
+    """Batch 1 (prompt 256) and the logit-scale regimes at batch 16."""
+    from streaming_decoding_b200 import step_params
+    out = {}
+    steps = min(a.steps, 150)
+    b1 = synth.CONFIGS["qwen3_8b_b1"]
+    rep.admit(synth.prompts(b1), b1["N"], b1["W"])
+    prm = step_params(b1["lam"], b1["tau"], False, b1["logit_scale"])
+    rep.eng.stream_step_async(prm, a.warmup)
+    ms, com, _ = rep.timed_async(prm, steps, 1)
+    out["batch1"] = {"workload": workload_desc(b1, "qwen3_8b_b1"), "tok_per_s": round(com / (ms / 1e3), 2),
+                     "ms_per_step": round(ms / steps, 4), "committed_per_step": round(com / steps, 3)}
+    reg = {}
+    prompts = synth.prompts(cfg)
+    for scale in cfg["logit_scales"]:
+        rep.admit(prompts, cfg["N"], cfg["W"])
+        prm = step_params(cfg["lam"], cfg["tau"], False, scale)
+        rep.eng.stream_step_async(prm, a.warmup)
+        n = min(steps, 40 if scale >= 16 else steps)
+        ms, com, _ = rep.timed_async(prm, n, cfg["B"])
+        reg[f"x{scale:g}"] = {"tok_per_s": round(com / (ms / 1e3), 2), "ms_per_step": round(ms / n, 4),
+                              "committed_per_step": round(com / n, 3)}
+    out["regimes_batch16"] = reg
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle --
+def cpu_baseline(cfg, budget_s: float, steps_max: int = 50, warmup: int = 1):
+    """The oracle as it stands on the host cores: one sequence of the workload
+    (its first 16 prompt tokens), decoded step by step until the time budget
+    or `steps_max` is used; weight widening and prefill are untimed."""
+    from oracle import wedlm_oracle as O
+    dims = cfg["model"]
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 0) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    w = synth.model_weights(dims, seed=0, dtype="bf16")
+    m = O.Model(dims, w, cache_fp64=True)
+    prompt = synth.prompts(cfg)[0][:16]
+    st = O.prefill(m, prompt, cfg["N"], cfg["W"])
+    for _ in range(warmup):
+        O.stream_step(m, st, cfg["lam"], cfg["tau"], False, cfg["logit_scale"], keep_trace=False)
+    c0 = len(st.out)
+    t0 = time.perf_counter()
+    n = 0
+    while n < steps_max and time.perf_counter() - t0 < budget_s and not st.done:
+        O.stream_step(m, st, cfg["lam"], cfg["tau"], False, cfg["logit_scale"], keep_trace=False)
+        n += 1
+    dt = time.perf_counter() - t0
+    com = len(st.out) - c0
+    return {"value": round(com / dt, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"1 sequence (first 16 prompt tokens), {n} decode steps after {warmup} untimed, "
+                      f"{com} tokens committed in {dt:.1f} s; fp64 numpy",
+            "s_per_step": round(dt / max(1, n), 3), "steps_timed": n}
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    cfg = dict(synth.CONFIGS[a.workload])
+    res = cpu_baseline(cfg, budget_s=120.0, steps_max=max(1, a.steps), warmup=max(1, min(a.warmup, 2)))
+    steps = res.pop("steps_timed")
+    line = {"impl": "reference", "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": a.warmup, "ms_per_step": round(res["s_per_step"] * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded random-init weights, uniform-random prompt ids)",
+            "config": {"workload": workload_desc(cfg, a.workload), "batch_per_gpu": cfg["B"], "window": cfg["W"]},
+            "cpu_baseline": res,
+            "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)

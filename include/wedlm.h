@@ -202,6 +202,31 @@ wedlm_status wedlm_get_stats(wedlm_ctx* ctx, int32_t slot, wedlm_seq_stats* out)
  * counted once; a captured graph counts its kernels at every replay). */
 wedlm_status wedlm_kernel_launches(const wedlm_ctx* ctx, int64_t* out);
 
+/* Per-kernel timing.  While enabled, every launch the context makes is
+ * bracketed by CUDA events on its stream (which adds a small gap between
+ * kernels) and its duration is added to the kind's total.  Kinds: */
+#define WEDLM_PROF_PREPARE       0   /* refill + reorder + embed + RMSNorm */
+#define WEDLM_PROF_GEMM_QKV      1
+#define WEDLM_PROF_QKV_ROPE      2   /* split-K sum + RoPE + K/V into pages */
+#define WEDLM_PROF_ATTENTION     3
+#define WEDLM_PROF_ATTN_COMBINE  4
+#define WEDLM_PROF_GEMM_O        5
+#define WEDLM_PROF_RESIDUAL_NORM 6
+#define WEDLM_PROF_GEMM_GATE_UP  7
+#define WEDLM_PROF_SWIGLU        8
+#define WEDLM_PROF_GEMM_DOWN     9
+#define WEDLM_PROF_GEMM_LM_HEAD 10
+#define WEDLM_PROF_ENTROPY      11
+#define WEDLM_PROF_SELECT       12
+#define WEDLM_PROF_KINDS        13
+
+/* Enable (1) or disable (0) per-kernel timing; enabling clears the totals. */
+wedlm_status wedlm_profile_enable(wedlm_ctx* ctx, int32_t on);
+
+/* Synchronise and return the totals: ms[WEDLM_PROF_KINDS] (milliseconds) and
+ * launches[WEDLM_PROF_KINDS] (either may be NULL). */
+wedlm_status wedlm_profile_read(wedlm_ctx* ctx, double* ms, int64_t* launches);
+
 /* ---------------------------------------------------------------------
  * Test hooks.  They expose intermediate state of the most recent step so the
  * tests can compare each stage with an independent CPU implementation.

@@ -63,6 +63,8 @@ _SIGS = {
     "wedlm_read_generated": (c_i32, [c_vp, c_i32, c_vp, c_i32, c_vp]),
     "wedlm_get_stats": (c_i32, [c_vp, c_i32, ctypes.POINTER(SeqStats)]),
     "wedlm_kernel_launches": (c_i32, [c_vp, ctypes.POINTER(c_i64)]),
+    "wedlm_profile_enable": (c_i32, [c_vp, c_i32]),
+    "wedlm_profile_read": (c_i32, [c_vp, c_vp, c_vp]),
     "wedlm_debug_read": (c_i32, [c_vp, c_i32, c_vp, c_i64]),
     "wedlm_debug_kv": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp]),
     "wedlm_debug_get_window": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i32, c_vp]),

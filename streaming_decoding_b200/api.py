@@ -137,6 +137,19 @@ class Engine:
         _check(self.lib.wedlm_kernel_launches(self.ctx, ctypes.byref(n)), "wedlm_kernel_launches")
         return n.value
 
+    def profile_enable(self, on: bool = True):
+        _check(self.lib.wedlm_profile_enable(self.ctx, 1 if on else 0), "wedlm_profile_enable", self.ctx)
+
+    def profile_read(self) -> dict:
+        """{kind: (total ms, launches)} for kinds WEDLM_PROF_* since profile_enable."""
+        nk = C["WEDLM_PROF_KINDS"]
+        ms = np.zeros(nk, np.float64)
+        n = np.zeros(nk, np.int64)
+        _check(self.lib.wedlm_profile_read(self.ctx, ms.ctypes.data, n.ctypes.data), "wedlm_profile_read", self.ctx)
+        names = {v: k[len("WEDLM_PROF_"):].lower() for k, v in C.items()
+                 if k.startswith("WEDLM_PROF_") and k != "WEDLM_PROF_KINDS"}
+        return {names[i]: (float(ms[i]), int(n[i])) for i in range(nk)}
+
     # -- test hooks ---------------------------------------------------------
     def debug_read(self, item: str, shape, dtype):
         out = np.zeros(shape, dtype)

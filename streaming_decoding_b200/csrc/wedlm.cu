@@ -129,6 +129,13 @@ struct wedlm_ctx {
     int last_stride = 0;
     int logits_splits_last = 1;
     int last_M = 0;
+    // per-kernel timing (wedlm_profile_enable)
+    bool prof = false;
+    std::vector<cudaEvent_t> ev_pool;
+    size_t ev_used = 0;
+    std::vector<std::pair<int, size_t>> ev_marks;  // (kind, index of the start event)
+    double prof_ms[WEDLM_PROF_KINDS] = {};
+    int64_t prof_n[WEDLM_PROF_KINDS] = {};
 };
 
 namespace {
@@ -136,6 +143,44 @@ namespace {
 wedlm_status fail(wedlm_ctx* c, wedlm_status s, const std::string& msg) {
     if (c) c->last_error = msg;
     return s;
+}
+
+// Profiling: bracket a launch with events when enabled.
+cudaEvent_t prof_event(wedlm_ctx* c) {
+    if (c->ev_used == c->ev_pool.size()) {
+        cudaEvent_t e;
+        cudaEventCreate(&e);
+        c->ev_pool.push_back(e);
+    }
+    return c->ev_pool[c->ev_used++];
+}
+
+struct ProfScope {
+    wedlm_ctx* c;
+    int kind;
+    ProfScope(wedlm_ctx* c_, int kind_) : c(c_), kind(kind_) {
+        if (c->prof) {
+            c->ev_marks.emplace_back(kind, c->ev_used);
+            cudaEventRecord(prof_event(c), c->stream);
+        }
+        c->launches++;
+    }
+    ~ProfScope() {
+        if (c->prof) cudaEventRecord(prof_event(c), c->stream);
+    }
+};
+
+void prof_collect(wedlm_ctx* c) {
+    if (c->ev_marks.empty()) return;
+    cudaStreamSynchronize(c->stream);
+    for (auto& m : c->ev_marks) {
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, c->ev_pool[m.second], c->ev_pool[m.second + 1]);
+        c->prof_ms[m.first] += ms;
+        c->prof_n[m.first] += 1;
+    }
+    c->ev_marks.clear();
+    c->ev_used = 0;
 }
 
 #define CK(call)                                                                                  \
@@ -166,12 +211,12 @@ const CUtensorMap* xmap(wedlm_ctx* c, const void* p, uint64_t rows, uint64_t col
 }
 
 // Y[M][N] (fp32 partial planes in ws or `out`) = X[M][K] * W[N][K]^T.
-wedlm_status gemm(wedlm_ctx* ctx, const void* X, const void* W, const CUtensorMap* tmW, int M, int N, int K,
-                  float* out, size_t out_cap_floats, int* splits_out, int max_splits = 32) {
+wedlm_status gemm(wedlm_ctx* ctx, int kind, const void* X, const void* W, const CUtensorMap* tmW, int M, int N,
+                  int K, float* out, size_t out_cap_floats, int* splits_out, int max_splits = 32) {
     if (!ctx->bf16) {
         if ((size_t)M * N > out_cap_floats) return fail(ctx, WEDLM_ERR_STATE, "gemm workspace too small");
+        ProfScope ps(ctx, kind);
         launch_gemm_f32((const float*)X, (const float*)W, out, M, N, K, ctx->stream);
-        ctx->launches++;
         *splits_out = 1;
         return WEDLM_OK;
     }
@@ -187,9 +232,12 @@ wedlm_status gemm(wedlm_ctx* ctx, const void* X, const void* W, const CUtensorMa
     }
     const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
     if (!tx) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for activations");
-    cudaError_t e = launch_gemm_bf16(*tmW, *tx, out, M, N, K, p, ctx->err, ctx->stream);
+    cudaError_t e;
+    {
+        ProfScope ps(ctx, kind);
+        e = launch_gemm_bf16(*tmW, *tx, out, M, N, K, p, ctx->err, ctx->stream);
+    }
     if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("gemm launch: ") + cudaGetErrorString(e));
-    ctx->launches++;
     *splits_out = p.splits;
     return WEDLM_OK;
 }
@@ -242,46 +290,58 @@ wedlm_status forward_layers(wedlm_ctx* ctx, int slot_base, int n_entries, int st
     for (int l = 0; l < ctx->L; ++l) {
         int sp = 1;
         wedlm_status s;
-        s = gemm(ctx, h, ctx->wqkv[l], ctx->bf16 ? &ctx->tm_qkv[l] : nullptr, M, ctx->Nqkv, ctx->d, ctx->ws,
-                 ctx->ws_floats, &sp);
+        s = gemm(ctx, WEDLM_PROF_GEMM_QKV, h, ctx->wqkv[l], ctx->bf16 ? &ctx->tm_qkv[l] : nullptr, M, ctx->Nqkv,
+                 ctx->d, ctx->ws, ctx->ws_floats, &sp);
         if (s) return s;
-        launch_qkv_rope<T>(ctx->ws, sp, (int64_t)M * ctx->Nqkv, M, ctx->hq, ctx->hkv, ctx->hd, qb, (T*)ctx->kv_pool,
-                           ctx->kvl, l, ctx->rope_cs, ctx->max_ctx, ctx->rs, ctx->ss, rm, ctx->err, ctx->stream);
-        ctx->launches++;
+        {
+            ProfScope ps(ctx, WEDLM_PROF_QKV_ROPE);
+            launch_qkv_rope<T>(ctx->ws, sp, (int64_t)M * ctx->Nqkv, M, ctx->hq, ctx->hkv, ctx->hd, qb,
+                               (T*)ctx->kv_pool, ctx->kvl, l, ctx->rope_cs, ctx->max_ctx, ctx->rs, ctx->ss, rm,
+                               ctx->err, ctx->stream);
+        }
         if (ctx->bf16) {
             const int kc = decode ? ctx->attn_kv_chunk : (1 << 30);
             const int ms = decode ? ctx->attn_max_splits : 1;
-            launch_attn_bf16((const bf16*)qb, (const bf16*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd,
-                             (bf16*)ao, ctx->attn_po, ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss, rm, ctx->err,
-                             ctx->stream);
-            ctx->launches++;
+            {
+                ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
+                launch_attn_bf16((const bf16*)qb, (const bf16*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv,
+                                 ctx->hd, (bf16*)ao, ctx->attn_po, ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss,
+                                 rm, ctx->err, ctx->stream);
+            }
             if (ms > 1) {
+                ProfScope ps(ctx, WEDLM_PROF_ATTN_COMBINE);
                 launch_attn_combine(ctx->attn_po, ctx->attn_pml, (bf16*)ao, M, ctx->hq, ctx->hd, kc, ms, rt, ctx->ss,
                                     rm, ctx->stream);
-                ctx->launches++;
             }
         } else {
+            ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
             launch_attn_f32((const float*)qb, (const float*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd,
                             (float*)ao, M, ctx->ss, rm, ctx->err, ctx->stream);
-            ctx->launches++;
         }
-        s = gemm(ctx, ao, ctx->wo[l], ctx->bf16 ? &ctx->tm_o[l] : nullptr, M, ctx->d, ctx->hq * ctx->hd, ctx->ws,
-                 ctx->ws_floats, &sp);
+        s = gemm(ctx, WEDLM_PROF_GEMM_O, ao, ctx->wo[l], ctx->bf16 ? &ctx->tm_o[l] : nullptr, M, ctx->d,
+                 ctx->hq * ctx->hd, ctx->ws, ctx->ws_floats, &sp);
         if (s) return s;
-        launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, ctx->ffn_norm[l], eps, rm,
-                                ctx->stream);
-        ctx->launches++;
-        s = gemm(ctx, h, ctx->wgu[l], ctx->bf16 ? &ctx->tm_gu[l] : nullptr, M, 2 * ctx->F, ctx->d, ctx->ws,
-                 ctx->ws_floats, &sp);
+        {
+            ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
+            launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, ctx->ffn_norm[l], eps, rm,
+                                    ctx->stream);
+        }
+        s = gemm(ctx, WEDLM_PROF_GEMM_GATE_UP, h, ctx->wgu[l], ctx->bf16 ? &ctx->tm_gu[l] : nullptr, M, 2 * ctx->F,
+                 ctx->d, ctx->ws, ctx->ws_floats, &sp);
         if (s) return s;
-        launch_swiglu<T>(ctx->ws, sp, (int64_t)M * 2 * ctx->F, M, ctx->F, act, rm, ctx->stream);
-        ctx->launches++;
-        s = gemm(ctx, act, ctx->wd[l], ctx->bf16 ? &ctx->tm_d[l] : nullptr, M, ctx->d, ctx->F, ctx->ws,
-                 ctx->ws_floats, &sp);
+        {
+            ProfScope ps(ctx, WEDLM_PROF_SWIGLU);
+            launch_swiglu<T>(ctx->ws, sp, (int64_t)M * 2 * ctx->F, M, ctx->F, act, rm, ctx->stream);
+        }
+        s = gemm(ctx, WEDLM_PROF_GEMM_DOWN, act, ctx->wd[l], ctx->bf16 ? &ctx->tm_d[l] : nullptr, M, ctx->d, ctx->F,
+                 ctx->ws, ctx->ws_floats, &sp);
         if (s) return s;
         const float* gnext = (l + 1 < ctx->L) ? ctx->attn_norm[l + 1] : ctx->final_norm;
-        launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, gnext, eps, rm, ctx->stream);
-        ctx->launches++;
+        {
+            ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
+            launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, gnext, eps, rm,
+                                    ctx->stream);
+        }
     }
     return WEDLM_OK;
 }
@@ -305,31 +365,38 @@ int max_active_window(const wedlm_ctx* c, int* n_entries) {
 // Enqueue one decode step over slots [0, n_entries) with row stride `stride`.
 wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_entries, int stride) {
     const int M = n_entries * stride;
-    if (ctx->bf16)
-        launch_decode_prepare<bf16>((const bf16*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
-                                    ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
-                                    (bf16*)ctx->h, ctx->stream);
-    else
-        launch_decode_prepare<float>((const float*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
-                                     ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
-                                     (float*)ctx->h, ctx->stream);
-    ctx->launches++;
+    {
+        ProfScope ps(ctx, WEDLM_PROF_PREPARE);
+        if (ctx->bf16)
+            launch_decode_prepare<bf16>((const bf16*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
+                                        ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
+                                        (bf16*)ctx->h, ctx->stream);
+        else
+            launch_decode_prepare<float>((const float*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
+                                         ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
+                                         (float*)ctx->h, ctx->stream);
+    }
     wedlm_status s = run_forward(ctx, 0, n_entries, stride, true);
     if (s) return s;
     int lsp = 1;
-    s = gemm(ctx, ctx->h, ctx->lm_head, ctx->bf16 ? &ctx->tm_lm : nullptr, M, ctx->V, ctx->d, ctx->logits,
-             ctx->logits_floats, &lsp, 4);
+    s = gemm(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, ctx->lm_head, ctx->bf16 ? &ctx->tm_lm : nullptr, M, ctx->V,
+             ctx->d, ctx->logits, ctx->logits_floats, &lsp, 4);
     if (s) return s;
-    launch_entropy_partials(ctx->logits, lsp, (int64_t)M * ctx->V, ctx->V, ctx->V, ctx->cfg.mask_id, prm->logit_scale,
-                            ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream);
-    ctx->launches++;
+    {
+        ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
+        launch_entropy_partials(ctx->logits, lsp, (int64_t)M * ctx->V, ctx->V, ctx->V, ctx->cfg.mask_id,
+                                prm->logit_scale, ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream);
+    }
     StepKnobs kn{prm->lambda, prm->tau, prm->logit_scale, prm->tau_none};
-    launch_select_commit(ctx->ent_part, kEntropyChunks, ctx->ss, ctx->rs, n_entries, stride, kn, ctx->err,
-                         ctx->stream);
-    ctx->launches++;
+    {
+        ProfScope ps(ctx, WEDLM_PROF_SELECT);
+        launch_select_commit(ctx->ent_part, kEntropyChunks, ctx->ss, ctx->rs, n_entries, stride, kn, ctx->err,
+                             ctx->stream);
+    }
     ctx->last_stride = stride;
     ctx->last_M = M;
     ctx->logits_splits_last = lsp;
+    if (ctx->prof && ctx->ev_marks.size() > 4096) prof_collect(ctx);
     return WEDLM_OK;
 }
 
@@ -559,6 +626,7 @@ void wedlm_destroy(wedlm_ctx* ctx) {
     ctx->state_arena.release();
     ctx->scratch_arena.release();
     if (ctx->res_host) cudaFreeHost(ctx->res_host);
+    for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
     delete ctx;
 }
 
@@ -807,6 +875,27 @@ wedlm_status wedlm_get_stats(wedlm_ctx* ctx, int32_t slot, wedlm_seq_stats* out)
     out->end = ctx->h_end[slot];
     out->window = ctx->h_W[slot];
     out->active = (ctx->h_W[slot] > 0 && ctx->h_S[slot] < ctx->h_end[slot]) ? 1 : 0;
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_profile_enable(wedlm_ctx* ctx, int32_t on) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    prof_collect(ctx);
+    ctx->prof = on != 0;
+    for (int i = 0; i < WEDLM_PROF_KINDS; ++i) {
+        ctx->prof_ms[i] = 0.0;
+        ctx->prof_n[i] = 0;
+    }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_profile_read(wedlm_ctx* ctx, double* ms, int64_t* launches) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    prof_collect(ctx);
+    for (int i = 0; i < WEDLM_PROF_KINDS; ++i) {
+        if (ms) ms[i] = ctx->prof_ms[i];
+        if (launches) launches[i] = ctx->prof_n[i];
+    }
     return WEDLM_OK;
 }
 
