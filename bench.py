@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the batch-1 and regime sweeps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="headline measurement only (for profiler runs)")
+    ap.add_argument("--kernel-case", default=None,
+                    help="run one projection of the batch-16 step (gemm_qkv|gemm_o|gemm_gate_up|gemm_down|"
+                         "gemm_lm_head) three times through wedlm_linear_bf16 and exit (single-kernel captures)")
     return ap.parse_args()
 
 
@@ -451,9 +454,26 @@ def run_reference(a):
     print(json.dumps(line))
 
 
+def kernel_case(name: str):
+    import torch
+    from streaming_decoding_b200 import linear_bf16
+    cfg = synth.CONFIGS["qwen3_8b_b16"]
+    dims = cfg["model"]
+    L, M, N, K = gemm_shapes(dims, cfg["B"] * cfg["W"])[name]
+    g = torch.Generator(device="cuda").manual_seed(0)
+    X = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+    for _ in range(3):
+        linear_bf16(X, W)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_case": name, "M": M, "N": N, "K": K, "weight_bytes": 2 * N * K}))
+
+
 if __name__ == "__main__":
     args = parse()
-    if args.impl == "reference":
+    if args.kernel_case:
+        kernel_case(args.kernel_case)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
