@@ -613,6 +613,7 @@ __global__ void __launch_bounds__(64) select_only_kernel(const float4* __restric
     for (int j = threadIdx.x; j < kMaxWindow; j += blockDim.x) {
         const bool m = j < nb && !filled[(int64_t)b * stride + j];
         smask[j] = m ? 1 : 0;
+        sfill[j] = 0;
         sh[j] = NAN;
         sa[j] = -1;
         if (m) {
