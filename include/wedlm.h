@@ -291,6 +291,32 @@ wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t ma
                                   const wedlm_step_params* params,
                                   float* htilde, int32_t* argmax, uint8_t* fill, void* stream);
 
+/* Allocation-free wedlm_entropy_select.  (Not a step of the method: the
+ * paper has no counterpart.)  It exists for callers that must not allocate
+ * device memory: for example a runtime that has already reserved the device
+ * for its own memory pool, where any further allocation fails or fragments
+ * that pool, or a latency-critical thread that cannot risk the device
+ * synchronisation an allocation may cause.  Same arguments, outputs and
+ * device-pointer rules as wedlm_entropy_select; it allocates nothing.
+ *
+ * Its scratch is a fixed array inside the library image (about 1 MiB: room
+ * for WEDLM_NOALLOC_MAX_ROWS rows), present on every GPU that loads the
+ * library until the process exits.
+ *   - n_seq * stride must be <= WEDLM_NOALLOC_MAX_ROWS; larger requests
+ *     return WEDLM_ERR_INVALID_ARG without launching anything.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array, and it keeps the previous
+ *     call's contents (each call rewrites what it reads).  Calls whose work
+ *     overlaps on the GPU (different streams or host threads without ordering
+ *     between them) race on it and must be serialised by the caller. */
+#define WEDLM_NOALLOC_MAX_ROWS 4096
+wedlm_status wedlm_entropy_select_noalloc(const float* logits, int32_t vocab, int32_t mask_id,
+                                          const uint8_t* filled, const int32_t* n, int32_t n_seq, int32_t stride,
+                                          const wedlm_step_params* params,
+                                          float* htilde, int32_t* argmax, uint8_t* fill, void* stream);
+
 /* Dense projection on the bf16 tensor-core path: Y = X * W^T with X bf16
  * [M][K], W bf16 [N][K] (nn.Linear layout), Y fp32 [M][N], all DEVICE
  * pointers owned by the caller (16-byte aligned; K % 8 == 0).  This is the

@@ -2,4 +2,4 @@
 
 The decode step runs in libwedlm.so (CUDA kernels behind the C ABI declared in
 include/wedlm.h); ``api`` is its Python binding."""
-from .api import Engine, step_params, reorder_window, entropy_select, linear_bf16  # noqa: F401
+from .api import Engine, step_params, reorder_window, entropy_select, entropy_select_noalloc, linear_bf16  # noqa: F401,E501

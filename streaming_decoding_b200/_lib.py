@@ -72,6 +72,8 @@ _SIGS = {
     "wedlm_reorder_window": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "wedlm_entropy_select": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_i32, ctypes.POINTER(StepParams),
                                      c_vp, c_vp, c_vp, c_vp]),
+    "wedlm_entropy_select_noalloc": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_i32,
+                                             ctypes.POINTER(StepParams), c_vp, c_vp, c_vp, c_vp]),
     "wedlm_linear_bf16": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp]),
 }
 

@@ -219,6 +219,21 @@ def entropy_select(logits, vocab: int, mask_id: int, filled, n, stride: int, par
     return ht, am, fill
 
 
+def entropy_select_noalloc(logits, vocab: int, mask_id: int, filled, n, stride: int, params: StepParams,
+                           stream=None):
+    """entropy_select without any device allocation (scratch in a fixed library array)."""
+    import torch
+    n_seq = filled.shape[0]
+    dev = logits.device
+    ht = torch.empty((n_seq, stride), dtype=torch.float32, device=dev)
+    am = torch.empty((n_seq, stride), dtype=torch.int32, device=dev)
+    fill = torch.empty((n_seq, stride), dtype=torch.uint8, device=dev)
+    _check(_lib.load().wedlm_entropy_select_noalloc(_ptr(logits), vocab, mask_id, _ptr(filled), _ptr(n), n_seq,
+                                                    stride, ctypes.byref(params), _ptr(ht), _ptr(am), _ptr(fill),
+                                                    _stream_handle(stream)), "wedlm_entropy_select_noalloc")
+    return ht, am, fill
+
+
 def linear_bf16(X, W, stream=None):
     """Y = X W^T (fp32) on the tcgen05 GEMM; X [M][K], W [N][K] torch.bfloat16 CUDA tensors."""
     import torch
