@@ -49,7 +49,8 @@ def parse():
     ap.add_argument("--quick", action="store_true", help="headline measurement only (for profiler runs)")
     ap.add_argument("--kernel-case", default=None,
                     help="run one projection of the batch-16 step (gemm_qkv|gemm_o|gemm_gate_up|gemm_down|"
-                         "gemm_lm_head) three times through wedlm_linear_bf16 and exit (single-kernel captures)")
+                         "gemm_lm_head) three times through wedlm_linear_bf16, or 'attention' (3 decode steps of "
+                         "a 2-layer model with the batch-16 shapes), and exit (single-kernel captures)")
     return ap.parse_args()
 
 
@@ -347,7 +348,8 @@ def run_ours(a):
              "step_ms_floor_algorithmic": round(step_floor_ms, 3),
              "step_roofline_frac": round(step_floor_ms / (ms / a.steps), 4),
              "profile_ms_per_step": {k: round(v[0] / 10, 4) for k, v in prof.items() if v[1]},
-             "e2e_wall_s": round(e_wall, 3)}
+             "e2e_wall_s": round(e_wall, 3),
+             "gemm_plans_rows%d" % (B * W): {k: rep.eng.gemm_plan(k, B * W) for k in gemm_shapes(dims, M)}}
     if not a.quick and not a.no_extra and world == 1:
         extra.update(sweeps(rep, cfg, a))
     cpu = None
@@ -389,7 +391,8 @@ def sweeps(rep, cfg, a):
     rep.eng.stream_step_async(prm, a.warmup)
     ms, com, _ = rep.timed_async(prm, steps, 1)
     out["batch1"] = {"workload": workload_desc(b1, "qwen3_8b_b1"), "tok_per_s": round(com / (ms / 1e3), 2),
-                     "ms_per_step": round(ms / steps, 4), "committed_per_step": round(com / steps, 3)}
+                     "ms_per_step": round(ms / steps, 4), "committed_per_step": round(com / steps, 3),
+                     "gemm_plans_rows16": {k: rep.eng.gemm_plan(k, b1["W"]) for k in gemm_shapes(rep.dims, 16)}}
     reg = {}
     prompts = synth.prompts(cfg)
     for scale in cfg["logit_scales"]:
@@ -454,9 +457,70 @@ def run_reference(a):
     print(json.dumps(line))
 
 
+def attention_case(steps: int = 3):
+    """Decode steps of a 2-layer model with the Qwen3-8B head layout on the
+    batch-16 prompts (same attention shapes per layer as the full model, a few
+    GB on the device): the case for single-kernel captures of the attention."""
+    import torch
+    from streaming_decoding_b200 import Engine, step_params
+    cfg = dict(synth.CONFIGS["qwen3_8b_b16"])
+    dims = dict(cfg["model"], L=2)
+    eng = Engine(dims, max_batch=cfg["B"], max_window=cfg["W"], max_ctx=1024 + cfg["N"])
+    eng.load_model(synth.iter_weights(dims, seed=0, dtype="bf16"))
+    for b, p in enumerate(synth.prompts(cfg)):
+        eng.prefill(b, p, cfg["N"], cfg["W"])
+    eng.stream_step_async(step_params(cfg["lam"], cfg["tau"], False, cfg["logit_scale"]), steps)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_case": "attention", "layers": 2, "batch": cfg["B"], "steps": steps,
+                      "prefill_attention_launches": cfg["B"] * 2}))
+
+
+def gemm_sweep():
+    """Time every projection shape of the batch-16 and batch-1 steps under each
+    (tile width, K split) choice and under the automatic plan (CUDA events)."""
+    import torch
+    from streaming_decoding_b200 import linear_bf16
+    cfg = synth.CONFIGS["qwen3_8b_b16"]
+    dims = cfg["model"]
+    g = torch.Generator(device="cuda").manual_seed(0)
+    out = []
+    for M in (256, 16):
+        X = torch.randn(M, max(dims["F"], dims["d"]), device="cuda", generator=g).to(torch.bfloat16)
+        for name, (_, _, N, K) in gemm_shapes(dims, M).items():
+            W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+            Xk = X[:, :K].contiguous()
+            bns = [0] + ([256, 128] if M > 128 else [16])
+            res = []
+            for bn in bns:
+                for sp in ([0] if bn == 0 else [1, 2, 3, 4, 6, 8]):
+                    for _ in range(2):
+                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp)
+                    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    st.record()
+                    for _ in range(10):
+                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp)
+                    en.record()
+                    en.synchronize()
+                    us = st.elapsed_time(en) * 100.0
+                    res.append({"bn": bn, "splits": sp, "us": round(us, 2),
+                                "weight_GBps": round(2 * N * K / us / 1e3, 1),
+                                "TFLOPs": round(2 * M * N * K / us / 1e6, 1)})
+            del W
+            best = min(res[1:], key=lambda r: r["us"])
+            out.append({"M": M, "gemm": name, "N": N, "K": K, "auto": res[0], "best": best, "all": res})
+            print(json.dumps({"M": M, "gemm": name, "auto_us": res[0]["us"], "best": best}), flush=True)
+    with open(os.path.join(ROOT, "gpurun_out", "gemm_sweep.json") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else os.devnull, "w") as f:
+        json.dump(out, f, indent=1)
+
+
 def kernel_case(name: str):
     import torch
     from streaming_decoding_b200 import linear_bf16
+    if name == "attention":
+        return attention_case()
+    if name == "gemm_sweep":
+        return gemm_sweep()
     cfg = synth.CONFIGS["qwen3_8b_b16"]
     dims = cfg["model"]
     L, M, N, K = gemm_shapes(dims, cfg["B"] * cfg["W"])[name]

@@ -220,6 +220,21 @@ wedlm_status wedlm_kernel_launches(const wedlm_ctx* ctx, int64_t* out);
 #define WEDLM_PROF_SELECT       12
 #define WEDLM_PROF_KINDS        13
 
+/* bf16 GEMM launch shapes.  With autotuning on (the default), the first time a
+ * projection kind (WEDLM_PROF_GEMM_*) runs at a given row count the context
+ * times each candidate shape (activation rows per tile, K slices) on that
+ * projection's weights with a plain store into scratch, on its own stream,
+ * and keeps the fastest for the rest of its life; off, a fixed cost model
+ * picks the shape.  Results depend on the shape only through fp32
+ * accumulation order.  wedlm_autotune clears the recorded shapes. */
+wedlm_status wedlm_autotune(wedlm_ctx* ctx, int32_t enable);
+
+/* The shape recorded for (kind, rows): tile_n activation rows per tile,
+ * k_splits slices of K, and the fastest timed launch in microseconds (-1 when
+ * the shape came from the cost model).  WEDLM_ERR_STATE if none is recorded. */
+wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_n, int32_t* k_splits,
+                             float* us);
+
 /* Enable (1) or disable (0) per-kernel timing; enabling clears the totals. */
 wedlm_status wedlm_profile_enable(wedlm_ctx* ctx, int32_t on);
 
@@ -324,6 +339,14 @@ wedlm_status wedlm_entropy_select_noalloc(const float* logits, int32_t vocab, in
  * (split-K partial planes are summed before returning). */
 wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
                                void* stream);
+
+/* wedlm_linear_bf16 with the launch shape pinned (tuning and test hook):
+ * tile_n in {16, 32, 64, 128, 256} activation rows per tile (0 = automatic) and
+ * k_splits in [1, 16] slices of K (0 = automatic; rounded to what K allows and
+ * forced to 1 when N % 4 != 0).  Results agree with the automatic plan to fp32
+ * accumulation order. */
+wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                    int32_t tile_n, int32_t k_splits, void* stream);
 
 #ifdef __cplusplus
 }

@@ -64,6 +64,8 @@ _SIGS = {
     "wedlm_get_stats": (c_i32, [c_vp, c_i32, ctypes.POINTER(SeqStats)]),
     "wedlm_kernel_launches": (c_i32, [c_vp, ctypes.POINTER(c_i64)]),
     "wedlm_profile_enable": (c_i32, [c_vp, c_i32]),
+    "wedlm_autotune": (c_i32, [c_vp, c_i32]),
+    "wedlm_gemm_plan": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp]),
     "wedlm_profile_read": (c_i32, [c_vp, c_vp, c_vp]),
     "wedlm_debug_read": (c_i32, [c_vp, c_i32, c_vp, c_i64]),
     "wedlm_debug_kv": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp]),
@@ -75,6 +77,7 @@ _SIGS = {
     "wedlm_entropy_select_noalloc": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_i32,
                                              ctypes.POINTER(StepParams), c_vp, c_vp, c_vp, c_vp]),
     "wedlm_linear_bf16": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp]),
+    "wedlm_linear_bf16_plan": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]),
 }
 
 _lib = None

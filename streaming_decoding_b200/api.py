@@ -137,6 +137,16 @@ class Engine:
         _check(self.lib.wedlm_kernel_launches(self.ctx, ctypes.byref(n)), "wedlm_kernel_launches")
         return n.value
 
+    def autotune(self, enable: bool = True):
+        _check(self.lib.wedlm_autotune(self.ctx, 1 if enable else 0), "wedlm_autotune", self.ctx)
+
+    def gemm_plan(self, kind: str, rows: int):
+        """(tile_n, k_splits, us) recorded for a projection kind ('gemm_qkv', ...) at `rows`, or None."""
+        tn, ks, us = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_float()
+        st = self.lib.wedlm_gemm_plan(self.ctx, C["WEDLM_PROF_" + kind.upper()], rows, ctypes.byref(tn),
+                                      ctypes.byref(ks), ctypes.byref(us))
+        return (tn.value, ks.value, round(us.value, 2)) if st == 0 else None
+
     def profile_enable(self, on: bool = True):
         _check(self.lib.wedlm_profile_enable(self.ctx, 1 if on else 0), "wedlm_profile_enable", self.ctx)
 
@@ -234,12 +244,14 @@ def entropy_select_noalloc(logits, vocab: int, mask_id: int, filled, n, stride: 
     return ht, am, fill
 
 
-def linear_bf16(X, W, stream=None):
-    """Y = X W^T (fp32) on the tcgen05 GEMM; X [M][K], W [N][K] torch.bfloat16 CUDA tensors."""
+def linear_bf16(X, W, stream=None, tile_n: int = 0, k_splits: int = 0):
+    """Y = X W^T (fp32) on the tcgen05 GEMM; X [M][K], W [N][K] torch.bfloat16 CUDA tensors.
+    tile_n / k_splits pin the launch shape (0 = automatic)."""
     import torch
     M, K = X.shape
     N = W.shape[0]
     Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
-    _check(_lib.load().wedlm_linear_bf16(_ptr(X.contiguous()), _ptr(W.contiguous()), _ptr(Y), M, N, K,
-                                         _stream_handle(stream)), "wedlm_linear_bf16")
+    X, W = X.contiguous(), W.contiguous()
+    _check(_lib.load().wedlm_linear_bf16_plan(_ptr(X), _ptr(W), _ptr(Y), M, N, K, tile_n, k_splits,
+                                              _stream_handle(stream)), "wedlm_linear_bf16_plan")
     return Y

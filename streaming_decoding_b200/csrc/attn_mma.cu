@@ -10,9 +10,10 @@
 // One CTA owns (batch entry, KV head, tile of RT window rows, key split).  Its
 // query rows are the RT rows times the g = hq/hkv query heads sharing the KV
 // head (g*RT <= 16*NW; one warp per 16 query rows), so every K/V byte loaded
-// serves all g heads.  Keys stream through shared memory in 64-key blocks (4
-// pages) with cp.async double buffering and an XOR swizzle of 16-byte chunks
-// that keeps ldmatrix conflict-free.  Online softmax in the exp2 domain.
+// serves all g heads.  The CTA's slice of the page table is staged in shared
+// memory; keys stream through a 3-stage cp.async ring of 64-key blocks (4
+// pages) with an XOR swizzle of 16-byte chunks that keeps ldmatrix
+// conflict-free.  Online softmax in the exp2 domain.
 // With more than one key split, unnormalised partial outputs plus (max, sum)
 // go to a workspace and attn_combine_kernel merges them.
 #include "kernels.cuh"
@@ -24,6 +25,8 @@ constexpr int HD = 128;
 constexpr int KBLK = 64;
 constexpr int CHUNKS = HD / 8;              // 16-byte chunks per key row
 constexpr int TILE_BYTES = KBLK * HD * 2;   // one K or V block in shared memory
+constexpr int ASTAGES = 3;                  // K/V blocks in flight per CTA
+constexpr int MAX_PAGES_SMEM = 2048;        // page-table entries staged per CTA (32k keys)
 
 __device__ __forceinline__ uint32_t swz(int key, int chunk) {
     return (uint32_t)(key * (HD * 2) + (((chunk ^ (key & 7))) << 4));
@@ -73,8 +76,11 @@ struct AttnParams {
     int* err;
 };
 
+// Issue cp.async copies of keys [kb0, kb0 + 64) (rows past ke zero-filled)
+// into one K and one V stage; pages come from the CTA's staged page list.
 __device__ __forceinline__ void load_kv_block(uint32_t sK, uint32_t sV, const AttnParams& p, int kvh,
-                                              const int32_t* pt, int kb0, int ke, int nthreads) {
+                                              const int32_t* spages, int page0, int npages, int kb0, int ke,
+                                              int nthreads) {
     for (int i = threadIdx.x; i < KBLK * CHUNKS; i += nthreads) {
         const int key = i / CHUNKS, ch = i - key * CHUNKS;
         const int t = kb0 + key;
@@ -82,8 +88,8 @@ __device__ __forceinline__ void load_kv_block(uint32_t sK, uint32_t sV, const At
         const bf16* srcV = p.kv_pool;
         int bytes = 0;
         if (t < ke) {
-            const int pidx = t / kPage;
-            const int page = pidx < p.ss.pages_per_seq ? pt[pidx] : -1;
+            const int pi = t / kPage - page0;
+            const int page = (pi >= 0 && pi < npages) ? spages[pi] : -1;
             if (page >= 0 && page < p.kvl.num_pages) {
                 const int64_t o = (int64_t)(t % kPage) * HD + ch * 8;
                 srcK = p.kv_pool + p.kvl.page_base(p.layer, page, 0, kvh) + o;
@@ -150,23 +156,38 @@ __global__ void __launch_bounds__(NW * 32) attn_bf16_kernel(const AttnParams p) 
     float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
     const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
 
+    // stage this CTA's slice of the page table in shared memory
+    int32_t* spages = reinterpret_cast<int32_t*>(smem + ASTAGES * 2 * TILE_BYTES);
+    const int page0 = ks / kPage;
+    const int npages = min((ke + kPage - 1) / kPage - page0, MAX_PAGES_SMEM);
+    for (int i = threadIdx.x; i < npages; i += NW * 32)
+        spages[i] = (page0 + i < p.ss.pages_per_seq) ? pt[page0 + i] : -1;
+    __syncthreads();
+
     const uint32_t sbase = smem_u32(smem);
     const int nblk = (ke - ks + KBLK - 1) / KBLK;
-    load_kv_block(sbase, sbase + TILE_BYTES, p, kvh, pt, ks, ke, NW * 32);
-    cp_async_commit();
+#pragma unroll
+    for (int st = 0; st < ASTAGES - 1; ++st) {
+        if (st < nblk) {
+            const uint32_t sK = sbase + st * 2 * TILE_BYTES;
+            load_kv_block(sK, sK + TILE_BYTES, p, kvh, spages, page0, npages, ks + st * KBLK, ke, NW * 32);
+        }
+        cp_async_commit();
+    }
     for (int b = 0; b < nblk; ++b) {
         const int kb0 = ks + b * KBLK;
-        const uint32_t sK = sbase + (b & 1) * 2 * TILE_BYTES;
-        const uint32_t sV = sK + TILE_BYTES;
-        if (b + 1 < nblk) {
-            const uint32_t nK = sbase + ((b + 1) & 1) * 2 * TILE_BYTES;
-            load_kv_block(nK, nK + TILE_BYTES, p, kvh, pt, kb0 + KBLK, ke, NW * 32);
+        {
+            const int nb = b + ASTAGES - 1;
+            if (nb < nblk) {
+                const uint32_t nK = sbase + (nb % ASTAGES) * 2 * TILE_BYTES;
+                load_kv_block(nK, nK + TILE_BYTES, p, kvh, spages, page0, npages, ks + nb * KBLK, ke, NW * 32);
+            }
             cp_async_commit();
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
         }
+        cp_async_wait<ASTAGES - 1>();
         __syncthreads();
+        const uint32_t sK = sbase + (b % ASTAGES) * 2 * TILE_BYTES;
+        const uint32_t sV = sK + TILE_BYTES;
 
         // S = Q K^T for 64 keys: 8 key tiles of 8.
         float s[8][4];
@@ -324,7 +345,7 @@ void launch_attn_bf16(const bf16* q, const bf16* kv_pool, KVLayout kvl, int laye
                  attn_rows_per_tile(g), ss, rm, err};
     const int tiles = (stride + p.rt - 1) / p.rt;
     dim3 grid(tiles, hkv, n_entries * max_splits);
-    const int smem = 4 * TILE_BYTES;
+    const int smem = ASTAGES * 2 * TILE_BYTES + MAX_PAGES_SMEM * 4;
     if (attn_warps(g) == 4) {
         static bool set4 = false;
         if (!set4) {

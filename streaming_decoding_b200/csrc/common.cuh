@@ -96,6 +96,20 @@ struct RowState {
     int32_t* perm;     // [Mmax] slot offset (decode) / r (prefill)
 };
 
+// Which rows of a forward belong to which slot: row = entry * stride + r,
+// slot = slot_base + entry, row is live iff r < n[slot].
+struct RowMap {
+    int slot_base;
+    int stride;
+    const int32_t* n;
+    __device__ __forceinline__ bool live(int row, int& slot, int& r) const {
+        const int e = row / stride;
+        r = row - e * stride;
+        slot = slot_base + e;
+        return r < n[slot];
+    }
+};
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -1,23 +1,30 @@
-// bf16 GEMM on tcgen05 tensor cores with TMA-fed shared-memory stages.
+// Persistent bf16 GEMM on tcgen05 tensor cores, TMA-fed, with fused epilogues.
 //
-// Y[M][N] = X[M][K] * W[N][K]^T for the dense projections (QKV, O, gate/up,
-// down) and the LM head.  In decoding, M (window rows of the batch) is small
-// (16..256) and N, K are the model's widths, so the kernel is laid out
-// "swap-AB": the 128-row MMA M side is taken by the weights and the MMA N
-// side by the activation rows.  Each CTA streams its weight tiles exactly once
-// from HBM; the step is bound by weight bytes until M approaches the
-// machine-balance point (about 250 rows), where it becomes tensor bound.
+// Y[M][N] = X[M][K] * W[N][K]^T for every dense projection of the step (QKV,
+// O, gate/up, down) and the LM head.  In decoding M (window rows of the
+// batch) is small, so the layout is "swap-AB": the 128-row MMA M side holds
+// weight rows, the MMA N side (bn = 16..256) holds activation rows.  Every
+// weight byte is read from HBM exactly once per launch; the kernel is bound by
+// weight bytes until M nears the machine-balance point (~250 rows).
 //
-// Warp roles (192 threads):
-//   warp 0      one elected thread issues TMA loads of A (weights, 128 x 64)
-//               and B (activations, bn x 64) into a STAGES-deep ring,
-//   warp 1      allocates TMEM and one elected thread issues tcgen05.mma
-//               (kind::f16, bf16 inputs, fp32 accumulate in TMEM), releasing
-//               each stage back to the producer with tcgen05.commit,
-//   warps 2..5  epilogue: tcgen05.ld the 128 x bn fp32 accumulator (warp w
-//               owns TMEM lanes 32*(w%4) .. +31) and store it row-major.
-// Every mbarrier wait is bounded; on timeout the kernel records an error and
-// unwinds (frees TMEM) instead of hanging.
+// One CTA per SM loops over work units (tile, K slice).  Warp roles (192
+// threads):
+//   warp 0      one thread issues TMA loads of A (weights, 128 x 64) and B
+//               (activations, bn x 64) into a STAGES-deep shared-memory ring
+//               that runs continuously across units,
+//   warp 1      allocates TMEM (two bn-column accumulators) and one thread
+//               issues tcgen05.mma (kind::f16, fp32 accumulation), releasing
+//               ring stages with tcgen05.commit; it alternates accumulators so
+//               the next unit's MMAs overlap the previous unit's epilogue,
+//   warps 2..5  epilogue: tcgen05.ld 16 columns at a time (warp w owns TMEM
+//               lanes 32*(w%4)..+31), then either the fused epilogue directly
+//               or, for K split over several CTAs, a partial plane; the CTAs
+//               of a tile (same round, co-resident by cooperative launch) wait
+//               for each other and each reduces a slice of the tile's rows in
+//               fixed split order (deterministic), then applies the epilogue.
+// Every mbarrier wait is bounded; on timeout the kernel records an error in
+// the device error word and unwinds (freeing TMEM) instead of hanging.
+#include <algorithm>
 #include <cmath>
 
 #include <cudaTypedefs.h>
@@ -31,11 +38,27 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 
-template <int BN> struct TileCfg {
+template <int BN> struct PCfg {
     static constexpr int B_STAGE_BYTES = BN * BK * 2;
-    static constexpr int STAGES = BN <= 32 ? 5 : (BN <= 64 ? 4 : (BN <= 128 ? 6 : 4));
-    static constexpr int TMEM_COLS = BN <= 32 ? 32 : BN;
-    static constexpr int SMEM_BYTES = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 12 ? 12 : (200 * 1024) / STAGE_BYTES;
+    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    static constexpr int META_BYTES = BN * 16;  // per activation row: live, pos, cache-row offset
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + META_BYTES;
+};
+
+// What the epilogue needs per activation row of the current unit, computed
+// once per unit into shared memory so the element loops issue their global
+// loads in batches (no load waits behind a store of the previous element).
+struct RowMeta {
+    int live;      // row < M and not padding
+    int pos;       // logical position (RoPE)
+    long long kv;  // element offset of (layer, page, K, head 0, token) in the pool; -1 if out of range
+};
+
+struct GemmArgs {
+    int M, N, K, kb_per_split, splits, n_tiles, m_tiles;
+    EpiParams ep;
 };
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -44,6 +67,10 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
@@ -87,22 +114,219 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+// 16 consecutive fp32 accumulator columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Barrier over the four epilogue warps that also ANDs a predicate across them,
+// so they leave the unit loop together (every wait before it is bounded).
+__device__ __forceinline__ bool epi_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+
+// Fill meta[0..BN) for activation rows m0..m0+BN-1 (the 128 epilogue threads).
+template <int BN>
+__device__ __forceinline__ void fill_row_meta(const EpiParams& ep, int m0, int M, RowMeta* meta, int et) {
+    for (int k = et; k < BN; k += 128) {
+        const int m = m0 + k;
+        RowMeta rmeta{0, 0, -1};
+        int slot = 0, r = m;
+        if (m < M && (!ep.check_rows || ep.rm.live(m, slot, r))) {
+            rmeta.live = 1;
+            if (ep.kind == EPI_QKV_ROPE) {
+                const int pos = __ldg(ep.rs.pos + m);
+                if (pos < 0 || pos >= ep.rope_max_pos) {
+                    set_error(ep.err, kErrBounds);
+                    rmeta.live = 0;
+                } else {
+                    rmeta.pos = pos;
+                    const int p = __ldg(ep.ss.S + slot) + r;
+                    const int pidx = p / kPage;
+                    const int page = pidx < ep.ss.pages_per_seq
+                                         ? __ldg(ep.ss.page_table + (int64_t)slot * ep.ss.pages_per_seq + pidx)
+                                         : -1;
+                    if (page < 0 || page >= ep.kvl.num_pages) {
+                        set_error(ep.err, kErrBounds);
+                    } else {
+                        rmeta.kv = ep.kvl.page_base(ep.layer, page, 0, 0) + (int64_t)(p % kPage) * 128;
+                    }
+                }
+            }
+        }
+        meta[k] = rmeta;
+    }
+}
+
+// Destination of dim `dim` of QKV head `head` for a row (q buffer or pages).
+__device__ __forceinline__ bf16* qkv_dst(const EpiParams& ep, int head, int m, const RowMeta& rm) {
+    if (head < ep.hq) return ep.act + ((int64_t)m * ep.hq + head) * 128;
+    if (rm.kv < 0) return nullptr;
+    const int kv = head < ep.hq + ep.hkv ? 0 : 1;
+    const int h = head - ep.hq - kv * ep.hkv;
+    return ep.kv_pool + rm.kv + (int64_t)(kv * ep.hkv + h) * (kPage * 128);
+}
+
+// Fused epilogue on 16 accumulator columns (activation rows mbase..mbase+15,
+// meta rows kbase..kbase+15) of weight row n held by this thread; row pairs
+// (n even, n odd) sit in adjacent lanes.
+__device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, int mbase, int kbase,
+                                           const RowMeta* meta, const float (&v)[16], int N, int lane) {
+    int live[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) live[k] = meta[kbase + k].live && n < N;
+    switch (ep.kind) {
+        case EPI_STORE:
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (live[k]) ep.out[(int64_t)(mbase + k) * N + n] = v[k];
+            break;
+        case EPI_RESIDUAL: {
+            float x[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) x[k] = live[k] ? ep.out[(int64_t)(mbase + k) * N + n] : 0.f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (live[k]) ep.out[(int64_t)(mbase + k) * N + n] = x[k] + v[k];
+            break;
+        }
+        case EPI_SWIGLU: {
+            const int F = N >> 1;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float partner = __shfl_xor_sync(0xffffffffu, v[k], 1);
+                if (!(lane & 1) && live[k])
+                    ep.act[(int64_t)(mbase + k) * F + (n >> 1)] =
+                        __float2bfloat16_rn(v[k] / (1.0f + expf(-v[k])) * partner);
+            }
+            break;
+        }
+        case EPI_QKV_ROPE: {
+            const int head = n0 >> 7;
+            const int t = n - n0;
+            const bool rot = head < ep.hq + ep.hkv;
+            const int i = t >> 1, odd = t & 1;
+            const int dim = rot ? (odd ? i + 64 : i) : t;
+            float2 cs[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                cs[k] = (rot && live[k]) ? __ldg(ep.rope_cs + (int64_t)meta[kbase + k].pos * 64 + i)
+                                         : make_float2(1.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float partner = rot ? __shfl_xor_sync(0xffffffffu, v[k], 1) : 0.f;
+                if (!live[k]) continue;
+                float val = v[k];
+                if (rot) {
+                    const float a = odd ? partner : val, b = odd ? val : partner;
+                    val = odd ? (b * cs[k].x + a * cs[k].y) : (a * cs[k].x - b * cs[k].y);
+                }
+                bf16* dst = qkv_dst(ep, head, mbase + k, meta[kbase + k]);
+                if (dst) dst[dim] = __float2bfloat16_rn(val);
+            }
+            break;
+        }
+        default: break;
+    }
+}
+
+// Fused epilogue on weight rows n..n+3 (both row pairs inside this thread) of
+// eight activation rows m = mrow[u], after a split-K reduction.
+__device__ __forceinline__ void epilogue_vec4x8(const EpiParams& ep, int n0, int n, const int (&mrow)[8],
+                                                const int (&krow)[8], const bool (&ok)[8], const RowMeta* meta,
+                                                const float4 (&v)[8], int N) {
+    bool live[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) live[u] = ok[u] && meta[krow[u]].live;
+    switch (ep.kind) {
+        case EPI_STORE:
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (live[u]) *reinterpret_cast<float4*>(ep.out + (int64_t)mrow[u] * N + n) = v[u];
+            break;
+        case EPI_RESIDUAL: {
+            float4 x[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                x[u] = live[u] ? *reinterpret_cast<const float4*>(ep.out + (int64_t)mrow[u] * N + n)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (live[u])
+                    *reinterpret_cast<float4*>(ep.out + (int64_t)mrow[u] * N + n) =
+                        make_float4(x[u].x + v[u].x, x[u].y + v[u].y, x[u].z + v[u].z, x[u].w + v[u].w);
+            break;
+        }
+        case EPI_SWIGLU: {
+            const int F = N >> 1;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (live[u]) {
+                    const float a = v[u].x / (1.0f + expf(-v[u].x)) * v[u].y;
+                    const float b = v[u].z / (1.0f + expf(-v[u].z)) * v[u].w;
+                    *reinterpret_cast<__nv_bfloat162*>(ep.act + (int64_t)mrow[u] * F + (n >> 1)) =
+                        __floats2bfloat162_rn(a, b);
+                }
+            break;
+        }
+        case EPI_QKV_ROPE: {
+            const int head = n0 >> 7;
+            const int t = n - n0;
+            const bool rot = head < ep.hq + ep.hkv;
+            const int i = t >> 1;
+            float2 c0[8], c1[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t base = (int64_t)meta[krow[u]].pos * 64 + i;
+                c0[u] = (rot && live[u]) ? __ldg(ep.rope_cs + base) : make_float2(1.f, 0.f);
+                c1[u] = (rot && live[u]) ? __ldg(ep.rope_cs + base + 1) : make_float2(1.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (!live[u]) continue;
+                bf16* dst = qkv_dst(ep, head, mrow[u], meta[krow[u]]);
+                if (!dst) continue;
+                if (rot) {
+                    // rows (t, t+1) = dims (i, i+64); rows (t+2, t+3) = dims (i+1, i+65)
+                    const float d0 = v[u].x * c0[u].x - v[u].y * c0[u].y;
+                    const float d2 = v[u].y * c0[u].x + v[u].x * c0[u].y;
+                    const float d1 = v[u].z * c1[u].x - v[u].w * c1[u].y;
+                    const float d3 = v[u].w * c1[u].x + v[u].z * c1[u].y;
+                    *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(d0, d1);
+                    *reinterpret_cast<__nv_bfloat162*>(dst + i + 64) = __floats2bfloat162_rn(d2, d3);
+                } else {
+                    *reinterpret_cast<__nv_bfloat162*>(dst + t) = __floats2bfloat162_rn(v[u].x, v[u].y);
+                    *reinterpret_cast<__nv_bfloat162*>(dst + t + 2) = __floats2bfloat162_rn(v[u].z, v[u].w);
+                }
+            }
+            break;
+        }
+        default: break;
+    }
 }
 
 template <int BN>
-__global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmW,
-                                                              const __grid_constant__ CUtensorMap tmX,
-                                                              float* __restrict__ out, int M, int N, int K,
-                                                              int kb_per_split, int* err) {
-    using C = TileCfg<BN>;
+__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
+                                                         const __grid_constant__ CUtensorMap tmX, const GemmArgs g) {
+    using C = PCfg<BN>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -110,14 +334,15 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
     uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE_BYTES);
     uint64_t* empty = full + STAGES;
-    uint64_t* accum = empty + STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+    uint64_t* accf = empty + STAGES;
+    uint64_t* acce = accf + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+    RowMeta* meta = reinterpret_cast<RowMeta*>(smem + STAGES * C::STAGE_BYTES + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BM, m0 = blockIdx.y * BN, split = blockIdx.z;
-    const int KB = (K + BK - 1) / BK;
-    const int kb0 = split * kb_per_split;
-    const int nkb = min(KB, kb0 + kb_per_split) - kb0;
+    const int KB = (g.K + BK - 1) / BK;
+    const int units = g.n_tiles * g.m_tiles * g.splits;
+    int* err = g.ep.err;
 
     if (threadIdx.x == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
@@ -126,7 +351,10 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 4);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -141,62 +369,174 @@ __global__ void __launch_bounds__(192, 1) gemm_bf16_tc_kernel(const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (nkb > 0) {
-        if (warp == 0) {
-            if (lane == 0) {
-                for (int i = 0; i < nkb; ++i) {
-                    const int s = i % STAGES;
-                    const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-                    if (!mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1u, err)) break;
-                    mbar_expect_tx(&full[s], A_STAGE_BYTES + C::B_STAGE_BYTES);
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int split = u % g.splits, tile = u / g.splits;
+                const int n0 = (tile / g.m_tiles) * BM, m0 = (tile % g.m_tiles) * BN;
+                const int kb0 = split * g.kb_per_split;
+                const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
+                for (int i = 0; i < nkb; ++i, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1u, err)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(&full[s], C::STAGE_BYTES);
                     const int kx = (kb0 + i) * BK;
                     tma_load_2d(sA + s * A_STAGE_BYTES, &tmW, kx, n0, &full[s]);
                     tma_load_2d(sB + s * C::B_STAGE_BYTES, &tmX, kx, m0, &full[s]);
                 }
             }
-        } else if (warp == 1) {
-            if (lane == 0) {
-                constexpr uint32_t idesc = idesc_bf16(BM, BN);
-                for (int i = 0; i < nkb; ++i) {
-                    const int s = i % STAGES;
-                    const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-                    if (!mbar_wait_bounded(smem_u32(&full[s]), ph, err)) break;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(BM, BN);
+            uint32_t it = 0, j = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++j) {
+                const int split = u % g.splits;
+                const int kb0 = split * g.kb_per_split;
+                const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
+                const uint32_t b = j & 1u, use = j >> 1;
+                if (!mbar_wait_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + b * BN;
+                for (int i = 0; i < nkb; ++i, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait_bounded(smem_u32(&full[s]), ph, err)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint8_t* a = sA + s * A_STAGE_BYTES;
-                    const uint8_t* b = sB + s * C::B_STAGE_BYTES;
+                    const uint8_t* bb = sB + s * C::B_STAGE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(tmem, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(b + kk * 32), idesc,
+                        umma_bf16(d, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(bb + kk * 32), idesc,
                                   (i > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
-                umma_commit(accum);
-            }
-        } else {
-            const int q = warp & 3;
-            const int n = n0 + q * 32 + lane;
-            float* o = out + (int64_t)split * M * N;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(accum), 0u, err));
-            if (ok) {
-                tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    uint32_t v[16];
-                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int m = m0 + c + j;
-                        if (m < M && n < N) o[(int64_t)m * N + n] = __uint_as_float(v[j]);
-                    }
-                }
+                umma_commit(&accf[b]);
             }
         }
-    } else if (warp >= 2) {
-        const int n = n0 + (warp & 3) * 32 + lane;
-        float* o = out + (int64_t)split * M * N;
-        for (int j = 0; j < BN; ++j) {
-            const int m = m0 + j;
-            if (m < M && n < N) o[(int64_t)m * N + n] = 0.f;
+    } else {
+        const int q = warp & 3;
+        uint32_t j = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++j) {
+            const int split = u % g.splits, tile = u / g.splits;
+            const int n0 = (tile / g.m_tiles) * BM, m0 = (tile % g.m_tiles) * BN;
+            const int n = n0 + q * 32 + lane;
+            const uint32_t b = j & 1u, use = j >> 1;
+            const bool ok = epi_all(mbar_wait_bounded(smem_u32(&accf[b]), use & 1u, err));
+            if (!ok) break;
+            tc_fence_after();
+            fill_row_meta<BN>(g.ep, m0, g.M, meta, threadIdx.x - 64);
+            epi_bar();
+            const uint32_t taddr = tmem + b * BN + ((uint32_t)(q * 32) << 16);
+            if (g.splits == 1) {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + (uint32_t)c, v);
+                    epilogue16(g.ep, n0, n, m0 + c, c, meta, v, g.N, lane);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[b]);
+            } else {
+                float* plane = g.ep.ws + (int64_t)split * g.M * g.N;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + (uint32_t)c, v);
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const int m = m0 + c + k;
+                        if (m < g.M && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[b]);
+                // Distributed fixup: the splits of a tile run in the same round
+                // on co-resident CTAs (cooperative launch); each one waits for
+                // all partial planes, then reduces its own slice of the tile's
+                // activation rows in fixed split order (deterministic) while the
+                // planes are still in L2.  The ticket counts 2*splits arrivals
+                // (written, then done reading) and the last one resets it.
+                __threadfence();
+                epi_bar();
+                int* ctr = g.ep.counters + tile;
+                if (threadIdx.x == 64) {
+                    atomicAdd(ctr, 1);
+                    const long long t0 = clock64();
+                    while (*reinterpret_cast<volatile int*>(ctr) < g.splits) {
+                        if (clock64() - t0 > 2000000000LL) {
+                            set_error(err, kErrTimeout);
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    __threadfence();
+                }
+                epi_bar();
+                const int rows = (BN + g.splits - 1) / g.splits;
+                const int r0 = split * rows, r1 = min(BN, r0 + rows);
+                const int et = threadIdx.x - 64;
+                const int nn = n0 + 4 * (et & 31);
+                const int mr = et >> 5;
+                const bool nok = nn < g.N;  // N % 4 == 0 whenever K is split
+#pragma unroll 1
+                for (int rb = r0 + mr; rb < r1; rb += 4 * 8) {
+                    float4 acc[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+                    for (int sp0 = 0; sp0 < g.splits; sp0 += 4) {
+                        // up to 4 planes x 8 rows of independent loads in flight
+                        float4 t4[4][8];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float* pl = g.ep.ws + (int64_t)(sp0 + j) * g.M * g.N;
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int rr = rb + 4 * u, m = m0 + rr;
+                                t4[j][u] = (sp0 + j < g.splits && nok && rr < r1 && m < g.M)
+                                               ? __ldcg(reinterpret_cast<const float4*>(pl + (int64_t)m * g.N + nn))
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                acc[u].x += t4[j][u].x;
+                                acc[u].y += t4[j][u].y;
+                                acc[u].z += t4[j][u].z;
+                                acc[u].w += t4[j][u].w;
+                            }
+                    }
+                    int mrow[8], krow[8];
+                    bool okr[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int rr = rb + 4 * u;
+                        krow[u] = rr < BN ? rr : 0;
+                        mrow[u] = m0 + rr;
+                        okr[u] = nok && rr < r1 && mrow[u] < g.M;
+                    }
+                    epilogue_vec4x8(g.ep, n0, nn, mrow, krow, okr, meta, acc, g.N);
+                }
+                epi_bar();
+                if (threadIdx.x == 64) {
+                    if (atomicAdd(ctr, 1) == 2 * g.splits - 1) atomicExch(ctr, 0);
+                }
+            }
         }
     }
     tc_fence_before();
@@ -222,50 +562,90 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, float* out, int M, int N, int K,
-                      const GemmPlan& p, int* err, cudaStream_t st) {
-    using C = TileCfg<BN>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM_BYTES);
+cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, int grid, cudaStream_t st) {
+    using C = PCfg<BN>;
+    static int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+        cudaError_t e =
+            cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_dev = dev;
     }
-    dim3 grid(p.n_tiles, p.m_tiles, p.splits);
-    gemm_bf16_tc_kernel<BN><<<grid, 192, C::SMEM_BYTES, st>>>(tmW, tmX, out, M, N, K, p.kb_per_split, err);
-    return cudaGetLastError();
+    if (a.splits == 1) {
+        gemm_tc_kernel<BN><<<grid, 192, C::SMEM_BYTES, st>>>(tmW, tmX, a);
+        return cudaGetLastError();
+    }
+    // CTAs of a split tile wait for one another: launch cooperatively so all of
+    // them are resident at once (the launch fails instead of deadlocking).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, tmW, tmX, a);
 }
 
 }  // namespace
 
-GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms) {
+namespace {
+int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
+
+GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits) {
     GemmPlan p;
-    p.bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
-    p.m_tiles = (M + p.bn - 1) / p.bn;
+    p.bn = bn;
+    p.m_tiles = (M + bn - 1) / bn;
     p.n_tiles = (N + BM - 1) / BM;
     const int KB = (K + BK - 1) / BK;
-    const int occ = p.bn <= 64 ? 2 : 1;
-    const double slots = (double)num_sms * occ;
-    const double tiles = (double)p.m_tiles * p.n_tiles;
-    const double wbytes = 2.0 * N * K;
-    double best = -1.0;
-    for (int s = 1; s <= KB && s <= 32; ++s) {
-        const int kbps = (KB + s - 1) / s;
-        const int sp = (KB + kbps - 1) / kbps;
-        if (sp != s) continue;
-        const double ctas = tiles * sp;
-        const double waves = std::ceil(ctas / slots);
-        const double eff = ctas / (waves * slots);
-        const double partial = sp > 1 ? (2.0 * sp * 4.0 * M * N) / wbytes : 0.0;
-        const double score = eff / (1.0 + 0.5 * partial);
-        if (score > best + 0.02) {
-            best = score;
-            p.splits = sp;
-            p.kb_per_split = kbps;
+    p.kb_per_split = (KB + splits - 1) / splits;
+    p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;
+    // Units are dealt in rounds of `grid`; a multiple of the split count keeps
+    // the splits of every tile in one round (they wait for each other).
+    const long units = (long)p.m_tiles * p.n_tiles * p.splits;
+    const int per_round = std::max(p.splits, (num_sms / p.splits) * p.splits);
+    p.grid = (int)std::min<long>(units, per_round);
+    return p;
+}
+}  // namespace
+
+GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits) {
+    const int KB = (K + BK - 1) / BK;
+    // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
+    const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
+    if (force_bn > 0 || force_splits > 0) {
+        const int bn = force_bn > 0 ? force_bn : bn_for(M);
+        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)));
+    }
+    // Cost in units of one 256-column k-block per CTA: rounds x k-block time x
+    // (k-blocks per unit + per-unit overhead + the partial plane's round trip
+    // when K is split).  Narrow tiles are bound by their weight stream, so a
+    // k-block costs at least a quarter of a full-width one.
+    GemmPlan best_p = make_plan(M, N, K, num_sms, bn_for(M), 1);
+    double best = 1e30;
+    int cands[2] = {bn_for(M), M > 128 ? 128 : 0};
+    for (int bn : cands) {
+        if (!bn) continue;
+        const long tiles = (long)((M + bn - 1) / bn) * ((N + BM - 1) / BM);
+        const double tkb = std::max(bn, 64) / 256.0;
+        for (int sp = 1; sp <= smax; ++sp) {
+            const int kbps = (KB + sp - 1) / sp;
+            if ((KB + kbps - 1) / kbps != sp) continue;
+            const int per_round = std::max(sp, (num_sms / sp) * sp);
+            const double rounds = std::ceil((double)(tiles * sp) / per_round);
+            const double cost = rounds * tkb * (kbps + 1.0 + (sp > 1 ? bn / 32.0 : 0.0));
+            if (cost < best * 0.98) {
+                best = cost;
+                best_p = make_plan(M, N, K, num_sms, bn, sp);
+            }
         }
     }
-    return p;
+    return best_p;
 }
 
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -281,14 +661,16 @@ bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
     return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, float* out, int M, int N, int K,
-                             const GemmPlan& p, int* err, cudaStream_t st) {
+cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K, const GemmPlan& p,
+                             const EpiParams& ep, cudaStream_t st) {
+    if (p.splits > 1 && (!ep.ws || !ep.counters)) return cudaErrorInvalidValue;
+    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, ep};
     switch (p.bn) {
-        case 16: return launch_bn<16>(tmW, tmX, out, M, N, K, p, err, st);
-        case 32: return launch_bn<32>(tmW, tmX, out, M, N, K, p, err, st);
-        case 64: return launch_bn<64>(tmW, tmX, out, M, N, K, p, err, st);
-        case 128: return launch_bn<128>(tmW, tmX, out, M, N, K, p, err, st);
-        case 256: return launch_bn<256>(tmW, tmX, out, M, N, K, p, err, st);
+        case 16: return launch_bn<16>(tmW, tmX, a, p.grid, st);
+        case 32: return launch_bn<32>(tmW, tmX, a, p.grid, st);
+        case 64: return launch_bn<64>(tmW, tmX, a, p.grid, st);
+        case 128: return launch_bn<128>(tmW, tmX, a, p.grid, st);
+        case 256: return launch_bn<256>(tmW, tmX, a, p.grid, st);
         default: return cudaErrorInvalidValue;
     }
 }

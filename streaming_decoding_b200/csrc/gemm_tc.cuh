@@ -1,4 +1,5 @@
-// bf16 dense projections on the 5th-generation tensor cores (tcgen05 + TMA).
+// bf16 dense projections on the 5th-generation tensor cores (tcgen05 + TMA),
+// persistent, with the projection's epilogue fused in.
 #pragma once
 
 #include <cuda.h>
@@ -7,26 +8,53 @@
 
 namespace wedlm {
 
-// How one Y[M][N] = X[M][K] * W[N][K]^T is cut into CTAs: 128 weight rows per
-// tile (the MMA's M), bn activation rows per tile (the MMA's N), and `splits`
-// slices of K, each writing its own fp32 partial plane out[split][M][N].
+// What the epilogue does with the fp32 accumulator Y[m][n]:
+//   EPI_STORE     out[m][n] = Y                                  (LM head, test hook)
+//   EPI_RESIDUAL  out[m][n] += Y, rows marked live only          (O and down projections)
+//   EPI_SWIGLU    act[m][n/2] = silu(Y[m][n]) * Y[m][n+1], n even (gate/up rows interleaved)
+//   EPI_QKV_ROPE  rotate q and k head dims (pairs interleaved in adjacent rows) at the
+//                 row's logical position; q -> act[m][hq][128], k and v -> KV pages at
+//                 cache index S + r of the row's sequence
+enum EpiKind : int { EPI_STORE = 0, EPI_QKV_ROPE = 1, EPI_SWIGLU = 2, EPI_RESIDUAL = 3 };
+
+struct EpiParams {
+    int kind = EPI_STORE;
+    float* out = nullptr;
+    bf16* act = nullptr;
+    bf16* kv_pool = nullptr;
+    KVLayout kvl{};
+    int layer = 0, hq = 0, hkv = 0;
+    const float2* rope_cs = nullptr;
+    int rope_max_pos = 0;
+    RowState rs{};
+    SlotState ss{};
+    RowMap rm{};
+    int check_rows = 0;        // 1: skip rows RowMap marks as padding
+    float* ws = nullptr;       // split-K partial planes [splits][M][N]
+    int* counters = nullptr;   // per-tile tickets; zero before and after every launch
+    int* err = nullptr;
+};
+
+// How Y[M][N] = X[M][K] * W[N][K]^T is cut: tiles of 128 weight rows (MMA M)
+// by bn activation rows (MMA N), K in `splits` slices; units = tiles * splits
+// are dealt round-robin to `grid` persistent CTAs (one per SM).
 struct GemmPlan {
     int bn = 16;
     int splits = 1;
     int kb_per_split = 1;
     int m_tiles = 1;
     int n_tiles = 1;
+    int grid = 1;
 };
 
-GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms);
+// max_splits: the most K slices the caller's partial workspace holds (>= 1).
+// force_bn / force_splits > 0 pin the tile width / split count (tuning hook).
+GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0);
 
-// 2-D bf16 tensor map over a row-major [rows][cols] matrix with a 64-column,
-// box_rows-row box and 128-byte swizzle.  Returns false if the driver refuses.
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
-// tmW: weights [N][K] with box_rows 128; tmX: activations [>=M][K] with
-// box_rows = plan.bn.  out: fp32 [plan.splits][M][N].
-cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, float* out, int M, int N, int K,
-                             const GemmPlan& plan, int* err, cudaStream_t st);
+// tmW: weights [N][K], box rows 128; tmX: activations [>=M][K], box rows plan.bn.
+cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K,
+                             const GemmPlan& plan, const EpiParams& ep, cudaStream_t st);
 
 }  // namespace wedlm

@@ -329,6 +329,46 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(const float* __restr
     for (int c = threadIdx.x; c < d; c += blockDim.x) hr[c] = from_f32<T>(xr[c] * inv * g[c]);
 }
 
+// RMSNorm of the residual stream into the next GEMM's bf16 input:
+// h = x / rms(x) * g, one CTA per row, the row held in registers (float4
+// loads; d % 4 == 0 and d <= 4 * 256 * kNormVec).
+constexpr int kNormVec = 8;
+__global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ h,
+                                                           const float* __restrict__ g, float eps, int d, RowMap rm) {
+    __shared__ float red[32];
+    const int row = blockIdx.x;
+    int slot, r;
+    if (!rm.live(row, slot, r)) return;
+    const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * d);
+    const float4* gr = reinterpret_cast<const float4*>(g);
+    const int nv = d >> 2;
+    float4 v[kNormVec];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = threadIdx.x + i * blockDim.x;
+        v[i] = c < nv ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    }
+    ss = block_sum(ss, red);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    __nv_bfloat162* hr = reinterpret_cast<__nv_bfloat162*>(h + (int64_t)row * d);
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+        const int c = threadIdx.x + i * blockDim.x;
+        if (c < nv) {
+            const float4 gg = gr[c];
+            hr[2 * c] = __floats2bfloat162_rn(v[i].x * inv * gg.x, v[i].y * inv * gg.y);
+            hr[2 * c + 1] = __floats2bfloat162_rn(v[i].z * inv * gg.z, v[i].w * inv * gg.w);
+        }
+    }
+}
+
+void launch_rmsnorm_bf16(const float* x, bf16* h, const float* g, float eps, int M, int d, RowMap rm,
+                         cudaStream_t st) {
+    rmsnorm_bf16_kernel<<<M, 256, 0, st>>>(x, h, g, eps, d, rm);
+}
+
 // SwiGLU: act = silu(gate) * up, gate = columns [0, F), up = [F, 2F).
 template <typename T>
 __global__ void __launch_bounds__(256) swiglu_kernel(const float* __restrict__ ws, int splits, int64_t sstride, int F,

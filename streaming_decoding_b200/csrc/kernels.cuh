@@ -5,20 +5,6 @@
 
 namespace wedlm {
 
-// Which rows of a forward belong to which slot: row = entry * stride + r,
-// slot = slot_base + entry, row is live iff r < n[slot].
-struct RowMap {
-    int slot_base;
-    int stride;
-    const int32_t* n;
-    __device__ __forceinline__ bool live(int row, int& slot, int& r) const {
-        const int e = row / stride;
-        r = row - e * stride;
-        slot = slot_base + e;
-        return r < n[slot];
-    }
-};
-
 struct StepKnobs {
     float lambda, tau, logit_scale;
     int tau_none;
@@ -51,6 +37,10 @@ void launch_attn_f32(const float* q, const float* kv_pool, KVLayout kvl, int lay
 template <typename T>
 void launch_residual_norm(const float* ws, int splits, int64_t split_stride, int M, int d, float* x, T* h,
                           const float* g, float eps, RowMap rm, cudaStream_t st);
+
+// bf16 mode: h = rmsnorm(x) * g (d % 4 == 0, d <= 8192).
+void launch_rmsnorm_bf16(const float* x, bf16* h, const float* g, float eps, int M, int d, RowMap rm,
+                         cudaStream_t st);
 
 template <typename T>
 void launch_swiglu(const float* ws, int splits, int64_t split_stride, int M, int F, T* act, RowMap rm,

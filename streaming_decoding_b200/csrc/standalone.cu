@@ -12,14 +12,6 @@ namespace {
 
 constexpr int kChunks = 16;
 
-__global__ void sum_planes_kernel(const float* __restrict__ src, int planes, int64_t plane, float* __restrict__ dst) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= plane) return;
-    float v = 0.f;
-    for (int p = 0; p < planes; ++p) v += src[p * plane + i];
-    dst[i] = v;
-}
-
 wedlm_status sync_status(cudaStream_t st) {
     if (cudaGetLastError() != cudaSuccess) return WEDLM_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return WEDLM_ERR_CUDA;
@@ -68,34 +60,45 @@ wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t ma
 }
 
 wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K, void* stream) {
+    return wedlm_linear_bf16_plan(X, W, Y, M, N, K, 0, 0, stream);
+}
+
+wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                    int32_t tile_n, int32_t k_splits, void* stream) {
     if (M < 1 || N < 1 || K < 8 || K % 8 || !X || !W || !Y) return WEDLM_ERR_INVALID_ARG;
+    if (tile_n != 0 && tile_n != 16 && tile_n != 32 && tile_n != 64 && tile_n != 128 && tile_n != 256)
+        return WEDLM_ERR_INVALID_ARG;
+    if (k_splits < 0 || k_splits > 16) return WEDLM_ERR_INVALID_ARG;
     if (((uintptr_t)X | (uintptr_t)W) & 15) return WEDLM_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    GemmPlan p = plan_gemm_bf16(M, N, K, sms);
+    GemmPlan p = plan_gemm_bf16(M, N, K, sms, 16, tile_n, k_splits);
     CUtensorMap tw, tx;
     if (!make_tmap_bf16(&tw, W, (uint64_t)N, (uint64_t)K, 128)) return WEDLM_ERR_CUDA;
     if (!make_tmap_bf16(&tx, X, (uint64_t)M, (uint64_t)K, (uint32_t)p.bn)) return WEDLM_ERR_CUDA;
-    int* err = nullptr;
-    float* planes = Y;
-    if (cudaMallocAsync((void**)&err, sizeof(int), st) != cudaSuccess) return WEDLM_ERR_OOM_DEVICE;
-    cudaMemsetAsync(err, 0, sizeof(int), st);
+    const size_t tiles = (size_t)p.m_tiles * p.n_tiles;
+    int* scratch = nullptr;  // error word, then tile tickets
+    float* planes = nullptr;
+    if (cudaMallocAsync((void**)&scratch, (1 + tiles) * sizeof(int), st) != cudaSuccess) return WEDLM_ERR_OOM_DEVICE;
+    cudaMemsetAsync(scratch, 0, (1 + tiles) * sizeof(int), st);
     if (p.splits > 1 && cudaMallocAsync((void**)&planes, (size_t)p.splits * M * N * 4, st) != cudaSuccess) {
-        cudaFreeAsync(err, st);
+        cudaFreeAsync(scratch, st);
         return WEDLM_ERR_OOM_DEVICE;
     }
+    EpiParams ep;
+    ep.kind = EPI_STORE;
+    ep.out = Y;
+    ep.ws = planes;
+    ep.counters = scratch + 1;
+    ep.err = scratch;
     wedlm_status s = WEDLM_OK;
-    if (launch_gemm_bf16(tw, tx, planes, M, N, K, p, err, st) != cudaSuccess) s = WEDLM_ERR_CUDA;
-    if (!s && p.splits > 1) {
-        const int64_t plane = (int64_t)M * N;
-        sum_planes_kernel<<<(unsigned)((plane + 255) / 256), 256, 0, st>>>(planes, p.splits, plane, Y);
-    }
+    if (launch_gemm_bf16(tw, tx, M, N, K, p, ep, st) != cudaSuccess) s = WEDLM_ERR_CUDA;
     int herr = 0;
-    cudaMemcpyAsync(&herr, err, sizeof(int), cudaMemcpyDeviceToHost, st);
-    if (p.splits > 1) cudaFreeAsync(planes, st);
-    cudaFreeAsync(err, st);
+    cudaMemcpyAsync(&herr, scratch, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (planes) cudaFreeAsync(planes, st);
+    cudaFreeAsync(scratch, st);
     wedlm_status s2 = sync_status(st);
     if (s) return s;
     if (s2) return s2;

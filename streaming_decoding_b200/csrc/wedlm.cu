@@ -20,6 +20,7 @@
 #include <cstdio>
 #include <cstring>
 #include <deque>
+#include <map>
 #include <string>
 #include <vector>
 
@@ -102,8 +103,30 @@ struct wedlm_ctx {
     void* q = nullptr;
     void* attn_out = nullptr;
     void* act = nullptr;
-    float* ws = nullptr;
+    float* ws = nullptr;           // split-K partial planes
     size_t ws_floats = 0;
+    int* tile_counters = nullptr;  // per-tile tickets of the split-K reduction
+    size_t n_tile_counters = 0;
+    // GEMM launch shapes chosen by timing candidates, per (projection kind, rows)
+    bool autotune = true;
+    struct Tuned {
+        GemmPlan plan;
+        float us;
+    };
+    std::map<std::pair<int, int>, Tuned> tuned;
+    // CUDA graph of one decode step, replayed while its shape and knobs match
+    bool use_graphs = true;
+    cudaGraphExec_t graph_exec = nullptr;
+    int64_t graph_launches = 0;
+    struct StepKey {
+        int n_entries = -1, stride = -1, tau_none = 0;
+        float lambda = 0.f, tau = 0.f, scale = 0.f;
+        bool operator==(const StepKey& o) const {
+            return n_entries == o.n_entries && stride == o.stride && tau_none == o.tau_none &&
+                   lambda == o.lambda && tau == o.tau && scale == o.scale;
+        }
+    };
+    StepKey graph_key, eager_key;
     float* logits = nullptr;
     size_t logits_floats = 0;
     float4* ent_part = nullptr;
@@ -210,42 +233,109 @@ const CUtensorMap* xmap(wedlm_ctx* c, const void* p, uint64_t rows, uint64_t col
     return &c->xmaps.back().tm;
 }
 
-// Y[M][N] (fp32 partial planes in ws or `out`) = X[M][K] * W[N][K]^T.
-wedlm_status gemm(wedlm_ctx* ctx, int kind, const void* X, const void* W, const CUtensorMap* tmW, int M, int N,
-                  int K, float* out, size_t out_cap_floats, int* splits_out, int max_splits = 32) {
-    if (!ctx->bf16) {
-        if ((size_t)M * N > out_cap_floats) return fail(ctx, WEDLM_ERR_STATE, "gemm workspace too small");
-        ProfScope ps(ctx, kind);
-        launch_gemm_f32((const float*)X, (const float*)W, out, M, N, K, ctx->stream);
-        *splits_out = 1;
-        return WEDLM_OK;
-    }
-    GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms);
-    // cap the K splits by the caller's limit and by the partial-plane capacity
-    const size_t plane = (size_t)M * N;
-    const int cap = (int)std::min<size_t>((size_t)max_splits, out_cap_floats / plane);
-    if (cap < 1) return fail(ctx, WEDLM_ERR_STATE, "gemm workspace too small");
-    if (p.splits > cap) {
-        const int KB = (K + 63) / 64;
-        p.kb_per_split = (KB + cap - 1) / cap;
-        p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;
-    }
-    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
-    if (!tx) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for activations");
-    cudaError_t e;
-    {
-        ProfScope ps(ctx, kind);
-        e = launch_gemm_bf16(*tmW, *tx, out, M, N, K, p, ctx->err, ctx->stream);
-    }
-    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("gemm launch: ") + cudaGetErrorString(e));
-    *splits_out = p.splits;
+// fp32 mode: C[M][N] = X[M][K] * W[N][K]^T into `out` (the epilogue kernels follow).
+wedlm_status gemm_f32(wedlm_ctx* ctx, int kind, const float* X, const float* W, int M, int N, int K) {
+    if ((size_t)M * N > ctx->ws_floats) return fail(ctx, WEDLM_ERR_STATE, "gemm workspace too small");
+    ProfScope ps(ctx, kind);
+    launch_gemm_f32(X, W, ctx->ws, M, N, K, ctx->stream);
     return WEDLM_OK;
 }
 
-size_t gemm_ws_need(const wedlm_ctx* c, int M, int N, int K) {
-    if (!c->bf16) return (size_t)M * N;
-    GemmPlan p = plan_gemm_bf16(M, N, K, c->num_sms);
-    return (size_t)p.splits * M * N;
+// Time the candidate launch shapes of one projection (kind, M) on its real
+// weights with a plain-store epilogue into scratch, and keep the fastest.
+// Runs once per (kind, M) on the context's stream; candidates that do not fit
+// the scratch buffers are skipped.
+void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* tmW, int M, int N, int K) {
+    const std::pair<int, int> key(kind, M);
+    if (ctx->tuned.count(key)) return;
+    ctx->tuned[key] = {plan_gemm_bf16(M, N, K, ctx->num_sms, 1), -1.f};
+    if ((size_t)M * N > ctx->logits_floats) return;
+    std::vector<int> bns;
+    if (M > 128) bns = {256, 128};
+    else if (M > 64) bns = {128, 64};
+    else bns = {M <= 16 ? 16 : M <= 32 ? 32 : 64};
+    cudaEvent_t e0 = prof_event(ctx), e1 = prof_event(ctx);
+    float best = 1e30f;
+    GemmPlan bestp = ctx->tuned[key].plan;
+    EpiParams ep;
+    ep.kind = EPI_STORE;
+    ep.out = ctx->logits;
+    ep.ws = ctx->ws;
+    ep.counters = ctx->tile_counters;
+    ep.err = ctx->err;
+    const int KB = (K + 63) / 64;
+    for (int bn : bns) {
+        for (int sp : {1, 2, 3, 4, 6, 8, 12, 16}) {
+            if (sp > KB || (sp > 1 && N % 4)) continue;
+            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, bn, sp);
+            if (p.splits != sp) continue;
+            if (p.splits > 1 && ((size_t)p.splits * M * N > ctx->ws_floats ||
+                                 (size_t)p.m_tiles * p.n_tiles > ctx->n_tile_counters))
+                continue;
+            const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
+            if (!tx) continue;
+            float t = 1e30f;
+            for (int rep = 0; rep < 4; ++rep) {
+                cudaEventRecord(e0, ctx->stream);
+                if (launch_gemm_bf16(*tmW, *tx, M, N, K, p, ep, ctx->stream) != cudaSuccess) {
+                    cudaGetLastError();
+                    t = 1e30f;
+                    break;
+                }
+                cudaEventRecord(e1, ctx->stream);
+                ctx->launches++;
+                cudaEventSynchronize(e1);
+                float ms = 0.f;
+                cudaEventElapsedTime(&ms, e0, e1);
+                if (rep > 0) t = std::min(t, ms * 1e3f);
+            }
+            if (t < best) {
+                best = t;
+                bestp = p;
+            }
+        }
+    }
+    ctx->ev_used -= 2;
+    ctx->tuned[key] = {bestp, best < 1e29f ? best : -1.f};
+}
+
+// bf16 mode: the persistent tcgen05 GEMM with its epilogue fused (gemm_tc.cuh).
+wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* tmW, int M, int N, int K,
+                       EpiParams ep, bool tune = true) {
+    GemmPlan p;
+    if (ctx->autotune && tune) {
+        autotune_shape(ctx, kind, X, tmW, M, N, K);
+        p = ctx->tuned[{kind, M}].plan;
+    } else {
+        const size_t plane = (size_t)M * N;
+        const int cap = (int)std::max<size_t>(1, std::min<size_t>(16, ctx->ws_floats / plane));
+        p = plan_gemm_bf16(M, N, K, ctx->num_sms, cap);
+    }
+    if (p.splits > 1 && ((size_t)p.n_tiles * p.m_tiles > ctx->n_tile_counters ||
+                         (size_t)p.splits * M * N > ctx->ws_floats))
+        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1);
+    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
+    if (!tx) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for activations");
+    ep.ws = ctx->ws;
+    ep.counters = ctx->tile_counters;
+    ep.err = ctx->err;
+    cudaError_t e;
+    {
+        ProfScope ps(ctx, kind);
+        e = launch_gemm_bf16(*tmW, *tx, M, N, K, p, ep, ctx->stream);
+    }
+    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("gemm launch: ") + cudaGetErrorString(e));
+    return WEDLM_OK;
+}
+
+// Partial-plane floats and tile tickets the bf16 GEMM plans of one shape may
+// need (room for the tuning candidates: up to `max_splits` slices).
+void gemm_needs(const wedlm_ctx* c, int M, int N, int K, int max_splits, size_t* ws, size_t* tiles) {
+    const int KB = (K + 63) / 64;
+    const int sp = std::min(max_splits, KB);
+    if (sp > 1 && N % 4 == 0) *ws = std::max(*ws, (size_t)sp * M * N);
+    const int bn_min = M > 128 ? 128 : 16;
+    *tiles = std::max(*tiles, (size_t)((M + bn_min - 1) / bn_min) * ((N + 127) / 128));
 }
 
 wedlm_status build_weight_maps(wedlm_ctx* ctx) {
@@ -270,6 +360,9 @@ wedlm_status build_weight_maps(wedlm_ctx* ctx) {
 wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
     if (code == 0) return WEDLM_OK;
     CK(cudaMemsetAsync(ctx->err, 0, sizeof(int), ctx->stream));
+    // a GEMM that gave up may leave split-K tickets behind
+    if (ctx->tile_counters)
+        CK(cudaMemsetAsync(ctx->tile_counters, 0, ctx->n_tile_counters * sizeof(int), ctx->stream));
     if (code == kErrTimeout) return fail(ctx, WEDLM_ERR_TIMEOUT, "a bounded device wait timed out");
     return fail(ctx, WEDLM_ERR_DEVICE_ASSERT, "a device bounds check fired");
 }
@@ -277,78 +370,121 @@ wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
 // The transformer stack over rows [entry * stride + r] of slots slot_base +
 // entry.  On entry x holds the embeddings and h the first RMSNorm; on exit h
 // holds the final-normed hidden states.
-template <typename T>
-wedlm_status forward_layers(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
+
+// fp32 (exact-parity) mode: SIMT GEMMs, separate epilogue kernels.
+wedlm_status forward_f32(wedlm_ctx* ctx, int slot_base, int n_entries, int stride) {
     const int M = n_entries * stride;
     RowMap rm{slot_base, stride, ctx->ss.n};
     const float eps = ctx->cfg.rms_eps;
-    T* h = (T*)ctx->h;
-    T* qb = (T*)ctx->q;
-    T* ao = (T*)ctx->attn_out;
-    T* act = (T*)ctx->act;
-    const int rt = ctx->bf16 ? attn_rows_per_tile(ctx->hq / ctx->hkv) : 1;
+    float* h = (float*)ctx->h;
+    float* qb = (float*)ctx->q;
+    float* ao = (float*)ctx->attn_out;
+    float* act = (float*)ctx->act;
+    wedlm_status s;
     for (int l = 0; l < ctx->L; ++l) {
-        int sp = 1;
-        wedlm_status s;
-        s = gemm(ctx, WEDLM_PROF_GEMM_QKV, h, ctx->wqkv[l], ctx->bf16 ? &ctx->tm_qkv[l] : nullptr, M, ctx->Nqkv,
-                 ctx->d, ctx->ws, ctx->ws_floats, &sp);
-        if (s) return s;
+        if ((s = gemm_f32(ctx, WEDLM_PROF_GEMM_QKV, h, (const float*)ctx->wqkv[l], M, ctx->Nqkv, ctx->d))) return s;
         {
             ProfScope ps(ctx, WEDLM_PROF_QKV_ROPE);
-            launch_qkv_rope<T>(ctx->ws, sp, (int64_t)M * ctx->Nqkv, M, ctx->hq, ctx->hkv, ctx->hd, qb,
-                               (T*)ctx->kv_pool, ctx->kvl, l, ctx->rope_cs, ctx->max_ctx, ctx->rs, ctx->ss, rm,
-                               ctx->err, ctx->stream);
+            launch_qkv_rope<float>(ctx->ws, 1, (int64_t)M * ctx->Nqkv, M, ctx->hq, ctx->hkv, ctx->hd, qb,
+                                   (float*)ctx->kv_pool, ctx->kvl, l, ctx->rope_cs, ctx->max_ctx, ctx->rs, ctx->ss, rm,
+                                   ctx->err, ctx->stream);
         }
-        if (ctx->bf16) {
-            const int kc = decode ? ctx->attn_kv_chunk : (1 << 30);
-            const int ms = decode ? ctx->attn_max_splits : 1;
-            {
-                ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
-                launch_attn_bf16((const bf16*)qb, (const bf16*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv,
-                                 ctx->hd, (bf16*)ao, ctx->attn_po, ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss,
-                                 rm, ctx->err, ctx->stream);
-            }
-            if (ms > 1) {
-                ProfScope ps(ctx, WEDLM_PROF_ATTN_COMBINE);
-                launch_attn_combine(ctx->attn_po, ctx->attn_pml, (bf16*)ao, M, ctx->hq, ctx->hd, kc, ms, rt, ctx->ss,
-                                    rm, ctx->stream);
-            }
-        } else {
+        {
             ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
-            launch_attn_f32((const float*)qb, (const float*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd,
-                            (float*)ao, M, ctx->ss, rm, ctx->err, ctx->stream);
+            launch_attn_f32(qb, (const float*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd, ao, M, ctx->ss,
+                            rm, ctx->err, ctx->stream);
         }
-        s = gemm(ctx, WEDLM_PROF_GEMM_O, ao, ctx->wo[l], ctx->bf16 ? &ctx->tm_o[l] : nullptr, M, ctx->d,
-                 ctx->hq * ctx->hd, ctx->ws, ctx->ws_floats, &sp);
-        if (s) return s;
+        if ((s = gemm_f32(ctx, WEDLM_PROF_GEMM_O, ao, (const float*)ctx->wo[l], M, ctx->d, ctx->hq * ctx->hd)))
+            return s;
         {
             ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
-            launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, ctx->ffn_norm[l], eps, rm,
-                                    ctx->stream);
+            launch_residual_norm<float>(ctx->ws, 1, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, ctx->ffn_norm[l], eps,
+                                        rm, ctx->stream);
         }
-        s = gemm(ctx, WEDLM_PROF_GEMM_GATE_UP, h, ctx->wgu[l], ctx->bf16 ? &ctx->tm_gu[l] : nullptr, M, 2 * ctx->F,
-                 ctx->d, ctx->ws, ctx->ws_floats, &sp);
-        if (s) return s;
+        if ((s = gemm_f32(ctx, WEDLM_PROF_GEMM_GATE_UP, h, (const float*)ctx->wgu[l], M, 2 * ctx->F, ctx->d)))
+            return s;
         {
             ProfScope ps(ctx, WEDLM_PROF_SWIGLU);
-            launch_swiglu<T>(ctx->ws, sp, (int64_t)M * 2 * ctx->F, M, ctx->F, act, rm, ctx->stream);
+            launch_swiglu<float>(ctx->ws, 1, (int64_t)M * 2 * ctx->F, M, ctx->F, act, rm, ctx->stream);
         }
-        s = gemm(ctx, WEDLM_PROF_GEMM_DOWN, act, ctx->wd[l], ctx->bf16 ? &ctx->tm_d[l] : nullptr, M, ctx->d, ctx->F,
-                 ctx->ws, ctx->ws_floats, &sp);
-        if (s) return s;
+        if ((s = gemm_f32(ctx, WEDLM_PROF_GEMM_DOWN, act, (const float*)ctx->wd[l], M, ctx->d, ctx->F))) return s;
         const float* gnext = (l + 1 < ctx->L) ? ctx->attn_norm[l + 1] : ctx->final_norm;
         {
             ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
-            launch_residual_norm<T>(ctx->ws, sp, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, gnext, eps, rm,
-                                    ctx->stream);
+            launch_residual_norm<float>(ctx->ws, 1, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, gnext, eps, rm,
+                                        ctx->stream);
+        }
+    }
+    return WEDLM_OK;
+}
+
+// bf16 mode: every projection is one persistent tcgen05 GEMM with its epilogue
+// fused (RoPE + K/V page scatter, residual add, SwiGLU); RMSNorm and attention
+// are the only other kernels of a layer.
+wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
+    const int M = n_entries * stride;
+    RowMap rm{slot_base, stride, ctx->ss.n};
+    const float eps = ctx->cfg.rms_eps;
+    bf16* h = (bf16*)ctx->h;
+    bf16* qb = (bf16*)ctx->q;
+    bf16* ao = (bf16*)ctx->attn_out;
+    bf16* act = (bf16*)ctx->act;
+    const int rt = attn_rows_per_tile(ctx->hq / ctx->hkv);
+    EpiParams base;
+    base.check_rows = 1;
+    base.rm = rm;
+    base.rs = ctx->rs;
+    base.ss = ctx->ss;
+    base.kvl = ctx->kvl;
+    base.kv_pool = (bf16*)ctx->kv_pool;
+    base.hq = ctx->hq;
+    base.hkv = ctx->hkv;
+    base.rope_cs = ctx->rope_cs;
+    base.rope_max_pos = ctx->max_ctx;
+    wedlm_status s;
+    for (int l = 0; l < ctx->L; ++l) {
+        EpiParams e = base;
+        e.layer = l;
+        e.kind = EPI_QKV_ROPE;
+        e.act = qb;
+        if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_QKV, h, &ctx->tm_qkv[l], M, ctx->Nqkv, ctx->d, e, decode))) return s;
+        const int kc = decode ? ctx->attn_kv_chunk : (1 << 30);
+        const int ms = decode ? ctx->attn_max_splits : 1;
+        {
+            ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
+            launch_attn_bf16(qb, (const bf16*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd, ao, ctx->attn_po,
+                             ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss, rm, ctx->err, ctx->stream);
+        }
+        if (ms > 1) {
+            ProfScope ps(ctx, WEDLM_PROF_ATTN_COMBINE);
+            launch_attn_combine(ctx->attn_po, ctx->attn_pml, ao, M, ctx->hq, ctx->hd, kc, ms, rt, ctx->ss, rm,
+                                ctx->stream);
+        }
+        e.kind = EPI_RESIDUAL;
+        e.out = ctx->x;
+        if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_O, ao, &ctx->tm_o[l], M, ctx->d, ctx->hq * ctx->hd, e, decode))) return s;
+        {
+            ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
+            launch_rmsnorm_bf16(ctx->x, h, ctx->ffn_norm[l], eps, M, ctx->d, rm, ctx->stream);
+        }
+        e.kind = EPI_SWIGLU;
+        e.act = act;
+        if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_GATE_UP, h, &ctx->tm_gu[l], M, 2 * ctx->F, ctx->d, e, decode))) return s;
+        e.kind = EPI_RESIDUAL;
+        e.out = ctx->x;
+        if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_DOWN, act, &ctx->tm_d[l], M, ctx->d, ctx->F, e, decode))) return s;
+        const float* gnext = (l + 1 < ctx->L) ? ctx->attn_norm[l + 1] : ctx->final_norm;
+        {
+            ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
+            launch_rmsnorm_bf16(ctx->x, h, gnext, eps, M, ctx->d, rm, ctx->stream);
         }
     }
     return WEDLM_OK;
 }
 
 wedlm_status run_forward(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
-    return ctx->bf16 ? forward_layers<bf16>(ctx, slot_base, n_entries, stride, decode)
-                     : forward_layers<float>(ctx, slot_base, n_entries, stride, decode);
+    return ctx->bf16 ? forward_bf16(ctx, slot_base, n_entries, stride, decode)
+                     : forward_f32(ctx, slot_base, n_entries, stride);
 }
 
 int max_active_window(const wedlm_ctx* c, int* n_entries) {
@@ -363,7 +499,7 @@ int max_active_window(const wedlm_ctx* c, int* n_entries) {
 }
 
 // Enqueue one decode step over slots [0, n_entries) with row stride `stride`.
-wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_entries, int stride) {
+wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_entries, int stride) {
     const int M = n_entries * stride;
     {
         ProfScope ps(ctx, WEDLM_PROF_PREPARE);
@@ -378,9 +514,18 @@ wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_en
     }
     wedlm_status s = run_forward(ctx, 0, n_entries, stride, true);
     if (s) return s;
-    int lsp = 1;
-    s = gemm(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, ctx->lm_head, ctx->bf16 ? &ctx->tm_lm : nullptr, M, ctx->V,
-             ctx->d, ctx->logits, ctx->logits_floats, &lsp, 4);
+    const int lsp = 1;
+    if (ctx->bf16) {
+        EpiParams e;
+        e.kind = EPI_STORE;
+        e.out = ctx->logits;
+        s = gemm_bf16(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, &ctx->tm_lm, M, ctx->V, ctx->d, e);
+    } else {
+        if ((size_t)M * ctx->V > ctx->logits_floats) return fail(ctx, WEDLM_ERR_STATE, "logits buffer too small");
+        ProfScope ps(ctx, WEDLM_PROF_GEMM_LM_HEAD);
+        launch_gemm_f32((const float*)ctx->h, (const float*)ctx->lm_head, ctx->logits, M, ctx->V, ctx->d, ctx->stream);
+        s = WEDLM_OK;
+    }
     if (s) return s;
     {
         ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
@@ -397,6 +542,62 @@ wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_en
     ctx->last_M = M;
     ctx->logits_splits_last = lsp;
     if (ctx->prof && ctx->ev_marks.size() > 4096) prof_collect(ctx);
+    return WEDLM_OK;
+}
+
+void drop_graph(wedlm_ctx* ctx) {
+    if (ctx->graph_exec) cudaGraphExecDestroy(ctx->graph_exec);
+    ctx->graph_exec = nullptr;
+    ctx->graph_key = wedlm_ctx::StepKey();
+}
+
+// Enqueue one decode step.  A step whose shape and knobs were already run
+// once is captured into a CUDA graph and replayed from then on (every
+// per-step size is read from device memory, so the graph stays valid); the
+// eager path is used on the legacy default stream and while profiling.
+wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_entries, int stride) {
+    wedlm_ctx::StepKey key;
+    key.n_entries = n_entries;
+    key.stride = stride;
+    key.tau_none = prm->tau_none;
+    key.lambda = prm->lambda;
+    key.tau = prm->tau;
+    key.scale = prm->logit_scale;
+    const bool graphable = ctx->use_graphs && ctx->bf16 && ctx->stream != nullptr && !ctx->prof;
+    if (graphable && ctx->graph_exec && ctx->graph_key == key) {
+        cudaError_t e = cudaGraphLaunch(ctx->graph_exec, ctx->stream);
+        if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("graph launch: ") + cudaGetErrorString(e));
+        ctx->launches += ctx->graph_launches;
+        return WEDLM_OK;
+    }
+    if (!graphable || !(ctx->eager_key == key)) {
+        ctx->eager_key = key;
+        return enqueue_step_kernels(ctx, prm, n_entries, stride);
+    }
+    drop_graph(ctx);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(ctx->stream, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
+    const int64_t l0 = ctx->launches;
+    wedlm_status s = enqueue_step_kernels(ctx, prm, n_entries, stride);
+    e = cudaStreamEndCapture(ctx->stream, &graph);
+    if (s) {
+        if (graph) cudaGraphDestroy(graph);
+        return s;
+    }
+    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("end capture: ") + cudaGetErrorString(e));
+    e = cudaGraphInstantiate(&ctx->graph_exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) {
+        ctx->graph_exec = nullptr;
+        return fail(ctx, WEDLM_ERR_CUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
+    }
+    ctx->graph_launches = ctx->launches - l0;
+    ctx->launches = l0;
+    ctx->graph_key = key;
+    e = cudaGraphLaunch(ctx->graph_exec, ctx->stream);
+    if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("graph launch: ") + cudaGetErrorString(e));
+    ctx->launches += ctx->graph_launches;
     return WEDLM_OK;
 }
 
@@ -448,6 +649,7 @@ bool valid_cfg(const wedlm_model_cfg* c, std::string* why) {
     } else if (c->dtype == WEDLM_DTYPE_BF16) {
         if (c->head_dim != 128) return bad("bf16 mode needs head_dim 128");
         if (c->d_model % 8 || c->ffn_dim % 8) return bad("bf16 mode needs d_model and ffn_dim multiples of 8");
+        if (c->d_model > 8192) return bad("bf16 mode supports d_model <= 8192");
     } else {
         return bad("unknown dtype");
     }
@@ -582,17 +784,24 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     xa.add(&ctx->q, (size_t)Mmax * ctx->hq * ctx->hd * elt);
     xa.add(&ctx->attn_out, (size_t)Mmax * ctx->hq * ctx->hd * elt);
     xa.add(&ctx->act, (size_t)Mmax * F * elt);
-    size_t need = 0;
-    for (int M : {ctx->Mdec, ctx->chunk}) {
-        need = std::max(need, gemm_ws_need(ctx, M, ctx->Nqkv, d));
-        need = std::max(need, gemm_ws_need(ctx, M, d, ctx->hq * ctx->hd));
-        need = std::max(need, gemm_ws_need(ctx, M, 2 * F, d));
-        need = std::max(need, gemm_ws_need(ctx, M, d, F));
+    size_t need = 0, tiles = 0;
+    if (ctx->bf16) {
+        for (int M : {ctx->Mdec, ctx->chunk}) {
+            const int ms = M == ctx->Mdec ? 16 : 4;
+            gemm_needs(ctx, M, ctx->Nqkv, d, ms, &need, &tiles);
+            gemm_needs(ctx, M, d, ctx->hq * ctx->hd, ms, &need, &tiles);
+            gemm_needs(ctx, M, 2 * F, d, std::min(ms, 8), &need, &tiles);
+            gemm_needs(ctx, M, d, F, ms, &need, &tiles);
+        }
+        gemm_needs(ctx, ctx->Mdec, V, d, 2, &need, &tiles);
+    } else {
+        need = (size_t)Mmax * std::max({(size_t)ctx->Nqkv, (size_t)2 * F, (size_t)d});
     }
-    ctx->ws_floats = need;
-    xa.add((void**)&ctx->ws, need * 4);
-    const size_t lsp = ctx->bf16 ? (size_t)std::min(4, plan_gemm_bf16(ctx->Mdec, V, d, ctx->num_sms).splits) : 1;
-    ctx->logits_floats = lsp * ctx->Mdec * (size_t)V;
+    ctx->ws_floats = std::max<size_t>(need, 1);
+    ctx->n_tile_counters = std::max<size_t>(tiles, 1);
+    xa.add((void**)&ctx->ws, ctx->ws_floats * 4);
+    xa.add((void**)&ctx->tile_counters, ctx->n_tile_counters * 4);
+    ctx->logits_floats = (size_t)ctx->Mdec * (size_t)V;
     xa.add((void**)&ctx->logits, ctx->logits_floats * 4);
     xa.add((void**)&ctx->ent_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float4));
     if (ctx->bf16 && ctx->attn_max_splits > 1) {
@@ -627,6 +836,7 @@ void wedlm_destroy(wedlm_ctx* ctx) {
     ctx->scratch_arena.release();
     if (ctx->res_host) cudaFreeHost(ctx->res_host);
     for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
+    drop_graph(ctx);
     delete ctx;
 }
 
@@ -660,10 +870,30 @@ wedlm_status wedlm_load_weights(wedlm_ctx* ctx, int32_t tensor, int32_t layer, c
         case WEDLM_T_WD: dst = (char*)ctx->wd[layer]; bytes = d * F * elt; break;
         default: return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad tensor id");
     }
-    CK(cudaMemcpyAsync(dst, src, bytes, src_mem == WEDLM_MEM_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice,
-                       ctx->stream));
+    const cudaMemcpyKind kind = src_mem == WEDLM_MEM_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice;
+    const size_t row = d * elt;
+    if (ctx->bf16 && (tensor == WEDLM_T_WQ || tensor == WEDLM_T_WK)) {
+        // Rows of each 128-dim head are stored with RoPE partners adjacent
+        // (row 2i = dim i, row 2i+1 = dim i+64) so the fused GEMM epilogue
+        // rotates a pair within one warp; outputs return to natural order.
+        const int heads = tensor == WEDLM_T_WQ ? ctx->hq : ctx->hkv;
+        for (int hh = 0; hh < heads; ++hh) {
+            char* hd0 = dst + (size_t)hh * 128 * row;
+            const char* hs0 = (const char*)src + (size_t)hh * 128 * row;
+            CK(cudaMemcpy2DAsync(hd0, 2 * row, hs0, row, row, 64, kind, ctx->stream));
+            CK(cudaMemcpy2DAsync(hd0 + row, 2 * row, hs0 + 64 * row, row, row, 64, kind, ctx->stream));
+        }
+    } else if (ctx->bf16 && (tensor == WEDLM_T_WG || tensor == WEDLM_T_WU)) {
+        // Gate row c -> row 2c, up row c -> row 2c+1 of the fused gate/up
+        // matrix, so SwiGLU pairs sit in adjacent rows of one GEMM tile.
+        char* base = (char*)ctx->wgu[layer] + (tensor == WEDLM_T_WU ? row : 0);
+        CK(cudaMemcpy2DAsync(base, 2 * row, src, row, row, F, kind, ctx->stream));
+    } else {
+        CK(cudaMemcpyAsync(dst, src, bytes, kind, ctx->stream));
+    }
     CK(cudaStreamSynchronize(ctx->stream));
     ctx->loaded[slot] = 1;
+    drop_graph(ctx);
     bool all = true;
     for (uint8_t f : ctx->loaded) all &= f != 0;
     ctx->weights_ready = all;
@@ -681,6 +911,7 @@ wedlm_status wedlm_prefill(wedlm_ctx* ctx, int32_t slot, const int32_t* prompt_i
     if (window < 1 || window > ctx->maxW) return fail(ctx, WEDLM_ERR_INVALID_ARG, "window out of range");
     if (!ctx->weights_ready) return fail(ctx, WEDLM_ERR_STATE, "weights not fully loaded");
     if (ctx->h_W[slot] != 0) return fail(ctx, WEDLM_ERR_STATE, "slot is in use (call wedlm_kv_reset)");
+    drop_graph(ctx);
     for (int i = 0; i < prompt_len; ++i)
         if (prompt_ids[i] < 0 || prompt_ids[i] >= ctx->V)
             return fail(ctx, WEDLM_ERR_INVALID_ARG, "prompt id out of range");
@@ -896,6 +1127,26 @@ wedlm_status wedlm_profile_read(wedlm_ctx* ctx, double* ms, int64_t* launches) {
         if (ms) ms[i] = ctx->prof_ms[i];
         if (launches) launches[i] = ctx->prof_n[i];
     }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_autotune(wedlm_ctx* ctx, int32_t enable) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    ctx->autotune = enable != 0;
+    ctx->tuned.clear();
+    drop_graph(ctx);
+    ctx->eager_key = wedlm_ctx::StepKey();
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_n, int32_t* k_splits,
+                             float* us) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    auto it = ctx->tuned.find({kind, rows});
+    if (it == ctx->tuned.end()) return fail(ctx, WEDLM_ERR_STATE, "no plan recorded for this kind and row count");
+    if (tile_n) *tile_n = it->second.plan.bn;
+    if (k_splits) *k_splits = it->second.plan.splits;
+    if (us) *us = it->second.us;
     return WEDLM_OK;
 }
 

@@ -111,3 +111,30 @@ def test_committed_kv_equals_recompute_bf16(model):
             k, v = eng.debug_kv(b, l, 0, len(seq))
             assert np.abs(k - fk[l]).max() <= LOGIT_TOL * np.abs(fk[l]).max()
             assert np.abs(v - fv[l]).max() <= LOGIT_TOL * np.abs(fv[l]).max()
+
+
+def test_graph_replay_matches_eager_decoding():
+    """A step captured into a CUDA graph and replayed (non-default stream) gives
+    exactly the tokens of eager launches (default stream) with the same launch
+    shapes (autotuning off on both)."""
+    import torch
+    from streaming_decoding_b200 import step_params
+    prompts = _prompts()
+    N, W = 24, 16
+    outs = []
+    for use_stream in (False, True):
+        stream = torch.cuda.Stream() if use_stream else None
+        eng = make_engine(MID, max_batch=3, max_window=16, max_ctx=1024, prefill_chunk=128, stream=stream)
+        eng.autotune(False)
+        for b, p in prompts.items():
+            eng.prefill(b, p, N, W)
+        prm = step_params(0.1, 6.0, False, 16.0)
+        active, steps = 3, 0
+        while active:
+            _, _, active = eng.stream_step(prm)
+            steps += 1
+        eng.stream_step_async(prm, 2)  # finished slots: replays are no-ops
+        outs.append(([eng.read_generated(b) for b in prompts], steps, eng.kernel_launches()))
+        eng.close()
+    assert outs[0][0] == outs[1][0]
+    assert outs[0][1] == outs[1][1]

@@ -1,0 +1,81 @@
+"""Full-size parity, sampled: the Qwen3-8B-shaped bf16 model at batch 16 and
+window 16 (the launch configuration bench.py times) against the fp64 oracle.
+
+The whole batch of 16 prompts (U[128, 1024] tokens) is prefilled and decoded
+for a few steps on the GPU.  One sequence (the shortest prompt, so the oracle
+finishes in about a minute) is then sampled: the oracle recomputes its cache
+and the logits of its masked rows for the step, driven by the GPU's window
+state and committed tokens (teacher forcing), and the GPU's values must agree
+within max relative error 2e-2 (per row, relative to the row's largest logit);
+sampled K/V rows of three layers are compared the same way.  Decisions taken
+from the GPU's own logits must equal the oracle's where comparable."""
+import numpy as np
+import pytest
+
+import synth
+from oracle import wedlm_oracle as O
+from _gpu_util import MARGIN, comparable, oracle_select
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+
+
+def test_full_size_batch16_sampled_against_oracle():
+    from streaming_decoding_b200 import Engine, step_params
+    cfg = synth.CONFIGS["qwen3_8b_b16"]
+    dims = cfg["model"]
+    B, W, N = cfg["B"], cfg["W"], cfg["N"]
+    prompts = synth.prompts(cfg)
+    eng = Engine(dims, max_batch=B, max_window=W, max_ctx=1024 + N, stream=torch.cuda.Stream())
+    eng.load_model(synth.iter_weights(dims, seed=0, dtype="bf16"))
+    for b, p in enumerate(prompts):
+        eng.prefill(b, p, N, W)
+    prm = step_params(cfg["lam"], cfg["tau"], False, cfg["logit_scale"])
+    eng.stream_step_async(prm, 3)
+    b = int(np.argmin([len(p) for p in prompts]))
+    f0, t0 = eng.get_window(b)
+    gen = eng.read_generated(b)
+    eng.stream_step(prm)
+    stride, rows = eng.last_rows()
+    assert (stride, rows) == (W, B * W)
+    kn = eng.debug_read("KN", (B, 3), np.int32)
+    k, n, nf = (int(v) for v in kn[b])
+    perm = eng.debug_read("PERM", rows, np.int32).reshape(B, W)[b, :n]
+    z = eng.debug_read("LOGITS", (rows, dims["V"]), np.float32).reshape(B, W, dims["V"])[b]
+    ht = eng.debug_read("HTILDE", (B, W), np.float32)[b]
+    fl = eng.debug_read("FILL", (B, W), np.uint8)[b]
+    seq = list(prompts[b]) + gen
+    S = len(seq)
+    kv_gpu = {l: eng.debug_kv(b, l, 0, S) for l in (0, 17, 35)}
+    eng.close()
+
+    filled = list(f0) + [0] * (n - len(f0))
+    tokens = list(t0) + [dims["mask_id"]] * (n - len(t0))
+    assert perm.tolist() == O.reorder(filled) and k == O.leading_filled(filled)
+
+    m = O.Model(dims, synth.model_weights(dims, seed=0, dtype="bf16"), cache_fp64=True)
+    cache = O.KVCache.empty(m)
+    _, wk, wv = O.forward_window(m, cache, seq, np.arange(S))
+    cache.append(wk, wv)
+    for l, (kg, vg) in kv_gpu.items():
+        assert np.abs(kg - cache.k[l]).max() <= TOL * np.abs(cache.k[l]).max(), l
+        assert np.abs(vg - cache.v[l]).max() <= TOL * np.abs(cache.v[l]).max(), l
+    order = O.reorder(filled)
+    hidden, _, _ = O.forward_window(m, cache, [tokens[j] if filled[j] else dims["mask_id"] for j in order],
+                                    [S + j for j in order])
+    worst = 0.0
+    for r in range(nf, n):
+        ref = O.lm_logits(m, hidden[r:r + 1], 1.0)[0]
+        err = np.abs(z[r] - ref).max() / np.abs(ref).max()
+        worst = max(worst, err)
+        assert err < TOL, (r, err)
+    Ht, _, fills = oracle_select({perm[r]: z[r] for r in range(nf, n)}, dims["mask_id"], cfg["lam"], cfg["tau"],
+                                 False, cfg["logit_scale"])
+    for j, v in Ht.items():
+        assert abs(ht[j] - v) < MARGIN
+    if comparable(Ht, cfg["tau"], False):
+        assert np.nonzero(fl[:n])[0].tolist() == fills
+    print(f"full-size sampled: sequence {b} (P={len(prompts[b])}, S={S}), {n - nf} masked rows, "
+          f"worst logits rel err {worst:.3e}")
