@@ -35,6 +35,17 @@ pages leave open are marked R1..R16 (the same numbering as the design notes):
       committed length reaches P+N.
   R15 prefill commits the whole prompt; the first window is all masks.
   R16 filled tokens are never re-masked.
+  R19 block-wise ("stop-and-wait") decoding, the comparison baseline: the same
+      step, except that nothing is committed until every slot of the window is
+      filled; then the whole window commits and the next window starts
+      (Summary/Method: block decoding must finalise the entire block before
+      any of it can be cached).
+  R18 the bf16 mode's precision contract: fp32 accumulation of operands held
+      in bf16 at five points (the normed hidden states entering a projection,
+      q/k/v after RoPE (k and v as stored in the cache), the attention output,
+      the SwiGLU product, the final normed hidden state).  ``Model(...,
+      act_round=round_bf16)`` applies exactly those roundings; the default
+      (None) is the exact fp64 definition.
 Parity pins for every function live in tests/test_oracle_*.py.
 """
 from __future__ import annotations
@@ -52,14 +63,23 @@ def _widen(a: np.ndarray) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
+def round_bf16(x) -> np.ndarray:
+    """Round to the nearest bfloat16 (ties to even) via float32, returned as
+    float64 (R18).  Finite inputs only."""
+    u = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 class Model:
     """A causal decoder (RMSNorm, GQA attention with RoPE, SwiGLU FFN, untied LM head).
 
     ``weights`` is the dict built by ``synth.model_weights``; matrices are in
     nn.Linear layout [out, in].  ``cache_fp64`` keeps widened copies (small
-    models); otherwise each matrix is widened when used."""
+    models); otherwise each matrix is widened when used.  ``act_round`` (R18)
+    is applied at the bf16 mode's five rounding points; None = exact."""
 
-    def __init__(self, dims: dict, weights: dict, cache_fp64: bool = True):
+    def __init__(self, dims: dict, weights: dict, cache_fp64: bool = True, act_round=None):
         self.L, self.d = dims["L"], dims["d"]
         self.hq, self.hkv, self.hd = dims["hq"], dims["hkv"], dims["hd"]
         self.F, self.V = dims["F"], dims["V"]
@@ -69,6 +89,10 @@ class Model:
         self.g = self.hq // self.hkv
         self.w = weights
         self._cache = {} if cache_fp64 else None
+        self.act_round = act_round
+
+    def rnd(self, x: np.ndarray) -> np.ndarray:
+        return x if self.act_round is None else self.act_round(x)
 
     def mat(self, name: str, layer: int | None = None) -> np.ndarray:
         key = (name, layer)
@@ -167,19 +191,19 @@ def forward_window(m: Model, cache: KVCache, toks, pos):
     x = m.embed_rows(toks)
     wk, wv = [], []
     for l in range(m.L):
-        h = rms_norm(x, m.mat("attn_norm", l), m.eps)
+        h = m.rnd(rms_norm(x, m.mat("attn_norm", l), m.eps))
         q = (h @ m.mat("wq", l).T).reshape(n, m.hq, m.hd)
         k = (h @ m.mat("wk", l).T).reshape(n, m.hkv, m.hd)
-        v = (h @ m.mat("wv", l).T).reshape(n, m.hkv, m.hd)
-        q = rope(q, pos, m.theta)
-        k = rope(k, pos, m.theta)
+        v = m.rnd((h @ m.mat("wv", l).T).reshape(n, m.hkv, m.hd))
+        q = m.rnd(rope(q, pos, m.theta))
+        k = m.rnd(rope(k, pos, m.theta))
         wk.append(k)
         wv.append(v)
-        a = window_attention(q, cache.k[l], cache.v[l], k, v)
+        a = m.rnd(window_attention(q, cache.k[l], cache.v[l], k, v))
         x = x + a.reshape(n, m.hq * m.hd) @ m.mat("wo", l).T
-        h = rms_norm(x, m.mat("ffn_norm", l), m.eps)
-        x = x + (silu(h @ m.mat("wg", l).T) * (h @ m.mat("wu", l).T)) @ m.mat("wd", l).T
-    return rms_norm(x, m.mat("final_norm"), m.eps), wk, wv
+        h = m.rnd(rms_norm(x, m.mat("ffn_norm", l), m.eps))
+        x = x + m.rnd(silu(h @ m.mat("wg", l).T) * (h @ m.mat("wu", l).T)) @ m.mat("wd", l).T
+    return m.rnd(rms_norm(x, m.mat("final_norm"), m.eps)), wk, wv
 
 
 def lm_logits(m: Model, hidden: np.ndarray, logit_scale: float) -> np.ndarray:
@@ -292,7 +316,8 @@ def prefill(m: Model, prompt, N: int, W: int) -> SeqState:
 
 
 def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
-                logit_scale: float, forward=None, keep_trace: bool = True, choose=None) -> StepTrace | None:
+                logit_scale: float, forward=None, keep_trace: bool = True, choose=None,
+                blockwise: bool = False) -> StepTrace | None:
     """One Streaming Parallel Decoding step (Summary/Method), in the pages' order:
     refill the window with masks, reorder, causal forward, commit the leftmost
     filled run, then fill selected masks (distance-penalised entropy rule).
@@ -301,7 +326,8 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
     replace the model forward (used by tests with a scripted predictor).
     ``choose(step_index, Ht, fills) -> fills`` lets a test make the oracle follow
     another implementation's fill decision where floating point leaves it open;
-    it does not change how anything is computed."""
+    it does not change how anything is computed.  ``blockwise`` selects the
+    block-wise baseline (R19): the commit run is the whole window or nothing."""
     if st.done:
         return None
     # refill: masks appended so the window holds min(W, end - S) slots (R12)
@@ -311,6 +337,8 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
         st.token.append(m.mask_id)
     filled = list(st.filled)
     k = leading_filled(filled)                                  # R1
+    if blockwise and k < n:
+        k = 0                                                   # R19
     perm = reorder(filled)
     toks = [st.token[j] if filled[j] else m.mask_id for j in perm]
     pos = [st.S + j for j in perm]                              # logical positions
@@ -353,14 +381,15 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
 
 def stream_decode(m: Model, prompt, N: int, W: int, lam: float, tau: float,
                   tau_none: bool = False, logit_scale: float = 1.0, max_steps: int | None = None,
-                  forward=None, choose=None) -> SeqState:
-    """Decode N tokens after ``prompt`` with Streaming Parallel Decoding."""
+                  forward=None, choose=None, blockwise: bool = False) -> SeqState:
+    """Decode N tokens after ``prompt`` with Streaming Parallel Decoding (or,
+    with ``blockwise``, the block-wise baseline, R19)."""
     st = prefill(m, prompt, N, W) if forward is None else SeqState(
         prompt=np.asarray(prompt), N=N, W=W, cache=KVCache.empty(m), S=len(prompt), end=len(prompt) + N)
     while not st.done:
         if max_steps is not None and st.steps >= max_steps:
             break
-        stream_step(m, st, lam, tau, tau_none, logit_scale, forward=forward, choose=choose)
+        stream_step(m, st, lam, tau, tau_none, logit_scale, forward=forward, choose=choose, blockwise=blockwise)
     return st
 
 

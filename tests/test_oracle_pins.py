@@ -303,7 +303,8 @@ class _StubModel:
 def test_decode_loop_matches_hand_trace(case):
     m = _StubModel(case["mask_id"])
     st = O.stream_decode(m, np.zeros(case["prompt_len"], np.int64), case["N"], case["W"],
-                         case["lambda"], case["tau"], forward=scripted_forward(case))
+                         case["lambda"], case["tau"], forward=scripted_forward(case),
+                         blockwise=case.get("blockwise", False))
     assert len(st.trace) == len(case["steps"])
     for tr, want in zip(st.trace, case["steps"]):
         assert (tr.S, tr.n, tr.k, tr.perm, tr.committed) == (want["S"], want["n"], want["k"], want["perm"],
@@ -368,6 +369,37 @@ def test_progress_and_workload_invariants(tiny_model, cfg_name, W):
     assert 0 < O.p_cache(st) <= 0.5
     if cfg_name == "tiny_f32_tau":
         assert max(len(tr.fills) for tr in st.trace) >= 2   # the multi-fill branch runs
+
+
+@pytest.mark.parametrize("cfg_name,W", [("tiny_f32_tau", 4), ("tiny_f32", 3)])
+def test_blockwise_commits_whole_windows_and_caches_exactly(tiny_model, cfg_name, W):
+    """Block-wise baseline (R19): every commit is a whole window, the committed
+    K/V still equal a from-scratch recompute, and it never commits more per
+    forward row than streaming does on the same inputs (p_cache ordering)."""
+    cfg = synth.CONFIGS[cfg_name]
+    prompt = synth.prompts(cfg)[0]
+    N = cfg["N"]
+    bw = O.stream_decode(tiny_model, prompt, N, W, cfg["lam"], cfg["tau"], logit_scale=cfg["logit_scale"],
+                         blockwise=True)
+    assert len(bw.out) == N
+    end = len(prompt) + N
+    for tr in bw.trace:
+        assert tr.k in (0, tr.n)
+        assert tr.n == min(W, end - tr.S)
+    fk, fv = O.full_causal_kv(tiny_model, list(prompt) + bw.out)
+    for l in range(tiny_model.L):
+        np.testing.assert_allclose(bw.cache.k[l], fk[l], rtol=1e-10, atol=1e-12)
+    st = O.stream_decode(tiny_model, prompt, N, W, cfg["lam"], cfg["tau"], logit_scale=cfg["logit_scale"])
+    assert O.p_cache(bw) <= O.p_cache(st) + 1e-12
+
+
+def test_blockwise_with_window_one_is_streaming(tiny_model):
+    """With W = 1 a block is one slot, so both decoders take identical steps."""
+    cfg = synth.CONFIGS["tiny_f32"]
+    prompt = synth.prompts(cfg)[0]
+    a = O.stream_decode(tiny_model, prompt, 10, 1, 0.0, cfg["tau"], logit_scale=cfg["logit_scale"])
+    b = O.stream_decode(tiny_model, prompt, 10, 1, 0.0, cfg["tau"], logit_scale=cfg["logit_scale"], blockwise=True)
+    assert a.out == b.out and a.steps == b.steps
 
 
 def test_one_by_one_mode_fills_exactly_one(tiny_model):
@@ -444,3 +476,40 @@ def test_hand_traces_detect_planted_loop_mistakes(monkeypatch, mutation):
         Ht = {int(j): O.penalised_entropy(h, int(j), case["lambda"]) for j, h in case["H"].items()}
         sel_fail += O.select_fills(Ht, tau, case["tau_none"]) != case["fills"]
     assert failures + sel_fail > 0
+
+
+# --------------------------------------------- bf16 precision contract (R18) ---
+def test_round_bf16_matches_torch_conversion():
+    """round_bf16 is float32 -> bfloat16 round-to-nearest-even (torch's conversion)."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-8, 8, 20000),
+                        # exact ties between two bf16 values: low half-word 0x8000, even and odd upper
+                        (np.array([0x3F808000, 0x3F818000, 0xBF808000, 0x40490000], np.uint32)).view(np.float32),
+                        np.array([0.0, -0.0, 1.0, -2.5])])
+    ref = torch.tensor(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x), ref)
+
+
+def test_act_round_hook_applies_only_at_the_contract_points():
+    """With an identity hook the forward is bit-identical to the exact one;
+    with round_bf16 the stored K/V are bf16 values and logits move by bf16-level
+    amounts only."""
+    w = pin_weights(PIN_DIMS)
+    toks = synth.token_ids(6, 0, PIN_DIMS["V"], 13, exclude=PIN_DIMS["mask_id"])
+    pos = np.arange(13)
+    exact = O.Model(PIN_DIMS, w)
+    ident = O.Model(PIN_DIMS, w, act_round=lambda a: a)
+    bf = O.Model(PIN_DIMS, w, act_round=O.round_bf16)
+    he, ke, ve = O.forward_window(exact, O.KVCache.empty(exact), toks, pos)
+    hi, ki, vi = O.forward_window(ident, O.KVCache.empty(ident), toks, pos)
+    hb, kb, vb = O.forward_window(bf, O.KVCache.empty(bf), toks, pos)
+    np.testing.assert_array_equal(hi, he)
+    for l in range(exact.L):
+        np.testing.assert_array_equal(ki[l], ke[l])
+        np.testing.assert_array_equal(O.round_bf16(kb[l]), kb[l])
+        np.testing.assert_array_equal(O.round_bf16(vb[l]), vb[l])
+    np.testing.assert_array_equal(O.round_bf16(hb), hb)
+    ze, zb = O.lm_logits(exact, he, 1.0), O.lm_logits(bf, hb, 1.0)
+    rel = np.abs(zb - ze).max() / np.abs(ze).max()
+    assert 0 < rel < 2e-2, rel
