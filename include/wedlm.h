@@ -229,11 +229,12 @@ wedlm_status wedlm_kernel_launches(const wedlm_ctx* ctx, int64_t* out);
  * accumulation order.  wedlm_autotune clears the recorded shapes. */
 wedlm_status wedlm_autotune(wedlm_ctx* ctx, int32_t enable);
 
-/* The shape recorded for (kind, rows): tile_n activation rows per tile,
- * k_splits slices of K, and the fastest timed launch in microseconds (-1 when
- * the shape came from the cost model).  WEDLM_ERR_STATE if none is recorded. */
-wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_n, int32_t* k_splits,
-                             float* us);
+/* The shape recorded for (kind, rows): tile_w weight rows (128 or 256) by
+ * tile_n activation rows per tile, k_splits slices of K, and the fastest timed
+ * launch in microseconds (-1 when the shape came from the cost model).  Any
+ * output pointer may be NULL.  WEDLM_ERR_STATE if none is recorded. */
+wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_w, int32_t* tile_n,
+                             int32_t* k_splits, float* us);
 
 /* Enable (1) or disable (0) per-kernel timing; enabling clears the totals. */
 wedlm_status wedlm_profile_enable(wedlm_ctx* ctx, int32_t on);

@@ -65,7 +65,7 @@ _SIGS = {
     "wedlm_kernel_launches": (c_i32, [c_vp, ctypes.POINTER(c_i64)]),
     "wedlm_profile_enable": (c_i32, [c_vp, c_i32]),
     "wedlm_autotune": (c_i32, [c_vp, c_i32]),
-    "wedlm_gemm_plan": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "wedlm_gemm_plan": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "wedlm_profile_read": (c_i32, [c_vp, c_vp, c_vp]),
     "wedlm_debug_read": (c_i32, [c_vp, c_i32, c_vp, c_i64]),
     "wedlm_debug_kv": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp]),

@@ -141,11 +141,11 @@ class Engine:
         _check(self.lib.wedlm_autotune(self.ctx, 1 if enable else 0), "wedlm_autotune", self.ctx)
 
     def gemm_plan(self, kind: str, rows: int):
-        """(tile_n, k_splits, us) recorded for a projection kind ('gemm_qkv', ...) at `rows`, or None."""
-        tn, ks, us = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_float()
-        st = self.lib.wedlm_gemm_plan(self.ctx, C["WEDLM_PROF_" + kind.upper()], rows, ctypes.byref(tn),
-                                      ctypes.byref(ks), ctypes.byref(us))
-        return (tn.value, ks.value, round(us.value, 2)) if st == 0 else None
+        """(tile_w, tile_n, k_splits, us) recorded for a projection kind ('gemm_qkv', ...) at `rows`, or None."""
+        tw, tn, ks, us = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32(), ctypes.c_float()
+        st = self.lib.wedlm_gemm_plan(self.ctx, C["WEDLM_PROF_" + kind.upper()], rows, ctypes.byref(tw),
+                                      ctypes.byref(tn), ctypes.byref(ks), ctypes.byref(us))
+        return (tw.value, tn.value, ks.value, round(us.value, 2)) if st == 0 else None
 
     def profile_enable(self, on: bool = True):
         _check(self.lib.wedlm_profile_enable(self.ctx, 1 if on else 0), "wedlm_profile_enable", self.ctx)

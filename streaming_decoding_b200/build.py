@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build", "wedlm")
 LIB = os.path.join(HERE, "libwedlm.so")
-SOURCES = ["kernels.cu", "gemm_tc.cu", "attn_mma.cu", "wedlm.cu", "standalone.cu", "noalloc.cu"]
+SOURCES = ["kernels.cu", "gemm_tc.cu", "attn_tc.cu", "wedlm.cu", "standalone.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.cuh", "gemm_tc.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

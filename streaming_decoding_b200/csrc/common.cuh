@@ -14,6 +14,31 @@ using bf16 = __nv_bfloat16;
 constexpr int kPage = WEDLM_PAGE_TOKENS;
 constexpr int kMaxWindow = 64;
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may begin
+// while the previous kernel of its stream is still running: it must call
+// griddep_wait() (which returns once that kernel has completed and its writes
+// are visible) before touching memory that kernel reads or writes, and calls
+// griddep_launch() after that wait (and after any TMEM allocation) to let the
+// next kernel start early in turn.  Under a plain launch both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Device error word codes (mirrors of the wedlm_status values they map to).
 constexpr int kErrBounds = 1;   // a bounds check refused an access
 constexpr int kErrTimeout = 2;  // a bounded wait gave up

@@ -36,13 +36,20 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int SUB_A_BYTES = BM * BK * 2;  // one 128-row weight sub-tile of a stage
 
-template <int BN> struct PCfg {
+// BN activation rows (MMA N) by WT weight sub-tiles of 128 rows (one MMA each
+// per k-step, sharing the activation operand: WT = 2 halves the activation
+// bytes a CTA moves per output).  NACC accumulators of WT*BN TMEM columns
+// (two when they fit, so a unit's MMAs overlap the previous unit's epilogue).
+template <int BN, int WT> struct PCfg {
+    static constexpr int A_STAGE_BYTES = WT * SUB_A_BYTES;
     static constexpr int B_STAGE_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
     static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 12 ? 12 : (200 * 1024) / STAGE_BYTES;
-    static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    static constexpr int ACC_COLS = WT * BN;
+    static constexpr int NACC = 2 * ACC_COLS <= 512 ? 2 : 1;
+    static constexpr int TMEM_COLS = NACC * ACC_COLS < 32 ? 32 : NACC * ACC_COLS;
     static constexpr int META_BYTES = BN * 16;  // per activation row: live, pos, cache-row offset
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + META_BYTES;
 };
@@ -323,15 +330,17 @@ __device__ __forceinline__ void epilogue_vec4x8(const EpiParams& ep, int n0, int
     }
 }
 
-template <int BN>
+template <int BN, int WT>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
                                                          const __grid_constant__ CUtensorMap tmX, const GemmArgs g) {
-    using C = PCfg<BN>;
+    using C = PCfg<BN, WT>;
+    constexpr int NACC = C::NACC;
+    constexpr int TW = BM * WT;  // weight rows per tile
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+    uint8_t* sB = smem + STAGES * C::A_STAGE_BYTES;
     uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_STAGE_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* accf = empty + STAGES;
@@ -371,28 +380,56 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 
     if (warp == 0) {
         if (lane == 0) {
+            // Weights never depend on the previous kernel: the first ring slots
+            // of the first unit get their weight tiles before the dependency
+            // wait (overlapping that kernel's tail), the activations after it.
             uint32_t it = 0;
+            int pre = 0;
+            if ((int)blockIdx.x < units) {
+                const int split = blockIdx.x % g.splits, tile = blockIdx.x / g.splits;
+                const int n0 = (tile / g.m_tiles) * TW;
+                const int kb0 = split * g.kb_per_split;
+                pre = min(min(KB, kb0 + g.kb_per_split) - kb0, STAGES);
+                for (int i = 0; i < pre; ++i) {
+                    mbar_expect_tx(&full[i], C::STAGE_BYTES);
+#pragma unroll
+                    for (int w = 0; w < WT; ++w)
+                        tma_load_2d(sA + i * C::A_STAGE_BYTES + w * SUB_A_BYTES, &tmW, (kb0 + i) * BK, n0 + w * BM,
+                                    &full[i]);
+                }
+            }
+            griddep_wait();
+            griddep_launch();
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const int split = u % g.splits, tile = u / g.splits;
-                const int n0 = (tile / g.m_tiles) * BM, m0 = (tile % g.m_tiles) * BN;
+                const int n0 = (tile / g.m_tiles) * TW, m0 = (tile % g.m_tiles) * BN;
                 const int kb0 = split * g.kb_per_split;
                 const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
                 for (int i = 0; i < nkb; ++i, ++it) {
                     const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1u, err)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_expect_tx(&full[s], C::STAGE_BYTES);
                     const int kx = (kb0 + i) * BK;
-                    tma_load_2d(sA + s * A_STAGE_BYTES, &tmW, kx, n0, &full[s]);
+                    if ((int)it >= pre) {
+                        const uint32_t ph = (it / STAGES) & 1u;
+                        if (!mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1u, err)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(&full[s], C::STAGE_BYTES);
+#pragma unroll
+                        for (int w = 0; w < WT; ++w)
+                            tma_load_2d(sA + s * C::A_STAGE_BYTES + w * SUB_A_BYTES, &tmW, kx, n0 + w * BM, &full[s]);
+                    }
                     tma_load_2d(sB + s * C::B_STAGE_BYTES, &tmX, kx, m0, &full[s]);
                 }
             }
+        } else {
+            griddep_wait();
+            griddep_launch();
         }
     } else if (warp == 1) {
+        griddep_wait();
+        griddep_launch();
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(BM, BN);
             uint32_t it = 0, j = 0;
@@ -401,10 +438,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 const int split = u % g.splits;
                 const int kb0 = split * g.kb_per_split;
                 const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
-                const uint32_t b = j & 1u, use = j >> 1;
+                const uint32_t b = j % NACC, use = j / NACC;
                 if (!mbar_wait_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err)) break;
                 tc_fence_after();
-                const uint32_t d = tmem + b * BN;
+                const uint32_t d = tmem + b * C::ACC_COLS;
                 for (int i = 0; i < nkb; ++i, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
@@ -413,37 +450,44 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                         break;
                     }
                     tc_fence_after();
-                    const uint8_t* a = sA + s * A_STAGE_BYTES;
+                    const uint8_t* a = sA + s * C::A_STAGE_BYTES;
                     const uint8_t* bb = sB + s * C::B_STAGE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        umma_bf16(d, sdesc_k_sw128(a + kk * 32), sdesc_k_sw128(bb + kk * 32), idesc,
-                                  (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int w = 0; w < WT; ++w)
+                            umma_bf16(d + w * BN, sdesc_k_sw128(a + w * SUB_A_BYTES + kk * 32),
+                                      sdesc_k_sw128(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 umma_commit(&accf[b]);
             }
         }
     } else {
+        griddep_wait();
+        griddep_launch();
         const int q = warp & 3;
         uint32_t j = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++j) {
             const int split = u % g.splits, tile = u / g.splits;
-            const int n0 = (tile / g.m_tiles) * BM, m0 = (tile % g.m_tiles) * BN;
-            const int n = n0 + q * 32 + lane;
-            const uint32_t b = j & 1u, use = j >> 1;
+            const int n0 = (tile / g.m_tiles) * TW, m0 = (tile % g.m_tiles) * BN;
+            const uint32_t b = j % NACC, use = j / NACC;
             const bool ok = epi_all(mbar_wait_bounded(smem_u32(&accf[b]), use & 1u, err));
             if (!ok) break;
             tc_fence_after();
             fill_row_meta<BN>(g.ep, m0, g.M, meta, threadIdx.x - 64);
             epi_bar();
-            const uint32_t taddr = tmem + b * BN + ((uint32_t)(q * 32) << 16);
+            const uint32_t tacc = tmem + b * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
             if (g.splits == 1) {
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    float v[16];
-                    tmem_ld16(taddr + (uint32_t)c, v);
-                    epilogue16(g.ep, n0, n, m0 + c, c, meta, v, g.N, lane);
+                for (int w = 0; w < WT; ++w) {
+                    const int nw = n0 + w * BM, n = nw + q * 32 + lane;
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 16) {
+                        float v[16];
+                        tmem_ld16(tacc + (uint32_t)(w * BN + c), v);
+                        epilogue16(g.ep, nw, n, m0 + c, c, meta, v, g.N, lane);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -451,13 +495,17 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             } else {
                 float* plane = g.ep.ws + (int64_t)split * g.M * g.N;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 16) {
-                    float v[16];
-                    tmem_ld16(taddr + (uint32_t)c, v);
+                for (int w = 0; w < WT; ++w) {
+                    const int n = n0 + w * BM + q * 32 + lane;
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 16) {
+                        float v[16];
+                        tmem_ld16(tacc + (uint32_t)(w * BN + c), v);
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const int m = m0 + c + k;
-                        if (m < g.M && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
+                        for (int k = 0; k < 16; ++k) {
+                            const int m = m0 + c + k;
+                            if (m < g.M && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
+                        }
                     }
                 }
                 tc_fence_before();
@@ -488,49 +536,53 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 const int rows = (BN + g.splits - 1) / g.splits;
                 const int r0 = split * rows, r1 = min(BN, r0 + rows);
                 const int et = threadIdx.x - 64;
-                const int nn = n0 + 4 * (et & 31);
                 const int mr = et >> 5;
-                const bool nok = nn < g.N;  // N % 4 == 0 whenever K is split
 #pragma unroll 1
-                for (int rb = r0 + mr; rb < r1; rb += 4 * 8) {
-                    float4 acc[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int w = 0; w < WT; ++w) {
+                    const int nw = n0 + w * BM;
+                    const int nn = nw + 4 * (et & 31);
+                    const bool nok = nn < g.N;  // N % 4 == 0 whenever K is split
 #pragma unroll 1
-                    for (int sp0 = 0; sp0 < g.splits; sp0 += 4) {
-                        // up to 4 planes x 8 rows of independent loads in flight
-                        float4 t4[4][8];
+                    for (int rb = r0 + mr; rb < r1; rb += 4 * 8) {
+                        float4 acc[8];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float* pl = g.ep.ws + (int64_t)(sp0 + j) * g.M * g.N;
+                        for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+                        for (int sp0 = 0; sp0 < g.splits; sp0 += 4) {
+                            // up to 4 planes x 8 rows of independent loads in flight
+                            float4 t4[4][8];
 #pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                const int rr = rb + 4 * u, m = m0 + rr;
-                                t4[j][u] = (sp0 + j < g.splits && nok && rr < r1 && m < g.M)
-                                               ? __ldcg(reinterpret_cast<const float4*>(pl + (int64_t)m * g.N + nn))
-                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int jj = 0; jj < 4; ++jj) {
+                                const float* pl = g.ep.ws + (int64_t)(sp0 + jj) * g.M * g.N;
+#pragma unroll
+                                for (int u = 0; u < 8; ++u) {
+                                    const int rr = rb + 4 * u, m = m0 + rr;
+                                    t4[jj][u] = (sp0 + jj < g.splits && nok && rr < r1 && m < g.M)
+                                                    ? __ldcg(reinterpret_cast<const float4*>(pl + (int64_t)m * g.N + nn))
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                                }
                             }
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                                for (int u = 0; u < 8; ++u) {
+                                    acc[u].x += t4[jj][u].x;
+                                    acc[u].y += t4[jj][u].y;
+                                    acc[u].z += t4[jj][u].z;
+                                    acc[u].w += t4[jj][u].w;
+                                }
                         }
+                        int mrow[8], krow[8];
+                        bool okr[8];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) {
-                                acc[u].x += t4[j][u].x;
-                                acc[u].y += t4[j][u].y;
-                                acc[u].z += t4[j][u].z;
-                                acc[u].w += t4[j][u].w;
-                            }
+                        for (int u = 0; u < 8; ++u) {
+                            const int rr = rb + 4 * u;
+                            krow[u] = rr < BN ? rr : 0;
+                            mrow[u] = m0 + rr;
+                            okr[u] = nok && rr < r1 && mrow[u] < g.M;
+                        }
+                        epilogue_vec4x8(g.ep, nw, nn, mrow, krow, okr, meta, acc, g.N);
                     }
-                    int mrow[8], krow[8];
-                    bool okr[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int rr = rb + 4 * u;
-                        krow[u] = rr < BN ? rr : 0;
-                        mrow[u] = m0 + rr;
-                        okr[u] = nok && rr < r1 && mrow[u] < g.M;
-                    }
-                    epilogue_vec4x8(g.ep, n0, nn, mrow, krow, okr, meta, acc, g.N);
                 }
                 epi_bar();
                 if (threadIdx.x == 64) {
@@ -561,22 +613,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-template <int BN>
+template <int BN, int WT>
 cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, int grid, cudaStream_t st) {
-    using C = PCfg<BN>;
+    using C = PCfg<BN, WT>;
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
         cudaError_t e =
-            cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            cudaFuncSetAttribute(gemm_tc_kernel<BN, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
-    if (a.splits == 1) {
-        gemm_tc_kernel<BN><<<grid, 192, C::SMEM_BYTES, st>>>(tmW, tmX, a);
-        return cudaGetLastError();
-    }
+    if (a.splits == 1) return launch_pdl(gemm_tc_kernel<BN, WT>, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
     // CTAs of a split tile wait for one another: launch cooperatively so all of
     // them are resident at once (the launch fails instead of deadlocking).
     cudaLaunchConfig_t cfg = {};
@@ -589,7 +638,7 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, tmW, tmX, a);
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, WT>, tmW, tmX, a);
 }
 
 }  // namespace
@@ -597,11 +646,12 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
 namespace {
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
-GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits) {
+GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1) {
     GemmPlan p;
     p.bn = bn;
+    p.wt = wt;
     p.m_tiles = (M + bn - 1) / bn;
-    p.n_tiles = (N + BM - 1) / BM;
+    p.n_tiles = (N + BM * wt - 1) / (BM * wt);
     const int KB = (K + BK - 1) / BK;
     p.kb_per_split = (KB + splits - 1) / splits;
     p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;
@@ -614,13 +664,15 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits) {
 }
 }  // namespace
 
-GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits) {
+GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
+                        int force_wt) {
     const int KB = (K + BK - 1) / BK;
     // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
     const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
     if (force_bn > 0 || force_splits > 0) {
         const int bn = force_bn > 0 ? force_bn : bn_for(M);
-        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)));
+        const int wt = (force_wt == 2 && bn >= 128) ? 2 : 1;
+        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)), wt);
     }
     // Cost in units of one 256-column k-block per CTA: rounds x k-block time x
     // (k-blocks per unit + per-unit overhead + the partial plane's round trip
@@ -665,12 +717,19 @@ cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int
                              const EpiParams& ep, cudaStream_t st) {
     if (p.splits > 1 && (!ep.ws || !ep.counters)) return cudaErrorInvalidValue;
     GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, ep};
+    if (p.wt == 2) {
+        switch (p.bn) {
+            case 128: return launch_bn<128, 2>(tmW, tmX, a, p.grid, st);
+            case 256: return launch_bn<256, 2>(tmW, tmX, a, p.grid, st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     switch (p.bn) {
-        case 16: return launch_bn<16>(tmW, tmX, a, p.grid, st);
-        case 32: return launch_bn<32>(tmW, tmX, a, p.grid, st);
-        case 64: return launch_bn<64>(tmW, tmX, a, p.grid, st);
-        case 128: return launch_bn<128>(tmW, tmX, a, p.grid, st);
-        case 256: return launch_bn<256>(tmW, tmX, a, p.grid, st);
+        case 16: return launch_bn<16, 1>(tmW, tmX, a, p.grid, st);
+        case 32: return launch_bn<32, 1>(tmW, tmX, a, p.grid, st);
+        case 64: return launch_bn<64, 1>(tmW, tmX, a, p.grid, st);
+        case 128: return launch_bn<128, 1>(tmW, tmX, a, p.grid, st);
+        case 256: return launch_bn<256, 1>(tmW, tmX, a, p.grid, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -35,11 +35,13 @@ struct EpiParams {
     int* err = nullptr;
 };
 
-// How Y[M][N] = X[M][K] * W[N][K]^T is cut: tiles of 128 weight rows (MMA M)
-// by bn activation rows (MMA N), K in `splits` slices; units = tiles * splits
-// are dealt round-robin to `grid` persistent CTAs (one per SM).
+// How Y[M][N] = X[M][K] * W[N][K]^T is cut: tiles of 128 * wt weight rows
+// (wt MMAs of M = 128 sharing the activation operand) by bn activation rows
+// (MMA N), K in `splits` slices; units = tiles * splits are dealt round-robin
+// to `grid` persistent CTAs (one per SM).  wt = 2 needs bn >= 128.
 struct GemmPlan {
     int bn = 16;
+    int wt = 1;
     int splits = 1;
     int kb_per_split = 1;
     int m_tiles = 1;
@@ -48,8 +50,10 @@ struct GemmPlan {
 };
 
 // max_splits: the most K slices the caller's partial workspace holds (>= 1).
-// force_bn / force_splits > 0 pin the tile width / split count (tuning hook).
-GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0);
+// force_bn / force_splits > 0 pin the tile width / split count, force_wt = 2
+// selects 256-row weight tiles (tuning hooks).
+GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0,
+                        int force_wt = 0);
 
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 

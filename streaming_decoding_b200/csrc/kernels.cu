@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(256) decode_prepare_kernel(const T* __restrict
                                                              float eps, int d, int mask_id, SlotState ss, RowState rs,
                                                              uint8_t* __restrict__ rowmask, int stride,
                                                              float* __restrict__ x, T* __restrict__ h) {
+    griddep_wait();
+    griddep_launch();
     __shared__ float red[32];
     __shared__ int s_n;
     const int slot = blockIdx.x;
@@ -335,6 +337,8 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(const float* __restr
 constexpr int kNormVec = 8;
 __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ h,
                                                            const float* __restrict__ g, float eps, int d, RowMap rm) {
+    griddep_wait();
+    griddep_launch();
     __shared__ float red[32];
     const int row = blockIdx.x;
     int slot, r;
@@ -366,7 +370,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float* __restri
 
 void launch_rmsnorm_bf16(const float* x, bf16* h, const float* g, float eps, int M, int d, RowMap rm,
                          cudaStream_t st) {
-    rmsnorm_bf16_kernel<<<M, 256, 0, st>>>(x, h, g, eps, d, rm);
+    launch_pdl(rmsnorm_bf16_kernel, dim3(M), dim3(256), 0, st, x, h, g, eps, d, rm);
 }
 
 // SwiGLU: act = silu(gate) * up, gate = columns [0, F), up = [F, 2F).
@@ -448,6 +452,8 @@ __global__ void __launch_bounds__(256) entropy_partial_kernel(const float* __res
                                                               int64_t sstride, int64_t ld, int V, int mask_id,
                                                               float scale, const uint8_t* __restrict__ rowmask,
                                                               int chunks, float4* __restrict__ part) {
+    griddep_wait();
+    griddep_launch();
     const int row = blockIdx.y, c = blockIdx.x;
     if (!rowmask[row]) return;
     const int csz = ((V + chunks - 1) / chunks + 3) & ~3;
@@ -530,6 +536,8 @@ __device__ __forceinline__ int choose_fills(const float* ht, const uint8_t* mask
 // fill the chosen masks with their argmax tokens; slide the window by k.
 __global__ void __launch_bounds__(64) select_commit_kernel(const float4* __restrict__ part, int chunks, SlotState ss,
                                                            RowState rs, int stride, StepKnobs kn, int* err) {
+    griddep_wait();
+    griddep_launch();
     const int slot = blockIdx.x;
     const int n = ss.n[slot];
     __shared__ float sh[kMaxWindow];
@@ -680,7 +688,8 @@ __global__ void __launch_bounds__(64) select_only_kernel(const float4* __restric
 template <typename T>
 void launch_decode_prepare(const T* embed, const float* g, float eps, int d, int mask_id, SlotState ss, RowState rs,
                            uint8_t* rowmask, int n_entries, int stride, float* x, T* h, cudaStream_t st) {
-    decode_prepare_kernel<T><<<n_entries, 256, 0, st>>>(embed, g, eps, d, mask_id, ss, rs, rowmask, stride, x, h);
+    launch_pdl(decode_prepare_kernel<T>, dim3(n_entries), dim3(256), 0, st, embed, g, eps, d, mask_id, ss, rs, rowmask,
+               stride, x, h);
 }
 
 template <typename T>
@@ -736,12 +745,13 @@ void launch_rope_table(float2* cs, int max_pos, int half, int hd, double theta, 
 void launch_entropy_partials(const float* logits, int splits, int64_t sstride, int64_t ld, int V, int mask_id,
                              float scale, const uint8_t* rowmask, int rows, int chunks, float4* part, cudaStream_t st) {
     dim3 grid(chunks, rows);
-    entropy_partial_kernel<<<grid, 256, 0, st>>>(logits, splits, sstride, ld, V, mask_id, scale, rowmask, chunks, part);
+    launch_pdl(entropy_partial_kernel, grid, dim3(256), 0, st, logits, splits, sstride, ld, V, mask_id, scale, rowmask,
+               chunks, part);
 }
 
 void launch_select_commit(const float4* part, int chunks, SlotState ss, RowState rs, int n_entries, int stride,
                           StepKnobs kn, int* err, cudaStream_t st) {
-    select_commit_kernel<<<n_entries, 64, 0, st>>>(part, chunks, ss, rs, stride, kn, err);
+    launch_pdl(select_commit_kernel, dim3(n_entries), dim3(64), 0, st, part, chunks, ss, rs, stride, kn, err);
 }
 
 void launch_reorder_only(const uint8_t* filled, const int32_t* n, const int32_t* S, int n_seq, int stride,

@@ -1,6 +1,8 @@
 // Kernel launch interface of libwedlm (host-callable wrappers).
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace wedlm {
@@ -66,14 +68,17 @@ void launch_select_only(const float4* part, int chunks, const uint8_t* filled, c
 void launch_rowmask_from_filled(const uint8_t* filled, const int32_t* n, int n_seq, int stride,
                                 uint8_t* rowmask, cudaStream_t st);
 
-// bf16 tensor-core paths (gemm_tc.cu, attn_mma.cu).
-struct TmaDesc;
-void launch_attn_bf16(const bf16* q, const bf16* kv_pool, KVLayout kvl, int layer, int hq, int hkv, int hd,
-                      bf16* out, float* part_o, float2* part_ml, int n_entries, int stride, int kv_chunk,
+// bf16 tensor-core paths (gemm_tc.cu, attn_tc.cu).
+// Tensor map over the whole KV pool viewed as [rows][128] bf16, 16-row boxes
+// of 64 dims with the 128-byte swizzle (one box = one page, one half).
+bool make_kv_tmap(CUtensorMap* tm, const bf16* kv_pool, const KVLayout& kvl, int n_layers);
+// Decode/prefill attention.  With more than one key chunk per row tile
+// (kv_chunk < keys), partials go to part_o / part_ml and the last chunk of
+// each (entry, KV head, tile) to finish merges them; `tickets` holds
+// entries * hkv * tiles ints that are zero between launches.
+void launch_attn_bf16(const CUtensorMap& tm_kv, const bf16* q, KVLayout kvl, int layer, int hq, int hkv, bf16* out,
+                      float* part_o, float2* part_ml, int* tickets, int n_entries, int stride, int kv_chunk,
                       int max_splits, SlotState ss, RowMap rm, int* err, cudaStream_t st);
-void launch_attn_combine(const float* part_o, const float2* part_ml, bf16* out, int M, int hq, int hd,
-                         int kv_chunk, int max_splits, int rows_per_tile, SlotState ss, RowMap rm,
-                         cudaStream_t st);
 int attn_rows_per_tile(int group);
 
 }  // namespace wedlm

@@ -132,6 +132,9 @@ struct wedlm_ctx {
     float4* ent_part = nullptr;
     float* attn_po = nullptr;
     float2* attn_pml = nullptr;
+    int* attn_tickets = nullptr;   // [maxB][hkv][tiles] merge tickets of the key-chunked attention
+    size_t n_attn_tickets = 0;
+    CUtensorMap tm_kv{};
     int attn_kv_chunk = 1 << 30, attn_max_splits = 1;
     int32_t* ids_dev = nullptr;
     // step results block for one device->host copy: counts[B], S[B], tokens[B][maxW], err
@@ -242,32 +245,37 @@ wedlm_status gemm_f32(wedlm_ctx* ctx, int kind, const float* X, const float* W, 
 }
 
 // Time the candidate launch shapes of one projection (kind, M) on its real
-// weights with a plain-store epilogue into scratch, and keep the fastest.
-// Runs once per (kind, M) on the context's stream; candidates that do not fit
-// the scratch buffers are skipped.
-void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* tmW, int M, int N, int K) {
+// weights with its real epilogue, and keep the fastest.  The residual add is
+// redirected into the logits scratch; the other epilogues write buffers the
+// launch that follows rewrites anyway (the q / activation scratch, and K/V
+// at the window's own cache positions).  Runs once per (kind, M) on the
+// context's stream; candidates that do not fit the scratch buffers are skipped.
+void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* tmW, int M, int N, int K,
+                    const EpiParams& ep_real) {
     const std::pair<int, int> key(kind, M);
     if (ctx->tuned.count(key)) return;
     ctx->tuned[key] = {plan_gemm_bf16(M, N, K, ctx->num_sms, 1), -1.f};
-    if ((size_t)M * N > ctx->logits_floats) return;
-    std::vector<int> bns;
-    if (M > 128) bns = {256, 128};
-    else if (M > 64) bns = {128, 64};
-    else bns = {M <= 16 ? 16 : M <= 32 ? 32 : 64};
+    EpiParams ep = ep_real;
+    if (ep.kind == EPI_STORE || ep.kind == EPI_RESIDUAL) {
+        if ((size_t)M * N > ctx->logits_floats) return;
+        ep.out = ctx->logits;
+    }
+    // (activation rows per tile, 128-row weight sub-tiles per tile)
+    std::vector<std::pair<int, int>> shapes;
+    if (M > 128) shapes = {{256, 1}, {128, 1}, {256, 2}, {128, 2}};
+    else if (M > 64) shapes = {{128, 1}, {64, 1}, {128, 2}};
+    else shapes = {{M <= 16 ? 16 : M <= 32 ? 32 : 64, 1}};
     cudaEvent_t e0 = prof_event(ctx), e1 = prof_event(ctx);
     float best = 1e30f;
     GemmPlan bestp = ctx->tuned[key].plan;
-    EpiParams ep;
-    ep.kind = EPI_STORE;
-    ep.out = ctx->logits;
     ep.ws = ctx->ws;
     ep.counters = ctx->tile_counters;
     ep.err = ctx->err;
     const int KB = (K + 63) / 64;
-    for (int bn : bns) {
+    for (auto [bn, wt] : shapes) {
         for (int sp : {1, 2, 3, 4, 6, 8, 12, 16}) {
             if (sp > KB || (sp > 1 && N % 4)) continue;
-            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, bn, sp);
+            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, bn, sp, wt);
             if (p.splits != sp) continue;
             if (p.splits > 1 && ((size_t)p.splits * M * N > ctx->ws_floats ||
                                  (size_t)p.m_tiles * p.n_tiles > ctx->n_tile_counters))
@@ -304,7 +312,7 @@ wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMa
                        EpiParams ep, bool tune = true) {
     GemmPlan p;
     if (ctx->autotune && tune) {
-        autotune_shape(ctx, kind, X, tmW, M, N, K);
+        autotune_shape(ctx, kind, X, tmW, M, N, K, ep);
         p = ctx->tuned[{kind, M}].plan;
     } else {
         const size_t plane = (size_t)M * N;
@@ -363,6 +371,8 @@ wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
     // a GEMM that gave up may leave split-K tickets behind
     if (ctx->tile_counters)
         CK(cudaMemsetAsync(ctx->tile_counters, 0, ctx->n_tile_counters * sizeof(int), ctx->stream));
+    if (ctx->attn_tickets)
+        CK(cudaMemsetAsync(ctx->attn_tickets, 0, ctx->n_attn_tickets * sizeof(int), ctx->stream));
     if (code == kErrTimeout) return fail(ctx, WEDLM_ERR_TIMEOUT, "a bounded device wait timed out");
     return fail(ctx, WEDLM_ERR_DEVICE_ASSERT, "a device bounds check fired");
 }
@@ -452,13 +462,8 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
         const int ms = decode ? ctx->attn_max_splits : 1;
         {
             ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
-            launch_attn_bf16(qb, (const bf16*)ctx->kv_pool, ctx->kvl, l, ctx->hq, ctx->hkv, ctx->hd, ao, ctx->attn_po,
-                             ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss, rm, ctx->err, ctx->stream);
-        }
-        if (ms > 1) {
-            ProfScope ps(ctx, WEDLM_PROF_ATTN_COMBINE);
-            launch_attn_combine(ctx->attn_po, ctx->attn_pml, ao, M, ctx->hq, ctx->hd, kc, ms, rt, ctx->ss, rm,
-                                ctx->stream);
+            launch_attn_bf16(ctx->tm_kv, qb, ctx->kvl, l, ctx->hq, ctx->hkv, ao, ctx->attn_po, ctx->attn_pml,
+                             ctx->attn_tickets, n_entries, stride, kc, ms, ctx->ss, rm, ctx->err, ctx->stream);
         }
         e.kind = EPI_RESIDUAL;
         e.out = ctx->x;
@@ -540,6 +545,11 @@ wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, 
     }
     ctx->last_stride = stride;
     ctx->last_M = M;
+    {
+        // launch-configuration errors of the void launch wrappers surface here
+        const cudaError_t le = cudaGetLastError();
+        if (le != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(le));
+    }
     ctx->logits_splits_last = lsp;
     if (ctx->prof && ctx->ev_marks.size() > 4096) prof_collect(ctx);
     return WEDLM_OK;
@@ -754,6 +764,22 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     sa.add((void**)&ctx->rs.perm, (size_t)Mmax * 4);
     sa.add((void**)&ctx->rowmask, (size_t)Mmax);
     sa.add((void**)&ctx->ids_dev, (size_t)ctx->chunk * 4);
+    // Attention key chunks for decode: fixed per context (a sequence's result
+    // does not depend on its batch neighbours), sized so that a full batch at
+    // half the context length gives about two CTAs per SM; at most 2048 keys.
+    if (ctx->bf16) {
+        const int g = ctx->hq / ctx->hkv;
+        const int rt = attn_rows_per_tile(g);
+        const int tiles = (maxW + rt - 1) / rt;
+        const long long pairs = (long long)B * tiles * ctx->hkv;
+        const long long blocks = pairs * std::max(1, (ctx->max_ctx / 2 + 63) / 64);
+        long long cb = (blocks + 2LL * ctx->num_sms - 1) / (2LL * ctx->num_sms);
+        cb = std::max(1LL, std::min(cb, 32LL));
+        ctx->attn_kv_chunk = (int)(cb * 64);
+        ctx->attn_max_splits = (ctx->max_ctx + ctx->attn_kv_chunk - 1) / ctx->attn_kv_chunk;
+        ctx->n_attn_tickets = (size_t)pairs;
+        sa.add((void**)&ctx->attn_tickets, ctx->n_attn_tickets * sizeof(int));
+    }
     if (sa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
     ss.out_count = ctx->res_dev;
     ss.S = ctx->res_dev + B;
@@ -764,18 +790,7 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     ss.gen_cap = ctx->max_ctx;
     if (cudaMallocHost((void**)&ctx->res_host, res_ints * 4) != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
 
-    // Attention key splits for decode (fixed per context so a sequence's
-    // result does not depend on its batch neighbours).
-    if (ctx->bf16) {
-        const int g = ctx->hq / ctx->hkv;
-        const int rt = attn_rows_per_tile(g);
-        const int tiles = (maxW + rt - 1) / rt;
-        const int base = B * tiles * ctx->hkv;
-        int splits = (2 * ctx->num_sms + base - 1) / base;
-        splits = std::max(1, std::min(splits, (ctx->max_ctx + 255) / 256));
-        ctx->attn_kv_chunk = (int)align_up((size_t)((ctx->max_ctx + splits - 1) / splits), 64);
-        ctx->attn_max_splits = (ctx->max_ctx + ctx->attn_kv_chunk - 1) / ctx->attn_kv_chunk;
-    }
+    if (ctx->bf16 && !make_kv_tmap(&ctx->tm_kv, (const bf16*)ctx->kv_pool, ctx->kvl, L)) return bail(WEDLM_ERR_CUDA);
 
     // Scratch.
     Arena& xa = ctx->scratch_arena;
@@ -960,7 +975,8 @@ wedlm_status wedlm_prefill(wedlm_ctx* ctx, int32_t slot, const int32_t* prompt_i
             return s;
         }
         // the ids buffer is reused by the next chunk: wait for this one
-        e = cudaStreamSynchronize(ctx->stream);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
         if (e != cudaSuccess) {
             give_back();
             return fail(ctx, WEDLM_ERR_CUDA, cudaGetErrorString(e));
@@ -1139,11 +1155,12 @@ wedlm_status wedlm_autotune(wedlm_ctx* ctx, int32_t enable) {
     return WEDLM_OK;
 }
 
-wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_n, int32_t* k_splits,
-                             float* us) {
+wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_w, int32_t* tile_n,
+                             int32_t* k_splits, float* us) {
     if (!ctx) return WEDLM_ERR_INVALID_ARG;
     auto it = ctx->tuned.find({kind, rows});
     if (it == ctx->tuned.end()) return fail(ctx, WEDLM_ERR_STATE, "no plan recorded for this kind and row count");
+    if (tile_w) *tile_w = 128 * it->second.plan.wt;
     if (tile_n) *tile_n = it->second.plan.bn;
     if (k_splits) *k_splits = it->second.plan.splits;
     if (us) *us = it->second.us;
