@@ -404,6 +404,20 @@ def sweeps(rep, cfg, a):
         reg[f"x{scale:g}"] = {"tok_per_s": round(com / (ms / 1e3), 2), "ms_per_step": round(ms / n, 4),
                               "committed_per_step": round(com / n, 3)}
     out["regimes_batch16"] = reg
+    # the pages' comparison decoders on the same kernels: block-wise
+    # (stop-and-wait) commits and sampled fills at T = 0.1, batch 16, x4
+    cmp_ = {}
+    scale = cfg["logit_scale"]
+    for name, kw in (("streaming_greedy", {}), ("blockwise_greedy", {"blockwise": True}),
+                     ("streaming_sampled_t0.1", {"temperature": 0.1, "seed": 1234})):
+        rep.admit(prompts, cfg["N"], cfg["W"])
+        prm = step_params(cfg["lam"], cfg["tau"], False, scale, **kw)
+        rep.eng.stream_step_async(prm, a.warmup)
+        n = min(steps, 60)
+        ms, com, _ = rep.timed_async(prm, n, cfg["B"])
+        cmp_[name] = {"tok_per_s": round(com / (ms / 1e3), 2), "ms_per_step": round(ms / n, 4),
+                      "committed_per_step": round(com / n, 3)}
+    out["decoders_batch16_x%g" % scale] = cmp_
     return out
 
 

@@ -153,12 +153,32 @@ wedlm_status wedlm_kv_reset(wedlm_ctx* ctx, int32_t slot);
 /* Decode knobs (sai.science review, Recommended Changes: lambda = 0.10 and
  * tau in {0.3, 0.5, 0.9}; Reproducibility & code: a threshold of None gives
  * one-by-one decoding).  logit_scale multiplies the LM-head logits before
- * entropy and argmax (an inverse temperature; 1 = the model as loaded). */
+ * entropy and argmax (an inverse temperature; 1 = the model as loaded).
+ *
+ * blockwise selects the block-wise ("stop-and-wait") baseline the method is
+ * compared against (hyper.ai summary, Method: block decoding must finalise the
+ * whole block before any of it is cached): nothing is committed until every
+ * slot of the window is filled, then the whole window is.
+ *
+ * temperature > 0 samples each fill token instead of taking the argmax (the
+ * pages' evaluation decodes at T = 0.1, sai.science review, Reproducibility):
+ * token = argmax_v (logit_scale * z_v / temperature + G_v) over v != mask_id
+ * with Gumbel noise G_v = -log(-log(u_v)).  u_v comes from a counter-based
+ * generator built on the SplitMix64 finaliser (Steele, Lea and Flood, "Fast
+ * splittable pseudorandom number generators", 2014), mix(z): z += 0x9E3779B97F4A7C15;
+ * z = (z ^ z >> 30) * 0xBF58476D1CE4E5B9; z = (z ^ z >> 27) * 0x94D049BB133111EB;
+ * z ^= z >> 31.  With h = mix(mix(mix(mix(seed ^ slot) ^ step) ^ position) ^ v)
+ * (slot = batch slot, step = that slot's decode steps so far, position = the
+ * masked slot's logical position), u_v = ((h >> 40) + 0.5) / 2^24.  The
+ * entropy that selects the slots is unchanged (temperature 1). */
 typedef struct wedlm_step_params {
     float   lambda;       /* distance penalty per slot offset (nats) */
     float   tau;          /* fill threshold on H~ (nats), strict < */
     int32_t tau_none;     /* nonzero: fill exactly the argmin each step */
     float   logit_scale;  /* > 0 */
+    int32_t blockwise;    /* nonzero: block-wise baseline (whole-window commits) */
+    float   temperature;  /* 0: greedy fill; > 0: Gumbel-max sampling at this temperature */
+    uint64_t seed;        /* sampling seed (ignored when temperature == 0) */
 } wedlm_step_params;
 
 /* Run one decode step for every active slot (a slot is active from prefill
@@ -268,6 +288,16 @@ wedlm_status wedlm_debug_read(wedlm_ctx* ctx, int32_t item, void* host_dst, int6
  * to fp32, into host arrays of [n][n_kv_heads][head_dim] each. */
 wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t pos0, int32_t n,
                             float* host_k, float* host_v);
+
+/* Residual-stream capture for per-layer comparisons.  While enabled (1), every
+ * decode step keeps x (fp32, the residual stream) entering each layer and
+ * after the last one; wedlm_debug_residual copies layer `layer` (0..n_layers,
+ * n_layers = after the last layer) for the first `rows` physical rows of the
+ * most recent step, [rows][d_model], to host memory.  Enabling allocates
+ * (n_layers + 1) * max_batch * max_window * d_model floats on the device and
+ * turns CUDA-graph replay off; 0 frees it.  Both synchronise the stream. */
+wedlm_status wedlm_debug_capture(wedlm_ctx* ctx, int32_t enable);
+wedlm_status wedlm_debug_residual(wedlm_ctx* ctx, int32_t layer, float* host_dst, int32_t rows);
 
 /* Read / replace a slot's window (host arrays of `n` entries; replacing is
  * used to drive both implementations from the same state). */

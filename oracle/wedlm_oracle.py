@@ -35,6 +35,13 @@ pages leave open are marked R1..R16 (the same numbering as the design notes):
       committed length reaches P+N.
   R15 prefill commits the whole prompt; the first window is all masks.
   R16 filled tokens are never re-masked.
+  R20 sampled fills (the pages decode at temperature 0.1): the fill token of a
+      selected slot is argmax_v (logit_scale * z_v / T + G_v), v != mask, with
+      Gumbel noise G_v = -log(-log u_v) (the Gumbel-max form of sampling from
+      softmax(logit_scale * z / T)); u_v comes from a counter-based generator on
+      the SplitMix64 finaliser keyed by (seed, batch slot, the slot's decode
+      step, logical position, v).  Slot selection still uses the temperature-1
+      entropy (R3).
   R19 block-wise ("stop-and-wait") decoding, the comparison baseline: the same
       step, except that nothing is committed until every slot of the window is
       filled; then the whole window commits and the next window starts
@@ -181,29 +188,42 @@ class KVCache:
             self.v[l] = np.concatenate([self.v[l], v_rows[l]], axis=0)
 
 
+def layer_forward(m: Model, l: int, x: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, pos):
+    """Layer l of the decoder on window rows x [n, d] (physical order) at logical
+    positions ``pos``, attending to a committed cache (k_cache, v_cache) of that
+    layer.  Returns (x after the layer, window K [n,hkv,hd], window V)."""
+    n = x.shape[0]
+    pos = np.asarray(pos, dtype=np.float64)
+    h = m.rnd(rms_norm(x, m.mat("attn_norm", l), m.eps))
+    q = (h @ m.mat("wq", l).T).reshape(n, m.hq, m.hd)
+    k = (h @ m.mat("wk", l).T).reshape(n, m.hkv, m.hd)
+    v = m.rnd((h @ m.mat("wv", l).T).reshape(n, m.hkv, m.hd))
+    q = m.rnd(rope(q, pos, m.theta))
+    k = m.rnd(rope(k, pos, m.theta))
+    a = m.rnd(window_attention(q, k_cache, v_cache, k, v))
+    x = x + a.reshape(n, m.hq * m.hd) @ m.mat("wo", l).T
+    h = m.rnd(rms_norm(x, m.mat("ffn_norm", l), m.eps))
+    x = x + m.rnd(silu(h @ m.mat("wg", l).T) * (h @ m.mat("wu", l).T)) @ m.mat("wd", l).T
+    return x, k, v
+
+
+def final_hidden(m: Model, x: np.ndarray) -> np.ndarray:
+    """Final RMSNorm of the residual stream (the LM head's input)."""
+    return m.rnd(rms_norm(x, m.mat("final_norm"), m.eps))
+
+
 def forward_window(m: Model, cache: KVCache, toks, pos):
     """Forward of window rows (physical order) against a committed cache.
 
     Returns (final-normed hidden [n, d], per-layer window K [n,hkv,hd], window V)."""
     toks = np.asarray(toks)
-    pos = np.asarray(pos, dtype=np.float64)
-    n = len(toks)
     x = m.embed_rows(toks)
     wk, wv = [], []
     for l in range(m.L):
-        h = m.rnd(rms_norm(x, m.mat("attn_norm", l), m.eps))
-        q = (h @ m.mat("wq", l).T).reshape(n, m.hq, m.hd)
-        k = (h @ m.mat("wk", l).T).reshape(n, m.hkv, m.hd)
-        v = m.rnd((h @ m.mat("wv", l).T).reshape(n, m.hkv, m.hd))
-        q = m.rnd(rope(q, pos, m.theta))
-        k = m.rnd(rope(k, pos, m.theta))
+        x, k, v = layer_forward(m, l, x, cache.k[l], cache.v[l], pos)
         wk.append(k)
         wv.append(v)
-        a = m.rnd(window_attention(q, cache.k[l], cache.v[l], k, v))
-        x = x + a.reshape(n, m.hq * m.hd) @ m.mat("wo", l).T
-        h = m.rnd(rms_norm(x, m.mat("ffn_norm", l), m.eps))
-        x = x + m.rnd(silu(h @ m.mat("wg", l).T) * (h @ m.mat("wu", l).T)) @ m.mat("wd", l).T
-    return m.rnd(rms_norm(x, m.mat("final_norm"), m.eps)), wk, wv
+    return final_hidden(m, x), wk, wv
 
 
 def lm_logits(m: Model, hidden: np.ndarray, logit_scale: float) -> np.ndarray:
@@ -268,6 +288,39 @@ def leading_filled(filled) -> int:
     return k
 
 
+# -------------------------------------------------------------- sampling ---
+_GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+
+
+def mix64(z) -> np.ndarray:
+    """SplitMix64 output function (Steele, Lea and Flood, "Fast splittable
+    pseudorandom number generators", OOPSLA 2014) on uint64 (wrapping):
+    z += golden gamma, then two xor-shift-multiply rounds and a final xor-shift."""
+    with np.errstate(over="ignore"):
+        z = np.asarray(z, dtype=np.uint64) + _GOLDEN
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+def sampling_uniforms(seed: int, slot: int, step: int, position: int, V: int) -> np.ndarray:
+    """u_v in (0, 1) for v = 0..V-1 (R20): h = mix(mix(mix(mix(seed ^ slot) ^ step)
+    ^ position) ^ v), u = ((h >> 40) + 1/2) / 2^24."""
+    h = mix64(np.uint64(seed) ^ np.uint64(slot))
+    h = mix64(h ^ np.uint64(step))
+    h = mix64(h ^ np.uint64(position))
+    h = mix64(h ^ np.arange(V, dtype=np.uint64))
+    return ((h >> np.uint64(40)).astype(np.float64) + 0.5) / float(1 << 24)
+
+
+def sample_token(z: np.ndarray, mask_id: int, logit_scale: float, temperature: float, u: np.ndarray) -> int:
+    """Gumbel-max draw from softmax(logit_scale * z / temperature) over ids != mask_id (R20)."""
+    key = np.array(z, dtype=np.float64) * (logit_scale / temperature) - np.log(-np.log(u))
+    if 0 <= mask_id < key.shape[0]:
+        key[mask_id] = -np.inf
+    return int(np.argmax(key))
+
+
 # ------------------------------------------------------------- decoding ---
 @dataclass
 class StepTrace:
@@ -317,7 +370,8 @@ def prefill(m: Model, prompt, N: int, W: int) -> SeqState:
 
 def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
                 logit_scale: float, forward=None, keep_trace: bool = True, choose=None,
-                blockwise: bool = False) -> StepTrace | None:
+                blockwise: bool = False, temperature: float = 0.0, seed: int = 0,
+                slot: int = 0) -> StepTrace | None:
     """One Streaming Parallel Decoding step (Summary/Method), in the pages' order:
     refill the window with masks, reorder, causal forward, commit the leftmost
     filled run, then fill selected masks (distance-penalised entropy rule).
@@ -327,7 +381,9 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
     ``choose(step_index, Ht, fills) -> fills`` lets a test make the oracle follow
     another implementation's fill decision where floating point leaves it open;
     it does not change how anything is computed.  ``blockwise`` selects the
-    block-wise baseline (R19): the commit run is the whole window or nothing."""
+    block-wise baseline (R19): the commit run is the whole window or nothing.
+    ``temperature`` > 0 samples the fill tokens (R20) with ``seed``; ``slot``
+    is the sequence's batch slot (one of the sampler's counters)."""
     if st.done:
         return None
     # refill: masks appended so the window holds min(W, end - S) slots (R12)
@@ -364,7 +420,11 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
         fills = list(choose(st.steps, Ht, fills))
     for j in fills:
         st.filled[j] = True
-        st.token[j] = amax[j]
+        if temperature > 0:
+            u = sampling_uniforms(seed, slot, st.steps, st.S + j, len(logits[j]))
+            st.token[j] = sample_token(logits[j], m.mask_id, 1.0, temperature, u)
+        else:
+            st.token[j] = amax[j]
     # slide the window past the committed run
     st.filled = st.filled[k:]
     st.token = st.token[k:]
@@ -381,7 +441,8 @@ def stream_step(m: Model, st: SeqState, lam: float, tau: float, tau_none: bool,
 
 def stream_decode(m: Model, prompt, N: int, W: int, lam: float, tau: float,
                   tau_none: bool = False, logit_scale: float = 1.0, max_steps: int | None = None,
-                  forward=None, choose=None, blockwise: bool = False) -> SeqState:
+                  forward=None, choose=None, blockwise: bool = False, temperature: float = 0.0,
+                  seed: int = 0, slot: int = 0) -> SeqState:
     """Decode N tokens after ``prompt`` with Streaming Parallel Decoding (or,
     with ``blockwise``, the block-wise baseline, R19)."""
     st = prefill(m, prompt, N, W) if forward is None else SeqState(
@@ -389,7 +450,8 @@ def stream_decode(m: Model, prompt, N: int, W: int, lam: float, tau: float,
     while not st.done:
         if max_steps is not None and st.steps >= max_steps:
             break
-        stream_step(m, st, lam, tau, tau_none, logit_scale, forward=forward, choose=choose, blockwise=blockwise)
+        stream_step(m, st, lam, tau, tau_none, logit_scale, forward=forward, choose=choose, blockwise=blockwise,
+                    temperature=temperature, seed=seed, slot=slot)
     return st
 
 

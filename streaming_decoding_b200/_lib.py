@@ -26,7 +26,8 @@ class ModelCfg(ctypes.Structure):
 
 
 class StepParams(ctypes.Structure):
-    _fields_ = [("lambda_", c_f32), ("tau", c_f32), ("tau_none", c_i32), ("logit_scale", c_f32)]
+    _fields_ = [("lambda_", c_f32), ("tau", c_f32), ("tau_none", c_i32), ("logit_scale", c_f32),
+                ("blockwise", c_i32), ("temperature", c_f32), ("seed", ctypes.c_uint64)]
 
 
 class SeqStats(ctypes.Structure):
@@ -65,6 +66,8 @@ _SIGS = {
     "wedlm_kernel_launches": (c_i32, [c_vp, ctypes.POINTER(c_i64)]),
     "wedlm_profile_enable": (c_i32, [c_vp, c_i32]),
     "wedlm_autotune": (c_i32, [c_vp, c_i32]),
+    "wedlm_debug_capture": (c_i32, [c_vp, c_i32]),
+    "wedlm_debug_residual": (c_i32, [c_vp, c_i32, c_vp, c_i32]),
     "wedlm_gemm_plan": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "wedlm_profile_read": (c_i32, [c_vp, c_vp, c_vp]),
     "wedlm_debug_read": (c_i32, [c_vp, c_i32, c_vp, c_i64]),

@@ -31,8 +31,10 @@ def _check(st: int, where: str, ctx=None):
         raise WedlmError(st, where, detail)
 
 
-def step_params(lam: float, tau: float, tau_none: bool = False, logit_scale: float = 1.0) -> StepParams:
-    return StepParams(float(lam), float(tau), 1 if tau_none else 0, float(logit_scale))
+def step_params(lam: float, tau: float, tau_none: bool = False, logit_scale: float = 1.0, blockwise: bool = False,
+                temperature: float = 0.0, seed: int = 0) -> StepParams:
+    return StepParams(float(lam), float(tau), 1 if tau_none else 0, float(logit_scale), 1 if blockwise else 0,
+                      float(temperature), int(seed))
 
 
 class Engine:
@@ -139,6 +141,17 @@ class Engine:
 
     def autotune(self, enable: bool = True):
         _check(self.lib.wedlm_autotune(self.ctx, 1 if enable else 0), "wedlm_autotune", self.ctx)
+
+    def debug_capture(self, enable: bool = True):
+        """Keep the residual stream at every layer boundary of each decode step (test hook)."""
+        _check(self.lib.wedlm_debug_capture(self.ctx, 1 if enable else 0), "wedlm_debug_capture", self.ctx)
+
+    def debug_residual(self, layer: int, rows: int) -> np.ndarray:
+        """x entering `layer` (layer = L: after the last layer), [rows][d] fp32, of the last step."""
+        out = np.empty((rows, self.dims["d"]), np.float32)
+        _check(self.lib.wedlm_debug_residual(self.ctx, layer, out.ctypes.data, rows), "wedlm_debug_residual",
+               self.ctx)
+        return out
 
     def gemm_plan(self, kind: str, rows: int):
         """(tile_w, tile_n, k_splits, us) recorded for a projection kind ('gemm_qkv', ...) at `rows`, or None."""

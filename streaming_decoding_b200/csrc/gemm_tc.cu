@@ -389,7 +389,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 const int split = blockIdx.x % g.splits, tile = blockIdx.x / g.splits;
                 const int n0 = (tile / g.m_tiles) * TW;
                 const int kb0 = split * g.kb_per_split;
-                pre = min(min(KB, kb0 + g.kb_per_split) - kb0, STAGES);
+                const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
+                pre = min(nkb, STAGES);
                 for (int i = 0; i < pre; ++i) {
                     mbar_expect_tx(&full[i], C::STAGE_BYTES);
 #pragma unroll
@@ -698,6 +699,18 @@ GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int fo
         }
     }
     return best_p;
+}
+
+bool encode_tmap_bf16(CUtensorMap* tm, const void* base, int rank, const cuuint64_t* gdim, const cuuint64_t* gstride,
+                      const cuuint32_t* box) {
+    auto fn = encode_fn();
+    if (!fn || rank < 1 || rank > 5) return false;
+    cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                    const_cast<cuuint64_t*>(gdim), const_cast<cuuint64_t*>(gstride), const_cast<cuuint32_t*>(box),
+                    estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {

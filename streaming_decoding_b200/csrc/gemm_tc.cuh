@@ -56,6 +56,10 @@ GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int fo
                         int force_wt = 0);
 
 bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// Any-rank bf16 tensor map with the 128-byte swizzle (box[0] * 2 bytes must be
+// 128); gstride[i] is the byte stride of dimension i + 1.
+bool encode_tmap_bf16(CUtensorMap* tm, const void* base, int rank, const cuuint64_t* gdim, const cuuint64_t* gstride,
+                      const cuuint32_t* box);
 
 // tmW: weights [N][K], box rows 128; tmX: activations [>=M][K], box rows plan.bn.
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K,

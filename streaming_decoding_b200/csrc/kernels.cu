@@ -29,77 +29,87 @@ __device__ void embed_norm_row(const T* __restrict__ E, int d, int tok, const fl
     for (int c = threadIdx.x; c < d; c += blockDim.x) h[c] = from_f32<T>(x[c] * inv * g[c]);
 }
 
-// Decode step window preparation, one CTA per batch entry [Method]:
-//   refill with masks to min(W, end - S) slots; k = leftmost filled run;
-//   stable partition (filled ascending, then masks ascending); logical
-//   position S + offset per physical row; embed + first RMSNorm.
+// Decode step window preparation [Method]: refill with masks to
+// min(W, end - S) slots; k = leftmost filled run; stable partition (filled
+// ascending, then masks ascending); logical position S + offset per physical
+// row; embed + first RMSNorm.  One CTA per (batch entry, physical row): each
+// derives its entry's partition in shared memory from the window as it was
+// before this step's refill (slots past the old window length count as
+// masks), and CTA (entry, 0) writes the entry's updated window state.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_prepare_kernel(const T* __restrict__ embed, const float* __restrict__ g,
                                                              float eps, int d, int mask_id, SlotState ss, RowState rs,
                                                              uint8_t* __restrict__ rowmask, int stride,
-                                                             float* __restrict__ x, T* __restrict__ h) {
+                                                             float* __restrict__ x, T* __restrict__ h, int blockwise) {
     griddep_wait();
     griddep_launch();
     __shared__ float red[32];
-    __shared__ int s_n;
-    const int slot = blockIdx.x;
+    __shared__ uint8_t s_f[kMaxWindow];
+    __shared__ int32_t s_t[kMaxWindow];
+    __shared__ int32_t s_perm[kMaxWindow];
+    __shared__ int s_k, s_nf;
+    const int slot = blockIdx.x, r = blockIdx.y;
     const int base = slot * stride;
-    if (threadIdx.x == 0) {
-        int n = 0;
-        const int W = ss.W[slot];
-        const int S = ss.S[slot];
-        const int end = ss.end[slot];
-        uint8_t* f = ss.filled + (int64_t)slot * ss.maxW;
-        int32_t* t = ss.token + (int64_t)slot * ss.maxW;
-        if (W > 0 && S < end) {
-            n = min(min(W, end - S), stride);
-            for (int j = ss.wlen[slot]; j < n; ++j) {  // refill
-                f[j] = 0;
-                t[j] = mask_id;
-            }
-            ss.wlen[slot] = n;
-        }
-        int k = 0;
-        while (k < n && f[k]) ++k;
-        int nf = 0;
-        for (int j = 0; j < n; ++j)
-            if (f[j]) {
-                rs.perm[base + nf] = j;
-                ++nf;
-            }
-        int m = nf;
-        for (int j = 0; j < n; ++j)
-            if (!f[j]) rs.perm[base + m++] = j;
-        for (int r = 0; r < stride; ++r) {
-            if (r < n) {
-                const int j = rs.perm[base + r];
-                rs.pos[base + r] = S + j;
-                rs.tok[base + r] = f[j] ? t[j] : mask_id;
-                rowmask[base + r] = f[j] ? 0 : 1;
-            } else {
-                rs.perm[base + r] = -1;
-                rs.pos[base + r] = -1;
-                rs.tok[base + r] = -1;
-                rowmask[base + r] = 0;
-            }
-        }
-        ss.n[slot] = n;
-        ss.k[slot] = k;
-        ss.nf[slot] = nf;
-        s_n = n;
+    const int W = ss.W[slot], S = ss.S[slot], end = ss.end[slot], wlen = ss.wlen[slot];
+    const bool active = W > 0 && S < end;
+    const int n = active ? min(min(W, end - S), stride) : 0;
+    uint8_t* f = ss.filled + (int64_t)slot * ss.maxW;
+    int32_t* t = ss.token + (int64_t)slot * ss.maxW;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        const bool fj = j < wlen && f[j];
+        s_f[j] = fj ? 1 : 0;
+        s_t[j] = fj ? t[j] : mask_id;
     }
     __syncthreads();
-    const int n = s_n;
-    for (int r = 0; r < stride; ++r) {
-        float* xr = x + (int64_t)(base + r) * d;
-        T* hr = h + (int64_t)(base + r) * d;
-        if (r < n) {
-            embed_norm_row<T>(embed, d, rs.tok[base + r], g, eps, xr, hr, red);
-        } else {
-            for (int c = threadIdx.x; c < d; c += blockDim.x) {
-                xr[c] = 0.f;
-                hr[c] = from_f32<T>(0.f);
-            }
+    if (threadIdx.x == 0) {
+        int nf = 0;
+        for (int j = 0; j < n; ++j)
+            if (s_f[j]) s_perm[nf++] = j;
+        int m = nf;
+        for (int j = 0; j < n; ++j)
+            if (!s_f[j]) s_perm[m++] = j;
+        int k = 0;
+        while (k < n && s_f[k]) ++k;
+        if (blockwise && k < n) k = 0;  // block-wise baseline: the whole window or nothing
+        s_k = k;
+        s_nf = nf;
+    }
+    __syncthreads();
+    if (r == 0) {
+        for (int j = wlen + threadIdx.x; j < n; j += blockDim.x) {  // refill
+            f[j] = 0;
+            t[j] = mask_id;
+        }
+        // (the window length itself is rewritten by the step's commit: every
+        // CTA of this launch reads the old value)
+        if (threadIdx.x == 0) {
+            ss.n[slot] = n;
+            ss.k[slot] = s_k;
+            ss.nf[slot] = s_nf;
+        }
+    }
+    float* xr = x + (int64_t)(base + r) * d;
+    T* hr = h + (int64_t)(base + r) * d;
+    if (r < n) {
+        const int j = s_perm[r];
+        const int tok = s_f[j] ? s_t[j] : mask_id;
+        if (threadIdx.x == 0) {
+            rs.perm[base + r] = j;
+            rs.pos[base + r] = S + j;
+            rs.tok[base + r] = tok;
+            rowmask[base + r] = s_f[j] ? 0 : 1;
+        }
+        embed_norm_row<T>(embed, d, tok, g, eps, xr, hr, red);
+    } else {
+        if (threadIdx.x == 0) {
+            rs.perm[base + r] = -1;
+            rs.pos[base + r] = -1;
+            rs.tok[base + r] = -1;
+            rowmask[base + r] = 0;
+        }
+        for (int c = threadIdx.x; c < d; c += blockDim.x) {
+            xr[c] = 0.f;
+            hr[c] = from_f32<T>(0.f);
         }
     }
 }
@@ -448,10 +458,37 @@ __device__ __forceinline__ EntAcc ent_shfl_merge(EntAcc e, int o) {
     return ent_merge(e, y);
 }
 
+// Sampled fills (temperature T > 0): Gumbel-max, token = argmax_v
+// (scale z_v / T + G_v), G_v = -log(-log u_v), with u_v from a counter-based
+// generator on the SplitMix64 output function (Steele, Lea and Flood, OOPSLA
+// 2014) keyed by (seed, slot, the slot's decode step, position, v).
+__device__ __forceinline__ unsigned long long splitmix_out(unsigned long long z) {
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+struct SampAcc {
+    float k;
+    int a;
+};
+
+__device__ __forceinline__ void samp_push(SampAcc& q, float key, int idx) {
+    if (key > q.k || (key == q.k && idx < q.a)) {
+        q.k = key;
+        q.a = idx;
+    }
+}
+
+__device__ __forceinline__ SampAcc samp_merge(SampAcc x, SampAcc y) {
+    return (y.k > x.k || (y.k == x.k && y.a < x.a)) ? y : x;
+}
+
 __global__ void __launch_bounds__(256) entropy_partial_kernel(const float* __restrict__ logits, int splits,
                                                               int64_t sstride, int64_t ld, int V, int mask_id,
                                                               float scale, const uint8_t* __restrict__ rowmask,
-                                                              int chunks, float4* __restrict__ part) {
+                                                              int chunks, float4* __restrict__ part, SampleArgs sa) {
     griddep_wait();
     griddep_launch();
     const int row = blockIdx.y, c = blockIdx.x;
@@ -459,39 +496,79 @@ __global__ void __launch_bounds__(256) entropy_partial_kernel(const float* __res
     const int csz = ((V + chunks - 1) / chunks + 3) & ~3;
     const int v0 = c * csz, v1 = min(V, v0 + csz);
     EntAcc e{-INFINITY, 0.f, 0.f, INT_MAX};
+    SampAcc q{-INFINITY, INT_MAX};
+    const bool sampling = sa.inv_t > 0.f;
+    unsigned long long hrow = 0;
+    if (sampling) {
+        const int slot = row / sa.stride;
+        hrow = splitmix_out(sa.seed ^ (unsigned long long)slot);
+        hrow = splitmix_out(hrow ^ (unsigned long long)sa.steps[(int64_t)slot * 4]);
+        hrow = splitmix_out(hrow ^ (unsigned long long)(long long)sa.pos[row]);
+    }
+    const float kz = scale * sa.inv_t;
+    auto push = [&](float z, int id) {
+        ent_push(e, scale * z, id);
+        if (sampling) {
+            const unsigned long long h = splitmix_out(hrow ^ (unsigned long long)id);
+            const float u = ((float)(h >> 40) + 0.5f) * 5.9604644775390625e-8f;  // 2^-24
+            samp_push(q, kz * z - logf(-logf(u)), id);
+        }
+    };
     const float* zr = logits + (int64_t)row * ld;
     if (splits == 1 && (ld & 3) == 0) {
         const int nvec = (v1 - v0) >> 2;
         const float4* z4 = reinterpret_cast<const float4*>(zr + v0);
         for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-            const float4 q = __ldg(z4 + i);
+            const float4 z = __ldg(z4 + i);
             const int id = v0 + 4 * i;
-            if (id != mask_id) ent_push(e, scale * q.x, id);
-            if (id + 1 != mask_id) ent_push(e, scale * q.y, id + 1);
-            if (id + 2 != mask_id) ent_push(e, scale * q.z, id + 2);
-            if (id + 3 != mask_id) ent_push(e, scale * q.w, id + 3);
+            if (id != mask_id) push(z.x, id);
+            if (id + 1 != mask_id) push(z.y, id + 1);
+            if (id + 2 != mask_id) push(z.z, id + 2);
+            if (id + 3 != mask_id) push(z.w, id + 3);
         }
         for (int id = v0 + 4 * nvec + threadIdx.x; id < v1; id += blockDim.x)
-            if (id != mask_id) ent_push(e, scale * zr[id], id);
+            if (id != mask_id) push(zr[id], id);
     } else {
         for (int id = v0 + threadIdx.x; id < v1; id += blockDim.x) {
             if (id == mask_id) continue;
             float z = 0.f;
             for (int s = 0; s < splits; ++s) z += logits[s * sstride + (int64_t)row * ld + id];
-            ent_push(e, scale * z, id);
+            push(z, id);
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) e = ent_shfl_merge(e, o);
+    for (int o = 16; o > 0; o >>= 1) {
+        e = ent_shfl_merge(e, o);
+        SampAcc y{__shfl_xor_sync(0xffffffffu, q.k, o), __shfl_xor_sync(0xffffffffu, q.a, o)};
+        q = samp_merge(q, y);
+    }
     __shared__ EntAcc sh[8];
+    __shared__ SampAcc shq[8];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) sh[warp] = e;
+    if (lane == 0) {
+        sh[warp] = e;
+        shq[warp] = q;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         EntAcc t = sh[0];
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) t = ent_merge(t, sh[w]);
+        SampAcc tq = shq[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) {
+            t = ent_merge(t, sh[w]);
+            tq = samp_merge(tq, shq[w]);
+        }
         part[(int64_t)row * chunks + c] = make_float4(t.m, t.s, t.t, __int_as_float(t.a));
+        if (sampling) sa.part[(int64_t)row * chunks + c] = make_float2(tq.k, __int_as_float(tq.a));
     }
+}
+
+__device__ __forceinline__ int combine_sample(const float2* part, int chunks, int row) {
+    SampAcc q{-INFINITY, INT_MAX};
+    for (int c = 0; c < chunks; ++c) {
+        const float2 v = part[(int64_t)row * chunks + c];
+        q = samp_merge(q, SampAcc{v.x, __float_as_int(v.y)});
+    }
+    return q.a;
 }
 
 __device__ __forceinline__ void combine_entropy(const float4* part, int chunks, int row, float& H, int& a) {
@@ -534,7 +611,8 @@ __device__ __forceinline__ int choose_fills(const float* ht, const uint8_t* mask
 // [Method]: H~_j = H_j + lambda * j over masked slots; commit the k slots of
 // the leftmost filled run (their K/V already sit at cache positions S..S+k-1);
 // fill the chosen masks with their argmax tokens; slide the window by k.
-__global__ void __launch_bounds__(64) select_commit_kernel(const float4* __restrict__ part, int chunks, SlotState ss,
+__global__ void __launch_bounds__(64) select_commit_kernel(const float4* __restrict__ part,
+                                                           const float2* __restrict__ spart, int chunks, SlotState ss,
                                                            RowState rs, int stride, StepKnobs kn, int* err) {
     griddep_wait();
     griddep_launch();
@@ -568,6 +646,7 @@ __global__ void __launch_bounds__(64) select_commit_kernel(const float4* __restr
         float H;
         int a;
         combine_entropy(part, chunks, row, H, a);
+        if (kn.temperature > 0.f) a = combine_sample(spart, chunks, row);  // the fill's sampled token
         if (j >= 0 && j < n) {
             sh[j] = H + kn.lambda * (float)j;
             sa[j] = a;
@@ -687,9 +766,10 @@ __global__ void __launch_bounds__(64) select_only_kernel(const float4* __restric
 // Host launch wrappers.
 template <typename T>
 void launch_decode_prepare(const T* embed, const float* g, float eps, int d, int mask_id, SlotState ss, RowState rs,
-                           uint8_t* rowmask, int n_entries, int stride, float* x, T* h, cudaStream_t st) {
-    launch_pdl(decode_prepare_kernel<T>, dim3(n_entries), dim3(256), 0, st, embed, g, eps, d, mask_id, ss, rs, rowmask,
-               stride, x, h);
+                           uint8_t* rowmask, int n_entries, int stride, float* x, T* h, int blockwise,
+                           cudaStream_t st) {
+    launch_pdl(decode_prepare_kernel<T>, dim3(n_entries, stride), dim3(256), 0, st, embed, g, eps, d, mask_id, ss, rs,
+               rowmask, stride, x, h, blockwise);
 }
 
 template <typename T>
@@ -743,15 +823,16 @@ void launch_rope_table(float2* cs, int max_pos, int half, int hd, double theta, 
 }
 
 void launch_entropy_partials(const float* logits, int splits, int64_t sstride, int64_t ld, int V, int mask_id,
-                             float scale, const uint8_t* rowmask, int rows, int chunks, float4* part, cudaStream_t st) {
+                             float scale, const uint8_t* rowmask, int rows, int chunks, float4* part, cudaStream_t st,
+                             SampleArgs sa) {
     dim3 grid(chunks, rows);
     launch_pdl(entropy_partial_kernel, grid, dim3(256), 0, st, logits, splits, sstride, ld, V, mask_id, scale, rowmask,
-               chunks, part);
+               chunks, part, sa);
 }
 
-void launch_select_commit(const float4* part, int chunks, SlotState ss, RowState rs, int n_entries, int stride,
-                          StepKnobs kn, int* err, cudaStream_t st) {
-    launch_pdl(select_commit_kernel, dim3(n_entries), dim3(64), 0, st, part, chunks, ss, rs, stride, kn, err);
+void launch_select_commit(const float4* part, const float2* spart, int chunks, SlotState ss, RowState rs,
+                          int n_entries, int stride, StepKnobs kn, int* err, cudaStream_t st) {
+    launch_pdl(select_commit_kernel, dim3(n_entries), dim3(64), 0, st, part, spart, chunks, ss, rs, stride, kn, err);
 }
 
 void launch_reorder_only(const uint8_t* filled, const int32_t* n, const int32_t* S, int n_seq, int stride,
@@ -773,7 +854,7 @@ void launch_rowmask_from_filled(const uint8_t* filled, const int32_t* n, int n_s
 // Explicit instantiations.
 #define WEDLM_INST(T)                                                                                             \
     template void launch_decode_prepare<T>(const T*, const float*, float, int, int, SlotState, RowState, uint8_t*, \
-                                           int, int, float*, T*, cudaStream_t);                                   \
+                                           int, int, float*, T*, int, cudaStream_t);                              \
     template void launch_prefill_prepare<T>(const T*, const float*, float, int, const int32_t*, int, int, int,     \
                                             SlotState, RowState, float*, T*, cudaStream_t);                       \
     template void launch_qkv_rope<T>(const float*, int, int64_t, int, int, int, int, T*, T*, KVLayout, int,        \

@@ -10,13 +10,16 @@ namespace wedlm {
 struct StepKnobs {
     float lambda, tau, logit_scale;
     int tau_none;
+    int blockwise;           // commit only whole windows (block-wise baseline)
+    float temperature;       // > 0: Gumbel-max sampling of fill tokens
+    unsigned long long seed;
 };
 
 // Window prepare for a decode step: refill, reorder, embed, first RMSNorm.
 template <typename T>
 void launch_decode_prepare(const T* embed, const float* norm_g, float eps, int d, int mask_id,
                            SlotState ss, RowState rs, uint8_t* rowmask, int n_entries, int stride,
-                           float* x, T* h, cudaStream_t st);
+                           float* x, T* h, int blockwise, cudaStream_t st);
 // Prefill rows: tokens from `ids` (device), logical positions S0 + r.
 template <typename T>
 void launch_prefill_prepare(const T* embed, const float* norm_g, float eps, int d, const int32_t* ids,
@@ -51,12 +54,26 @@ void launch_swiglu(const float* ws, int splits, int64_t split_stride, int M, int
 void launch_rope_table(float2* cs, int max_pos, int half, int hd, double theta, cudaStream_t st);
 
 // Entropy / argmax partials over vocabulary chunks for rows with rowmask[row] != 0.
+// Sampled fills: inv_t = 1 / temperature (0 = greedy, nothing sampled); row r
+// belongs to slot r / stride, at logical position pos[r]; steps = the per-slot
+// counters block (its first field counts the slot's decode steps); part gets
+// one (best key, token) pair per (row, chunk).
+struct SampleArgs {
+    float inv_t = 0.f;
+    unsigned long long seed = 0;
+    int stride = 1;
+    const int32_t* pos = nullptr;
+    const int64_t* steps = nullptr;
+    float2* part = nullptr;
+};
+
 void launch_entropy_partials(const float* logits, int splits, int64_t split_stride, int64_t ld, int V,
                              int mask_id, float scale, const uint8_t* rowmask, int rows, int chunks,
-                             float4* part, cudaStream_t st);
+                             float4* part, cudaStream_t st, SampleArgs sa = SampleArgs());
 
-void launch_select_commit(const float4* part, int chunks, SlotState ss, RowState rs, int n_entries,
-                          int stride, StepKnobs knobs, int* err, cudaStream_t st);
+// spart: the sampling partials (read only when knobs.temperature > 0).
+void launch_select_commit(const float4* part, const float2* spart, int chunks, SlotState ss, RowState rs,
+                          int n_entries, int stride, StepKnobs knobs, int* err, cudaStream_t st);
 
 void launch_reorder_only(const uint8_t* filled, const int32_t* n, const int32_t* S, int n_seq, int stride,
                          int32_t* perm, int32_t* pos, int32_t* k, int32_t* nf, cudaStream_t st);
@@ -72,13 +89,20 @@ void launch_rowmask_from_filled(const uint8_t* filled, const int32_t* n, int n_s
 // Tensor map over the whole KV pool viewed as [rows][128] bf16, 16-row boxes
 // of 64 dims with the 128-byte swizzle (one box = one page, one half).
 bool make_kv_tmap(CUtensorMap* tm, const bf16* kv_pool, const KVLayout& kvl, int n_layers);
+// Tensor map over q [rows][hq][128] with boxes of 64 dims x g heads x the
+// attention's rows per tile (dual: the tile of windows with <= 64 query rows).
+bool make_q_tmap(CUtensorMap* tm, const bf16* q, int rows, int hq, int hkv, bool dual);
 // Decode/prefill attention.  With more than one key chunk per row tile
 // (kv_chunk < keys), partials go to part_o / part_ml and the last chunk of
 // each (entry, KV head, tile) to finish merges them; `tickets` holds
-// entries * hkv * tiles ints that are zero between launches.
-void launch_attn_bf16(const CUtensorMap& tm_kv, const bf16* q, KVLayout kvl, int layer, int hq, int hkv, bf16* out,
-                      float* part_o, float2* part_ml, int* tickets, int n_entries, int stride, int kv_chunk,
-                      int max_splits, SlotState ss, RowMap rm, int* err, cudaStream_t st);
+// entries * hkv * tiles ints that are zero between launches; max_splits <=
+// attn_max_splits().
+void launch_attn_bf16(const CUtensorMap& tm_kv, const CUtensorMap& tm_q, const CUtensorMap& tm_q_dual, KVLayout kvl,
+                      int layer, int hq, int hkv, bf16* out, float* part_o, float2* part_ml, int* tickets,
+                      int n_entries, int stride, int kv_chunk, int max_splits, SlotState ss, RowMap rm, int* err,
+                      cudaStream_t st);
+int attn_max_splits();
+int attn_dual_rows_per_tile(int group);
 int attn_rows_per_tile(int group);
 
 }  // namespace wedlm

@@ -119,22 +119,27 @@ struct wedlm_ctx {
     cudaGraphExec_t graph_exec = nullptr;
     int64_t graph_launches = 0;
     struct StepKey {
-        int n_entries = -1, stride = -1, tau_none = 0;
-        float lambda = 0.f, tau = 0.f, scale = 0.f;
+        int n_entries = -1, stride = -1, tau_none = 0, blockwise = 0;
+        float lambda = 0.f, tau = 0.f, scale = 0.f, temperature = 0.f;
+        uint64_t seed = 0;
         bool operator==(const StepKey& o) const {
             return n_entries == o.n_entries && stride == o.stride && tau_none == o.tau_none &&
-                   lambda == o.lambda && tau == o.tau && scale == o.scale;
+                   blockwise == o.blockwise && lambda == o.lambda && tau == o.tau && scale == o.scale &&
+                   temperature == o.temperature && seed == o.seed;
         }
     };
     StepKey graph_key, eager_key;
     float* logits = nullptr;
     size_t logits_floats = 0;
     float4* ent_part = nullptr;
+    float2* samp_part = nullptr;  // Gumbel-max partials of sampled fills
+    float* dbg_resid = nullptr;   // test hook: residual stream before each layer and after the last [L+1][Mdec][d]
     float* attn_po = nullptr;
     float2* attn_pml = nullptr;
     int* attn_tickets = nullptr;   // [maxB][hkv][tiles] merge tickets of the key-chunked attention
     size_t n_attn_tickets = 0;
     CUtensorMap tm_kv{};
+    CUtensorMap tm_q{}, tm_q_dual{};
     int attn_kv_chunk = 1 << 30, attn_max_splits = 1;
     int32_t* ids_dev = nullptr;
     // step results block for one device->host copy: counts[B], S[B], tokens[B][maxW], err
@@ -382,7 +387,15 @@ wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
 // holds the final-normed hidden states.
 
 // fp32 (exact-parity) mode: SIMT GEMMs, separate epilogue kernels.
-wedlm_status forward_f32(wedlm_ctx* ctx, int slot_base, int n_entries, int stride) {
+// Test hook: keep the residual stream entering layer `idx` (idx = L: after the
+// last layer) of a decode step.
+void capture_residual(wedlm_ctx* ctx, int idx, int M, bool decode) {
+    if (!ctx->dbg_resid || !decode) return;
+    cudaMemcpyAsync(ctx->dbg_resid + (size_t)idx * ctx->Mdec * ctx->d, ctx->x, (size_t)M * ctx->d * sizeof(float),
+                    cudaMemcpyDeviceToDevice, ctx->stream);
+}
+
+wedlm_status forward_f32(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
     const int M = n_entries * stride;
     RowMap rm{slot_base, stride, ctx->ss.n};
     const float eps = ctx->cfg.rms_eps;
@@ -391,6 +404,7 @@ wedlm_status forward_f32(wedlm_ctx* ctx, int slot_base, int n_entries, int strid
     float* ao = (float*)ctx->attn_out;
     float* act = (float*)ctx->act;
     wedlm_status s;
+    capture_residual(ctx, 0, M, decode);
     for (int l = 0; l < ctx->L; ++l) {
         if ((s = gemm_f32(ctx, WEDLM_PROF_GEMM_QKV, h, (const float*)ctx->wqkv[l], M, ctx->Nqkv, ctx->d))) return s;
         {
@@ -424,6 +438,7 @@ wedlm_status forward_f32(wedlm_ctx* ctx, int slot_base, int n_entries, int strid
             launch_residual_norm<float>(ctx->ws, 1, (int64_t)M * ctx->d, M, ctx->d, ctx->x, h, gnext, eps, rm,
                                         ctx->stream);
         }
+        capture_residual(ctx, l + 1, M, decode);
     }
     return WEDLM_OK;
 }
@@ -452,6 +467,7 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
     base.rope_cs = ctx->rope_cs;
     base.rope_max_pos = ctx->max_ctx;
     wedlm_status s;
+    capture_residual(ctx, 0, M, decode);
     for (int l = 0; l < ctx->L; ++l) {
         EpiParams e = base;
         e.layer = l;
@@ -462,8 +478,9 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
         const int ms = decode ? ctx->attn_max_splits : 1;
         {
             ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
-            launch_attn_bf16(ctx->tm_kv, qb, ctx->kvl, l, ctx->hq, ctx->hkv, ao, ctx->attn_po, ctx->attn_pml,
-                             ctx->attn_tickets, n_entries, stride, kc, ms, ctx->ss, rm, ctx->err, ctx->stream);
+            launch_attn_bf16(ctx->tm_kv, ctx->tm_q, ctx->tm_q_dual, ctx->kvl, l, ctx->hq, ctx->hkv, ao,
+                             ctx->attn_po, ctx->attn_pml, ctx->attn_tickets, n_entries, stride, kc, ms, ctx->ss, rm,
+                             ctx->err, ctx->stream);
         }
         e.kind = EPI_RESIDUAL;
         e.out = ctx->x;
@@ -478,6 +495,7 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
         e.kind = EPI_RESIDUAL;
         e.out = ctx->x;
         if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_DOWN, act, &ctx->tm_d[l], M, ctx->d, ctx->F, e, decode))) return s;
+        capture_residual(ctx, l + 1, M, decode);
         const float* gnext = (l + 1 < ctx->L) ? ctx->attn_norm[l + 1] : ctx->final_norm;
         {
             ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
@@ -489,7 +507,7 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
 
 wedlm_status run_forward(wedlm_ctx* ctx, int slot_base, int n_entries, int stride, bool decode) {
     return ctx->bf16 ? forward_bf16(ctx, slot_base, n_entries, stride, decode)
-                     : forward_f32(ctx, slot_base, n_entries, stride);
+                     : forward_f32(ctx, slot_base, n_entries, stride, decode);
 }
 
 int max_active_window(const wedlm_ctx* c, int* n_entries) {
@@ -511,11 +529,11 @@ wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, 
         if (ctx->bf16)
             launch_decode_prepare<bf16>((const bf16*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
                                         ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
-                                        (bf16*)ctx->h, ctx->stream);
+                                        (bf16*)ctx->h, prm->blockwise, ctx->stream);
         else
             launch_decode_prepare<float>((const float*)ctx->embed, ctx->attn_norm[0], ctx->cfg.rms_eps, ctx->d,
                                          ctx->cfg.mask_id, ctx->ss, ctx->rs, ctx->rowmask, n_entries, stride, ctx->x,
-                                         (float*)ctx->h, ctx->stream);
+                                         (float*)ctx->h, prm->blockwise, ctx->stream);
     }
     wedlm_status s = run_forward(ctx, 0, n_entries, stride, true);
     if (s) return s;
@@ -534,13 +552,23 @@ wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, 
     if (s) return s;
     {
         ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
+        SampleArgs sa;
+        if (prm->temperature > 0.f) {
+            sa.inv_t = 1.0f / prm->temperature;
+            sa.seed = prm->seed;
+            sa.stride = stride;
+            sa.pos = ctx->rs.pos;
+            sa.steps = ctx->ss.counters;
+            sa.part = ctx->samp_part;
+        }
         launch_entropy_partials(ctx->logits, lsp, (int64_t)M * ctx->V, ctx->V, ctx->V, ctx->cfg.mask_id,
-                                prm->logit_scale, ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream);
+                                prm->logit_scale, ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream, sa);
     }
-    StepKnobs kn{prm->lambda, prm->tau, prm->logit_scale, prm->tau_none};
+    StepKnobs kn{prm->lambda, prm->tau, prm->logit_scale, prm->tau_none, prm->blockwise, prm->temperature, prm->seed};
     {
         ProfScope ps(ctx, WEDLM_PROF_SELECT);
-        launch_select_commit(ctx->ent_part, kEntropyChunks, ctx->ss, ctx->rs, n_entries, stride, kn, ctx->err,
+        launch_select_commit(ctx->ent_part, ctx->samp_part, kEntropyChunks, ctx->ss, ctx->rs, n_entries, stride, kn,
+                             ctx->err,
                              ctx->stream);
     }
     ctx->last_stride = stride;
@@ -573,7 +601,10 @@ wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_en
     key.lambda = prm->lambda;
     key.tau = prm->tau;
     key.scale = prm->logit_scale;
-    const bool graphable = ctx->use_graphs && ctx->bf16 && ctx->stream != nullptr && !ctx->prof;
+    key.blockwise = prm->blockwise ? 1 : 0;
+    key.temperature = prm->temperature;
+    key.seed = prm->seed;
+    const bool graphable = ctx->use_graphs && ctx->bf16 && ctx->stream != nullptr && !ctx->prof && !ctx->dbg_resid;
     if (graphable && ctx->graph_exec && ctx->graph_key == key) {
         cudaError_t e = cudaGraphLaunch(ctx->graph_exec, ctx->stream);
         if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("graph launch: ") + cudaGetErrorString(e));
@@ -775,6 +806,9 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         const long long blocks = pairs * std::max(1, (ctx->max_ctx / 2 + 63) / 64);
         long long cb = (blocks + 2LL * ctx->num_sms - 1) / (2LL * ctx->num_sms);
         cb = std::max(1LL, std::min(cb, 32LL));
+        // at most attn_max_splits() chunks per row tile (the merge keeps its weights on chip)
+        const long long ms_cap = attn_max_splits();
+        cb = std::max(cb, ((long long)ctx->max_ctx + 64 * ms_cap - 1) / (64 * ms_cap));
         ctx->attn_kv_chunk = (int)(cb * 64);
         ctx->attn_max_splits = (ctx->max_ctx + ctx->attn_kv_chunk - 1) / ctx->attn_kv_chunk;
         ctx->n_attn_tickets = (size_t)pairs;
@@ -819,12 +853,16 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     ctx->logits_floats = (size_t)ctx->Mdec * (size_t)V;
     xa.add((void**)&ctx->logits, ctx->logits_floats * 4);
     xa.add((void**)&ctx->ent_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float4));
+    xa.add((void**)&ctx->samp_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float2));
     if (ctx->bf16 && ctx->attn_max_splits > 1) {
         const size_t pairs = (size_t)ctx->Mdec * ctx->hq * ctx->attn_max_splits;
         xa.add((void**)&ctx->attn_po, pairs * ctx->hd * 4);
         xa.add((void**)&ctx->attn_pml, pairs * sizeof(float2));
     }
     if (xa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+    if (ctx->bf16 && !(make_q_tmap(&ctx->tm_q, (const bf16*)ctx->q, Mmax, ctx->hq, ctx->hkv, false) &&
+                       make_q_tmap(&ctx->tm_q_dual, (const bf16*)ctx->q, Mmax, ctx->hq, ctx->hkv, true)))
+        return bail(WEDLM_ERR_CUDA);
 
     launch_rope_table(ctx->rope_cs, ctx->max_ctx, ctx->hd / 2, ctx->hd, cfg->rope_theta, ctx->stream);
     std::vector<int32_t> pt((size_t)B * ctx->pages_per_seq, -1);
@@ -849,6 +887,7 @@ void wedlm_destroy(wedlm_ctx* ctx) {
     ctx->weights_arena.release();
     ctx->state_arena.release();
     ctx->scratch_arena.release();
+    if (ctx->dbg_resid) cudaFree(ctx->dbg_resid);
     if (ctx->res_host) cudaFreeHost(ctx->res_host);
     for (cudaEvent_t e : ctx->ev_pool) cudaEventDestroy(e);
     drop_graph(ctx);
@@ -1024,6 +1063,8 @@ static wedlm_status check_params(wedlm_ctx* ctx, const wedlm_step_params* p) {
     if (!p) return fail(ctx, WEDLM_ERR_INVALID_ARG, "null params");
     if (!(p->logit_scale > 0.f) || !std::isfinite(p->logit_scale) || std::isnan(p->lambda) || std::isnan(p->tau))
         return fail(ctx, WEDLM_ERR_INVALID_ARG, "logit_scale must be finite and > 0; lambda, tau not NaN");
+    if (!(p->temperature >= 0.f) || !std::isfinite(p->temperature))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "temperature must be finite and >= 0");
     if (!ctx->weights_ready) return fail(ctx, WEDLM_ERR_STATE, "weights not fully loaded");
     return WEDLM_OK;
 }
@@ -1268,6 +1309,35 @@ wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t
                     (kv ? host_v : host_k)[((size_t)i * hkv + hh) * hd + c] = v;
                 }
     }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_capture(wedlm_ctx* ctx, int32_t enable) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(ctx->stream));
+    if (enable && !ctx->dbg_resid) {
+        const size_t bytes = (size_t)(ctx->L + 1) * ctx->Mdec * ctx->d * sizeof(float);
+        if (cudaMalloc((void**)&ctx->dbg_resid, bytes) != cudaSuccess) {
+            ctx->dbg_resid = nullptr;
+            return fail(ctx, WEDLM_ERR_OOM_DEVICE, "residual capture buffer");
+        }
+        CK(cudaMemset(ctx->dbg_resid, 0, bytes));
+        drop_graph(ctx);
+    } else if (!enable && ctx->dbg_resid) {
+        cudaFree(ctx->dbg_resid);
+        ctx->dbg_resid = nullptr;
+    }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_residual(wedlm_ctx* ctx, int32_t layer, float* host_dst, int32_t rows) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (!ctx->dbg_resid) return fail(ctx, WEDLM_ERR_STATE, "residual capture is off");
+    if (layer < 0 || layer > ctx->L || rows < 0 || rows > ctx->Mdec || !host_dst)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad arguments");
+    CK(cudaStreamSynchronize(ctx->stream));
+    CK(cudaMemcpy(host_dst, ctx->dbg_resid + (size_t)layer * ctx->Mdec * ctx->d, (size_t)rows * ctx->d * sizeof(float),
+                  cudaMemcpyDeviceToHost));
     return WEDLM_OK;
 }
 

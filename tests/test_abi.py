@@ -41,6 +41,7 @@ int main(void) {
          sizeof(wedlm_step_params), sizeof(wedlm_seq_stats));
   P(wedlm_model_cfg, rope_theta); P(wedlm_model_cfg, rms_eps); P(wedlm_model_cfg, dtype);
   P(wedlm_model_cfg, prefill_chunk); P(wedlm_step_params, tau_none); P(wedlm_step_params, logit_scale);
+  P(wedlm_step_params, blockwise); P(wedlm_step_params, temperature); P(wedlm_step_params, seed);
   P(wedlm_seq_stats, committed_len); P(wedlm_seq_stats, active);
   return 0;
 }
@@ -61,6 +62,9 @@ def test_struct_layouts_match_c(tmp_path):
     assert int(c["wedlm_model_cfg.prefill_chunk"]) == ModelCfg.prefill_chunk.offset
     assert int(c["wedlm_step_params.tau_none"]) == StepParams.tau_none.offset
     assert int(c["wedlm_step_params.logit_scale"]) == StepParams.logit_scale.offset
+    assert int(c["wedlm_step_params.blockwise"]) == StepParams.blockwise.offset
+    assert int(c["wedlm_step_params.temperature"]) == StepParams.temperature.offset
+    assert int(c["wedlm_step_params.seed"]) == StepParams.seed.offset
     assert int(c["wedlm_seq_stats.committed_len"]) == SeqStats.committed_len.offset
     assert int(c["wedlm_seq_stats.active"]) == SeqStats.active.offset
 

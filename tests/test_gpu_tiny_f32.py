@@ -19,12 +19,12 @@ def model():
     return oracle_model(DIMS)
 
 
-def run_gpu_traced(eng, slot_prompts, N, W, lam, tau, tau_none, scale):
+def run_gpu_traced(eng, slot_prompts, N, W, lam, tau, tau_none, scale, blockwise=False, temperature=0.0, seed=0):
     """Decode to completion; per step record (k, n, perm, fills, H~) of each slot."""
     from streaming_decoding_b200 import step_params
     for b, p in slot_prompts.items():
         eng.prefill(b, p, N, W[b] if isinstance(W, dict) else W)
-    prm = step_params(lam, tau, tau_none, scale)
+    prm = step_params(lam, tau, tau_none, scale, blockwise=blockwise, temperature=temperature, seed=seed)
     traces = {b: [] for b in slot_prompts}
     out = {b: [] for b in slot_prompts}
     active = len(slot_prompts)
@@ -49,7 +49,8 @@ def run_gpu_traced(eng, slot_prompts, N, W, lam, tau, tau_none, scale):
     return out, traces
 
 
-def lockstep_oracle(model, prompt, N, W, lam, tau, tau_none, scale, gtrace):
+def lockstep_oracle(model, prompt, N, W, lam, tau, tau_none, scale, gtrace, blockwise=False, temperature=0.0,
+                    seed=0, slot=0):
     """Run the oracle alongside a recorded GPU trace.  Where the oracle's H~
     leave the decision open within MARGIN, the GPU's decision must be a valid
     one and the oracle then follows it; elsewhere decisions must be equal.
@@ -65,7 +66,8 @@ def lockstep_oracle(model, prompt, N, W, lam, tau, tau_none, scale, gtrace):
             near[0] += 1
         return g
 
-    st = O.stream_decode(model, prompt, N, W, lam, tau, tau_none=tau_none, logit_scale=scale, choose=choose)
+    st = O.stream_decode(model, prompt, N, W, lam, tau, tau_none=tau_none, logit_scale=scale, choose=choose,
+                         blockwise=blockwise, temperature=temperature, seed=seed, slot=slot)
     return st, near[0]
 
 
@@ -97,6 +99,47 @@ def test_token_stream_and_decisions_match_oracle(model, cfg_name):
     s = eng.stats(0)
     assert (s["steps"], s["forward_rows"], s["committed"], s["active"]) == (st.steps, st.rows, len(st.out), 0)
     assert s["fills"] == st.n_fills
+
+
+@pytest.mark.parametrize("cfg_name", ["tiny_f32", "tiny_f32_tau"])
+def test_blockwise_baseline_matches_oracle(model, cfg_name):
+    """The block-wise (stop-and-wait) baseline on the same kernels: every step's
+    commit run (whole window or nothing), order, H~ and fills equal the oracle's."""
+    cfg = synth.CONFIGS[cfg_name]
+    prompt = synth.prompts(cfg)[0]
+    eng = make_engine(DIMS, max_batch=1, max_window=cfg["W"], max_ctx=64)
+    out, tr = run_gpu_traced(eng, {0: prompt}, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"], False,
+                             cfg["logit_scale"], blockwise=True)
+    st, near = lockstep_oracle(model, prompt, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"], False,
+                               cfg["logit_scale"], tr[0], blockwise=True)
+    compare_traces(st, tr[0])
+    assert near <= 2
+    assert all(t["k"] in (0, t["n"]) for t in tr[0])
+    assert out[0] == st.out
+    s = eng.stats(0)
+    assert (s["steps"], s["forward_rows"], s["committed"]) == (st.steps, st.rows, len(st.out))
+
+
+@pytest.mark.parametrize("temperature", [0.1, 1.0])
+def test_sampled_fills_match_oracle(model, temperature):
+    """Seeded Gumbel-max sampling of fill tokens (two slots, so the slot is part
+    of the generator's key): token streams and decisions equal the oracle's."""
+    cfg = synth.CONFIGS["tiny_f32_tau"]
+    prompts = synth.prompts(cfg)
+    slot_prompts = {0: prompts[0], 1: prompts[0][::-1].copy()}
+    eng = make_engine(DIMS, max_batch=2, max_window=cfg["W"], max_ctx=64)
+    out, tr = run_gpu_traced(eng, slot_prompts, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"], False,
+                             cfg["logit_scale"], temperature=temperature, seed=20251202)
+    greedy = O.stream_decode(model, prompts[0], cfg["N"], cfg["W"], cfg["lam"], cfg["tau"],
+                             logit_scale=cfg["logit_scale"]).out
+    for b, p in slot_prompts.items():
+        st, near = lockstep_oracle(model, p, cfg["N"], cfg["W"], cfg["lam"], cfg["tau"], False, cfg["logit_scale"],
+                                   tr[b], temperature=temperature, seed=20251202, slot=b)
+        compare_traces(st, tr[b])
+        assert near <= 2
+        assert out[b] == st.out
+    if temperature >= 1.0:
+        assert out[0] != greedy  # sampling at T = 1 departs from the greedy stream
 
 
 def test_window_one_is_greedy_autoregression(model):

@@ -513,3 +513,37 @@ def test_act_round_hook_applies_only_at_the_contract_points():
     ze, zb = O.lm_logits(exact, he, 1.0), O.lm_logits(bf, hb, 1.0)
     rel = np.abs(zb - ze).max() / np.abs(ze).max()
     assert 0 < rel < 2e-2, rel
+
+
+# ---------------------------------------------------- sampled fills (R20) ---
+def test_mix64_reproduces_published_splitmix64_outputs():
+    """The SplitMix64 generator seeded with 0 outputs 0xE220A8397B1DCDAF, then
+    0x6E789E6AA1B965F4 (its state advances by the golden gamma per draw)."""
+    assert int(O.mix64(np.uint64(0))) == 0xE220A8397B1DCDAF
+    assert int(O.mix64(np.uint64(0x9E3779B97F4A7C15))) == 0x6E789E6AA1B965F4
+
+
+def test_sampling_uniforms_are_open_interval_and_key_sensitive():
+    u = O.sampling_uniforms(7, 3, 11, 1234, 5000)
+    assert u.min() > 0.0 and u.max() < 1.0 and len(np.unique(u)) > 4990
+    assert abs(u.mean() - 0.5) < 0.02
+    for other in (O.sampling_uniforms(8, 3, 11, 1234, 5000), O.sampling_uniforms(7, 4, 11, 1234, 5000),
+                  O.sampling_uniforms(7, 3, 12, 1234, 5000), O.sampling_uniforms(7, 3, 11, 1235, 5000)):
+        assert np.mean(other == u) < 0.01
+
+
+def test_gumbel_max_draws_follow_the_tempered_softmax():
+    """Frequencies of the sampled token over many keys match softmax(z / T)
+    (mask id excluded) within 4 standard errors; T -> 0 gives the argmax."""
+    z = np.array([1.0, 0.2, -0.5, 1.3, 0.0, 9.0])
+    mask_id, T, n = 5, 0.7, 20000
+    counts = np.zeros(len(z))
+    for i in range(n):
+        counts[O.sample_token(z, mask_id, 1.0, T, O.sampling_uniforms(1, 0, 0, i, len(z)))] += 1
+    p = np.exp(np.where(np.arange(len(z)) == mask_id, -np.inf, z / T))
+    p /= p.sum()
+    assert counts[mask_id] == 0
+    se = np.sqrt(p * (1 - p) / n)
+    assert np.all(np.abs(counts / n - p) <= 4 * se + 1e-12), (counts / n, p)
+    u = O.sampling_uniforms(1, 0, 0, 0, len(z))
+    assert O.sample_token(z, mask_id, 1.0, 1e-6, u) == 3
