@@ -35,14 +35,16 @@ namespace wedlm {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 64;
-constexpr int SUB_A_BYTES = BM * BK * 2;  // one 128-row weight sub-tile of a stage
+constexpr int BK_DEFAULT = 64;  // k-block depth of the 128-byte-swizzle tiles
 
 // BN activation rows (MMA N) by WT weight sub-tiles of 128 rows (one MMA each
 // per k-step, sharing the activation operand: WT = 2 halves the activation
 // bytes a CTA moves per output).  NACC accumulators of WT*BN TMEM columns
 // (two when they fit, so a unit's MMAs overlap the previous unit's epilogue).
-template <int BN, int WT> struct PCfg {
+// BK = 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte
+// swizzle: half the bytes per stage, so twice the stages in flight).
+template <int BN, int WT, int BK> struct PCfg {
+    static constexpr int SUB_A_BYTES = BM * BK * 2;  // one 128-row weight sub-tile of a stage
     static constexpr int A_STAGE_BYTES = WT * SUB_A_BYTES;
     static constexpr int B_STAGE_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
@@ -90,15 +92,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, in
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Shared-memory matrix descriptor of a K-major tile stored with the 128-byte
-// swizzle (rows of 64 bf16 = 128 B; 8-row swizzle atoms 1024 B apart).
-__device__ __forceinline__ uint64_t sdesc_k_sw128(const void* p) {
+// Shared-memory matrix descriptor of a K-major tile of BK-element rows stored
+// with the matching swizzle: BK = 64 -> 128-byte rows, 128-byte swizzle, 8-row
+// atoms 1024 B apart; BK = 32 -> 64-byte rows, 64-byte swizzle, atoms 512 B apart.
+template <int BK>
+__device__ __forceinline__ uint64_t sdesc_k(const void* p) {
+    static_assert(BK == 64 || BK == 32, "k-block depth");
     const uint32_t a = smem_u32(p);
     uint64_t d = (uint64_t)((a >> 4) & 0x3FFFu);
-    d |= (uint64_t)1 << 16;               // leading-dimension byte offset (unused with swizzle)
-    d |= (uint64_t)(1024 >> 4) << 32;     // stride byte offset between 8-row atoms
-    d |= (uint64_t)1 << 46;               // descriptor version for tcgen05
-    d |= (uint64_t)2 << 61;               // 128-byte swizzle
+    d |= (uint64_t)1 << 16;                      // leading-dimension byte offset (unused with swizzle)
+    d |= (uint64_t)((8 * BK * 2) >> 4) << 32;    // stride byte offset between 8-row atoms
+    d |= (uint64_t)1 << 46;                      // descriptor version for tcgen05
+    d |= (uint64_t)(BK == 64 ? 2 : 4) << 61;     // 128-byte or 64-byte swizzle
     return d;
 }
 
@@ -330,10 +335,11 @@ __device__ __forceinline__ void epilogue_vec4x8(const EpiParams& ep, int n0, int
     }
 }
 
-template <int BN, int WT>
+template <int BN, int WT, int BK>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
                                                          const __grid_constant__ CUtensorMap tmX, const GemmArgs g) {
-    using C = PCfg<BN, WT>;
+    using C = PCfg<BN, WT, BK>;
+    constexpr int SUB_A_BYTES = C::SUB_A_BYTES;
     constexpr int NACC = C::NACC;
     constexpr int TW = BM * WT;  // weight rows per tile
     constexpr int STAGES = C::STAGES;
@@ -457,8 +463,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     for (int kk = 0; kk < BK / 16; ++kk)
 #pragma unroll
                         for (int w = 0; w < WT; ++w)
-                            umma_bf16(d + w * BN, sdesc_k_sw128(a + w * SUB_A_BYTES + kk * 32),
-                                      sdesc_k_sw128(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                            umma_bf16(d + w * BN, sdesc_k<BK>(a + w * SUB_A_BYTES + kk * 32),
+                                      sdesc_k<BK>(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 umma_commit(&accf[b]);
@@ -614,19 +620,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-template <int BN, int WT>
+template <int BN, int WT, int BK>
 cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, int grid, cudaStream_t st) {
-    using C = PCfg<BN, WT>;
+    using C = PCfg<BN, WT, BK>;
     static int attr_dev = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
         cudaError_t e =
-            cudaFuncSetAttribute(gemm_tc_kernel<BN, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            cudaFuncSetAttribute(gemm_tc_kernel<BN, WT, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
-    if (a.splits == 1) return launch_pdl(gemm_tc_kernel<BN, WT>, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
+    if (a.splits == 1) return launch_pdl(gemm_tc_kernel<BN, WT, BK>, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
     // CTAs of a split tile wait for one another: launch cooperatively so all of
     // them are resident at once (the launch fails instead of deadlocking).
     cudaLaunchConfig_t cfg = {};
@@ -639,7 +645,7 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, WT>, tmW, tmX, a);
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, WT, BK>, tmW, tmX, a);
 }
 
 }  // namespace
@@ -647,13 +653,14 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
 namespace {
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
-GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1) {
+GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1, int bk = BK_DEFAULT) {
     GemmPlan p;
     p.bn = bn;
     p.wt = wt;
+    p.bk = bk;
     p.m_tiles = (M + bn - 1) / bn;
     p.n_tiles = (N + BM * wt - 1) / (BM * wt);
-    const int KB = (K + BK - 1) / BK;
+    const int KB = (K + bk - 1) / bk;
     p.kb_per_split = (KB + splits - 1) / splits;
     p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;
     // Units are dealt in rounds of `grid`; a multiple of the split count keeps
@@ -666,14 +673,16 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
 }  // namespace
 
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                        int force_wt) {
-    const int KB = (K + BK - 1) / BK;
+                        int force_wt, int force_bk) {
+    const int KB = (K + BK_DEFAULT - 1) / BK_DEFAULT;
     // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
     const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
     if (force_bn > 0 || force_splits > 0) {
         const int bn = force_bn > 0 ? force_bn : bn_for(M);
         const int wt = (force_wt == 2 && bn >= 128) ? 2 : 1;
-        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)), wt);
+        const int bk = (force_bk == 32 && bn >= 128) ? 32 : BK_DEFAULT;
+        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)), wt,
+                         bk);
     }
     // Cost in units of one 256-column k-block per CTA: rounds x k-block time x
     // (k-blocks per unit + per-unit overhead + the partial plane's round trip
@@ -713,16 +722,16 @@ bool encode_tmap_bf16(CUtensorMap* tm, const void* base, int rank, const cuuint6
     return r == CUDA_SUCCESS;
 }
 
-bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, int bk) {
     auto fn = encode_fn();
-    if (!fn) return false;
+    if (!fn || (bk != 64 && bk != 32)) return false;
     cuuint64_t gdim[2] = {cols, rows};
     cuuint64_t gstride[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)bk, box_rows};
     cuuint32_t estride[2] = {1, 1};
     CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, bk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -730,19 +739,25 @@ cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int
                              const EpiParams& ep, cudaStream_t st) {
     if (p.splits > 1 && (!ep.ws || !ep.counters)) return cudaErrorInvalidValue;
     GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, ep};
+    if (p.bk == 32) {
+        if (p.wt == 2 && p.bn == 256) return launch_bn<256, 2, 32>(tmW, tmX, a, p.grid, st);
+        if (p.wt == 2 && p.bn == 128) return launch_bn<128, 2, 32>(tmW, tmX, a, p.grid, st);
+        if (p.wt == 1 && p.bn == 256) return launch_bn<256, 1, 32>(tmW, tmX, a, p.grid, st);
+        return cudaErrorInvalidValue;
+    }
     if (p.wt == 2) {
         switch (p.bn) {
-            case 128: return launch_bn<128, 2>(tmW, tmX, a, p.grid, st);
-            case 256: return launch_bn<256, 2>(tmW, tmX, a, p.grid, st);
+            case 128: return launch_bn<128, 2, 64>(tmW, tmX, a, p.grid, st);
+            case 256: return launch_bn<256, 2, 64>(tmW, tmX, a, p.grid, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (p.bn) {
-        case 16: return launch_bn<16, 1>(tmW, tmX, a, p.grid, st);
-        case 32: return launch_bn<32, 1>(tmW, tmX, a, p.grid, st);
-        case 64: return launch_bn<64, 1>(tmW, tmX, a, p.grid, st);
-        case 128: return launch_bn<128, 1>(tmW, tmX, a, p.grid, st);
-        case 256: return launch_bn<256, 1>(tmW, tmX, a, p.grid, st);
+        case 16: return launch_bn<16, 1, 64>(tmW, tmX, a, p.grid, st);
+        case 32: return launch_bn<32, 1, 64>(tmW, tmX, a, p.grid, st);
+        case 64: return launch_bn<64, 1, 64>(tmW, tmX, a, p.grid, st);
+        case 128: return launch_bn<128, 1, 64>(tmW, tmX, a, p.grid, st);
+        case 256: return launch_bn<256, 1, 64>(tmW, tmX, a, p.grid, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -42,6 +42,7 @@ struct EpiParams {
 struct GemmPlan {
     int bn = 16;
     int wt = 1;
+    int bk = 64;       // k-block depth: 64 (128-byte swizzle) or 32 (64-byte swizzle, bn >= 128)
     int splits = 1;
     int kb_per_split = 1;
     int m_tiles = 1;
@@ -53,15 +54,18 @@ struct GemmPlan {
 // force_bn / force_splits > 0 pin the tile width / split count, force_wt = 2
 // selects 256-row weight tiles (tuning hooks).
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0,
-                        int force_wt = 0);
+                        int force_wt = 0, int force_bk = 0);
 
-bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// 2-D bf16 tensor map [rows][cols], boxes of bk columns (64: 128-byte swizzle,
+// 32: 64-byte swizzle) by box_rows rows.
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, int bk = 64);
 // Any-rank bf16 tensor map with the 128-byte swizzle (box[0] * 2 bytes must be
 // 128); gstride[i] is the byte stride of dimension i + 1.
 bool encode_tmap_bf16(CUtensorMap* tm, const void* base, int rank, const cuuint64_t* gdim, const cuuint64_t* gstride,
                       const cuuint32_t* box);
 
-// tmW: weights [N][K], box rows 128; tmX: activations [>=M][K], box rows plan.bn.
+// tmW: weights [N][K], box rows 128; tmX: activations [>=M][K], box rows plan.bn;
+// both with boxes of plan.bk columns.
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K,
                              const GemmPlan& plan, const EpiParams& ep, cudaStream_t st);
 

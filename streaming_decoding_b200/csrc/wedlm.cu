@@ -85,8 +85,13 @@ struct wedlm_ctx {
     std::vector<uint8_t> loaded;  // per tensor slot
     bool weights_ready = false;
     // bf16 tensor maps of the weights (box 128 rows)
-    std::vector<CUtensorMap> tm_qkv, tm_o, tm_gu, tm_d;
-    CUtensorMap tm_lm{};
+    // Weight tensor maps for both k-block depths (64: 128-byte swizzle, 32: 64-byte).
+    struct WMap {
+        CUtensorMap k64{}, k32{};
+        const CUtensorMap& of(int bk) const { return bk == 32 ? k32 : k64; }
+    };
+    std::vector<WMap> tm_qkv, tm_o, tm_gu, tm_d;
+    WMap tm_lm{};
     bool maps_ready = false;
     // KV pool
     void* kv_pool = nullptr;
@@ -150,6 +155,7 @@ struct wedlm_ctx {
         const void* p;
         uint64_t rows, cols;
         uint32_t box;
+        int bk;
         CUtensorMap tm;
     };
     std::deque<XMap> xmaps;
@@ -232,11 +238,11 @@ int tensor_slot(const wedlm_ctx* c, int tensor, int layer) {
     return 3 + layer * 9 + (tensor - WEDLM_T_ATTN_NORM);
 }
 
-const CUtensorMap* xmap(wedlm_ctx* c, const void* p, uint64_t rows, uint64_t cols, uint32_t box) {
+const CUtensorMap* xmap(wedlm_ctx* c, const void* p, uint64_t rows, uint64_t cols, uint32_t box, int bk) {
     for (auto& m : c->xmaps)
-        if (m.p == p && m.rows == rows && m.cols == cols && m.box == box) return &m.tm;
-    wedlm_ctx::XMap m{p, rows, cols, box, {}};
-    if (!make_tmap_bf16(&m.tm, p, rows, cols, box)) return nullptr;
+        if (m.p == p && m.rows == rows && m.cols == cols && m.box == box && m.bk == bk) return &m.tm;
+    wedlm_ctx::XMap m{p, rows, cols, box, bk, {}};
+    if (!make_tmap_bf16(&m.tm, p, rows, cols, box, bk)) return nullptr;
     c->xmaps.push_back(m);
     return &c->xmaps.back().tm;
 }
@@ -255,7 +261,7 @@ wedlm_status gemm_f32(wedlm_ctx* ctx, int kind, const float* X, const float* W, 
 // launch that follows rewrites anyway (the q / activation scratch, and K/V
 // at the window's own cache positions).  Runs once per (kind, M) on the
 // context's stream; candidates that do not fit the scratch buffers are skipped.
-void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* tmW, int M, int N, int K,
+void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WMap* tmW, int M, int N, int K,
                     const EpiParams& ep_real) {
     const std::pair<int, int> key(kind, M);
     if (ctx->tuned.count(key)) return;
@@ -265,11 +271,15 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* 
         if ((size_t)M * N > ctx->logits_floats) return;
         ep.out = ctx->logits;
     }
-    // (activation rows per tile, 128-row weight sub-tiles per tile)
-    std::vector<std::pair<int, int>> shapes;
-    if (M > 128) shapes = {{256, 1}, {128, 1}, {256, 2}, {128, 2}};
-    else if (M > 64) shapes = {{128, 1}, {64, 1}, {128, 2}};
-    else shapes = {{M <= 16 ? 16 : M <= 32 ? 32 : 64, 1}};
+    // (activation rows per tile, 128-row weight sub-tiles per tile, k-block depth)
+    struct Shape {
+        int bn, wt, bk;
+    };
+    std::vector<Shape> shapes;
+    if (M > 128)
+        shapes = {{256, 1, 64}, {128, 1, 64}, {256, 2, 64}, {128, 2, 64}, {256, 2, 32}, {128, 2, 32}, {256, 1, 32}};
+    else if (M > 64) shapes = {{128, 1, 64}, {64, 1, 64}, {128, 2, 64}, {128, 2, 32}};
+    else shapes = {{M <= 16 ? 16 : M <= 32 ? 32 : 64, 1, 64}};
     cudaEvent_t e0 = prof_event(ctx), e1 = prof_event(ctx);
     float best = 1e30f;
     GemmPlan bestp = ctx->tuned[key].plan;
@@ -277,20 +287,20 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* 
     ep.counters = ctx->tile_counters;
     ep.err = ctx->err;
     const int KB = (K + 63) / 64;
-    for (auto [bn, wt] : shapes) {
+    for (const Shape& sh : shapes) {
         for (int sp : {1, 2, 3, 4, 6, 8, 12, 16}) {
             if (sp > KB || (sp > 1 && N % 4)) continue;
-            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, bn, sp, wt);
+            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, sh.bn, sp, sh.wt, sh.bk);
             if (p.splits != sp) continue;
             if (p.splits > 1 && ((size_t)p.splits * M * N > ctx->ws_floats ||
                                  (size_t)p.m_tiles * p.n_tiles > ctx->n_tile_counters))
                 continue;
-            const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
+            const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn, p.bk);
             if (!tx) continue;
             float t = 1e30f;
             for (int rep = 0; rep < 4; ++rep) {
                 cudaEventRecord(e0, ctx->stream);
-                if (launch_gemm_bf16(*tmW, *tx, M, N, K, p, ep, ctx->stream) != cudaSuccess) {
+                if (launch_gemm_bf16(tmW->of(p.bk), *tx, M, N, K, p, ep, ctx->stream) != cudaSuccess) {
                     cudaGetLastError();
                     t = 1e30f;
                     break;
@@ -313,7 +323,7 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* 
 }
 
 // bf16 mode: the persistent tcgen05 GEMM with its epilogue fused (gemm_tc.cuh).
-wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMap* tmW, int M, int N, int K,
+wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WMap* tmW, int M, int N, int K,
                        EpiParams ep, bool tune = true) {
     GemmPlan p;
     if (ctx->autotune && tune) {
@@ -326,8 +336,8 @@ wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMa
     }
     if (p.splits > 1 && ((size_t)p.n_tiles * p.m_tiles > ctx->n_tile_counters ||
                          (size_t)p.splits * M * N > ctx->ws_floats))
-        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1);
-    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn);
+        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk);
+    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn, p.bk);
     if (!tx) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for activations");
     ep.ws = ctx->ws;
     ep.counters = ctx->tile_counters;
@@ -335,7 +345,7 @@ wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const CUtensorMa
     cudaError_t e;
     {
         ProfScope ps(ctx, kind);
-        e = launch_gemm_bf16(*tmW, *tx, M, N, K, p, ep, ctx->stream);
+        e = launch_gemm_bf16(tmW->of(p.bk), *tx, M, N, K, p, ep, ctx->stream);
     }
     if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("gemm launch: ") + cudaGetErrorString(e));
     return WEDLM_OK;
@@ -359,12 +369,16 @@ wedlm_status build_weight_maps(wedlm_ctx* ctx) {
     ctx->tm_d.resize(ctx->L);
     bool ok = true;
     for (int l = 0; l < ctx->L; ++l) {
-        ok &= make_tmap_bf16(&ctx->tm_qkv[l], ctx->wqkv[l], ctx->Nqkv, ctx->d, 128);
-        ok &= make_tmap_bf16(&ctx->tm_o[l], ctx->wo[l], ctx->d, (uint64_t)ctx->hq * ctx->hd, 128);
-        ok &= make_tmap_bf16(&ctx->tm_gu[l], ctx->wgu[l], 2 * (uint64_t)ctx->F, ctx->d, 128);
-        ok &= make_tmap_bf16(&ctx->tm_d[l], ctx->wd[l], ctx->d, ctx->F, 128);
+        for (int bk : {64, 32}) {
+            auto pick = [&](wedlm_ctx::WMap& m) { return bk == 32 ? &m.k32 : &m.k64; };
+            ok &= make_tmap_bf16(pick(ctx->tm_qkv[l]), ctx->wqkv[l], ctx->Nqkv, ctx->d, 128, bk);
+            ok &= make_tmap_bf16(pick(ctx->tm_o[l]), ctx->wo[l], ctx->d, (uint64_t)ctx->hq * ctx->hd, 128, bk);
+            ok &= make_tmap_bf16(pick(ctx->tm_gu[l]), ctx->wgu[l], 2 * (uint64_t)ctx->F, ctx->d, 128, bk);
+            ok &= make_tmap_bf16(pick(ctx->tm_d[l]), ctx->wd[l], ctx->d, ctx->F, 128, bk);
+        }
     }
-    ok &= make_tmap_bf16(&ctx->tm_lm, ctx->lm_head, ctx->V, ctx->d, 128);
+    ok &= make_tmap_bf16(&ctx->tm_lm.k64, ctx->lm_head, ctx->V, ctx->d, 128, 64);
+    ok &= make_tmap_bf16(&ctx->tm_lm.k32, ctx->lm_head, ctx->V, ctx->d, 128, 32);
     if (!ok) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for weights");
     ctx->maps_ready = true;
     return WEDLM_OK;
