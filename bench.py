@@ -253,7 +253,7 @@ def roofline(prof, dims, M, pk, workload):
     t_hbm = bytes_tot / (pk["hbm"] * 1e9)
     t_tc = flops_tot / (pk["tc_sus"] * 1e12)
     sec = ms_tot / 1e3
-    traffic = measured_traffic("gemm_bf16_tc", workload)
+    traffic = measured_traffic("gemm_tc", workload)
     if t_hbm >= t_tc:
         ach = bytes_tot / sec / 1e9
         out = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
@@ -262,7 +262,7 @@ def roofline(prof, dims, M, pk, workload):
         ach = flops_tot / sec / 1e12
         out = {"bound": "tensor", "achieved": round(ach, 1), "peak": pk["tc_sus"], "unit": "TFLOP/s",
                "frac": round(ach / pk["tc_sus"], 4)}
-    out.update({"traffic": traffic, "kernel": "gemm_bf16_tc_kernel (all projections and LM head)",
+    out.update({"traffic": traffic, "kernel": "gemm_tc_kernel (all projections and LM head)",
                 "launches_profiled": launches, "avg_launch_us": round(ms_tot * 1e3 / max(1, launches), 2),
                 "algorithmic_bytes_per_launch": round(bytes_tot / max(1, launches)),
                 "peak_source": f"{pk['src']} ({'hbm_gbs' if out['bound'] == 'hbm' else 'bf16_tflops_sustained'})"})

@@ -9,19 +9,21 @@
 //
 // One CTA per SM loops over work units (tile, K slice).  Warp roles (192
 // threads):
-//   warp 0      one thread issues TMA loads of A (weights, 128 x 64) and B
-//               (activations, bn x 64) into a STAGES-deep shared-memory ring
+//   warp 0      one thread issues TMA loads of A (weights, 128*wt x bk) and B
+//               (activations, bn x bk) into a STAGES-deep shared-memory ring
 //               that runs continuously across units,
-//   warp 1      allocates TMEM (two bn-column accumulators) and one thread
-//               issues tcgen05.mma (kind::f16, fp32 accumulation), releasing
-//               ring stages with tcgen05.commit; it alternates accumulators so
-//               the next unit's MMAs overlap the previous unit's epilogue,
+//   warp 1      allocates TMEM (accumulators of wt*bn columns, two when they
+//               fit) and one thread issues tcgen05.mma (kind::f16, fp32
+//               accumulation), releasing ring stages with tcgen05.commit; with
+//               two accumulators the next unit's MMAs overlap the previous
+//               unit's epilogue,
 //   warps 2..5  epilogue: tcgen05.ld 16 columns at a time (warp w owns TMEM
 //               lanes 32*(w%4)..+31), then either the fused epilogue directly
-//               or, for K split over several CTAs, a partial plane; the CTAs
-//               of a tile (same round, co-resident by cooperative launch) wait
-//               for each other and each reduces a slice of the tile's rows in
-//               fixed split order (deterministic), then applies the epilogue.
+//               or, for K split over several CTAs, a partial plane and a
+//               ticket; either the slices of a tile (co-resident by
+//               cooperative launch) wait for each other and each reduces a
+//               share of the rows, or the slice that finishes last reduces the
+//               tile alone and nobody waits; both sum in fixed split order.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
 // the device error word and unwinds (freeing TMEM) instead of hanging.
 #include <algorithm>
@@ -67,6 +69,7 @@ struct RowMeta {
 
 struct GemmArgs {
     int M, N, K, kb_per_split, splits, n_tiles, m_tiles;
+    int coop;  // split fixup: 1 distributed (cooperative launch), 0 last arriver
     EpiParams ep;
 };
 
@@ -352,6 +355,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     uint64_t* accf = empty + STAGES;
     uint64_t* acce = accf + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+    int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // epilogue warps: this CTA reduces the tile
     RowMeta* meta = reinterpret_cast<RowMeta*>(smem + STAGES * C::STAGE_BYTES + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -518,30 +522,42 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acce[b]);
-                // Distributed fixup: the splits of a tile run in the same round
-                // on co-resident CTAs (cooperative launch); each one waits for
-                // all partial planes, then reduces its own slice of the tile's
-                // activation rows in fixed split order (deterministic) while the
-                // planes are still in L2.  The ticket counts 2*splits arrivals
-                // (written, then done reading) and the last one resets it.
+                // Two fixups of the K slices (both sum in fixed split order, so
+                // results are deterministic):
+                //  - distributed (g.coop, cooperative launch: the slices of a tile
+                //    run co-resident in the same round): every slice waits for all
+                //    planes, then reduces its own share of the tile's rows; the
+                //    ticket counts 2*splits arrivals (written, then done reading);
+                //  - last arriver: every slice leaves its plane and takes a ticket;
+                //    the one that arrives last reduces the whole tile and resets
+                //    the ticket; nobody waits.
                 __threadfence();
                 epi_bar();
                 int* ctr = g.ep.counters + tile;
-                if (threadIdx.x == 64) {
-                    atomicAdd(ctr, 1);
-                    const long long t0 = clock64();
-                    while (*reinterpret_cast<volatile int*>(ctr) < g.splits) {
-                        if (clock64() - t0 > 2000000000LL) {
-                            set_error(err, kErrTimeout);
-                            break;
+                int r0 = 0, r1 = BN;
+                if (g.coop) {
+                    if (threadIdx.x == 64) {
+                        atomicAdd(ctr, 1);
+                        const long long t0 = clock64();
+                        while (*reinterpret_cast<volatile int*>(ctr) < g.splits) {
+                            if (clock64() - t0 > 2000000000LL) {
+                                set_error(err, kErrTimeout);
+                                break;
+                            }
+                            __nanosleep(64);
                         }
-                        __nanosleep(64);
+                        __threadfence();
                     }
+                    epi_bar();
+                    const int rows = (BN + g.splits - 1) / g.splits;
+                    r0 = split * rows;
+                    r1 = min(BN, r0 + rows);
+                } else {
+                    if (threadIdx.x == 64) *last_flag = (atomicAdd(ctr, 1) == g.splits - 1) ? 1 : 0;
+                    epi_bar();
+                    if (!*last_flag) continue;
                     __threadfence();
                 }
-                epi_bar();
-                const int rows = (BN + g.splits - 1) / g.splits;
-                const int r0 = split * rows, r1 = min(BN, r0 + rows);
                 const int et = threadIdx.x - 64;
                 const int mr = et >> 5;
 #pragma unroll 1
@@ -593,7 +609,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 }
                 epi_bar();
                 if (threadIdx.x == 64) {
-                    if (atomicAdd(ctr, 1) == 2 * g.splits - 1) atomicExch(ctr, 0);
+                    if (!g.coop) *ctr = 0;
+                    else if (atomicAdd(ctr, 1) == 2 * g.splits - 1) atomicExch(ctr, 0);
                 }
             }
         }
@@ -632,9 +649,10 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
         if (e != cudaSuccess) return e;
         attr_dev = dev;
     }
-    if (a.splits == 1) return launch_pdl(gemm_tc_kernel<BN, WT, BK>, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
-    // CTAs of a split tile wait for one another: launch cooperatively so all of
-    // them are resident at once (the launch fails instead of deadlocking).
+    if (!(a.splits > 1 && a.coop))
+        return launch_pdl(gemm_tc_kernel<BN, WT, BK>, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
+    // The slices of a tile wait for one another: launch cooperatively so all CTAs
+    // are resident at once (the launch fails instead of deadlocking).
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(192);
@@ -673,7 +691,14 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
 }  // namespace
 
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                        int force_wt, int force_bk) {
+                        int force_wt, int force_bk, int force_coop) {
+    GemmPlan p = plan_gemm_bf16_shape(M, N, K, num_sms, max_splits, force_bn, force_splits, force_wt, force_bk);
+    p.coop = force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
+    return p;
+}
+
+GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
+                              int force_wt, int force_bk) {
     const int KB = (K + BK_DEFAULT - 1) / BK_DEFAULT;
     // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
     const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
@@ -738,7 +763,7 @@ bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K, const GemmPlan& p,
                              const EpiParams& ep, cudaStream_t st) {
     if (p.splits > 1 && (!ep.ws || !ep.counters)) return cudaErrorInvalidValue;
-    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, ep};
+    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, ep};
     if (p.bk == 32) {
         if (p.wt == 2 && p.bn == 256) return launch_bn<256, 2, 32>(tmW, tmX, a, p.grid, st);
         if (p.wt == 2 && p.bn == 128) return launch_bn<128, 2, 32>(tmW, tmX, a, p.grid, st);

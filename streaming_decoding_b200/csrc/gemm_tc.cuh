@@ -43,6 +43,7 @@ struct GemmPlan {
     int bn = 16;
     int wt = 1;
     int bk = 64;       // k-block depth: 64 (128-byte swizzle) or 32 (64-byte swizzle, bn >= 128)
+    int coop = 1;      // K-split fixup: 1 the slices wait and share the reduction, 0 the last one reduces
     int splits = 1;
     int kb_per_split = 1;
     int m_tiles = 1;
@@ -53,8 +54,12 @@ struct GemmPlan {
 // max_splits: the most K slices the caller's partial workspace holds (>= 1).
 // force_bn / force_splits > 0 pin the tile width / split count, force_wt = 2
 // selects 256-row weight tiles (tuning hooks).
+// force_coop: 1 / 0 pick the K-split fixup, -1 the default (distributed for
+// M > 128 rows, last arriver otherwise).
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0,
-                        int force_wt = 0, int force_bk = 0);
+                        int force_wt = 0, int force_bk = 0, int force_coop = -1);
+GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
+                              int force_wt, int force_bk);
 
 // 2-D bf16 tensor map [rows][cols], boxes of bk columns (64: 128-byte swizzle,
 // 32: 64-byte swizzle) by box_rows rows.

@@ -277,7 +277,8 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
     };
     std::vector<Shape> shapes;
     if (M > 128)
-        shapes = {{256, 1, 64}, {128, 1, 64}, {256, 2, 64}, {128, 2, 64}, {256, 2, 32}, {128, 2, 32}, {256, 1, 32}};
+        shapes = {{256, 1, 64}, {128, 1, 64}, {64, 1, 64}, {256, 2, 64}, {128, 2, 64}, {256, 2, 32}, {128, 2, 32},
+                  {256, 1, 32}};
     else if (M > 64) shapes = {{128, 1, 64}, {64, 1, 64}, {128, 2, 64}, {128, 2, 32}};
     else shapes = {{M <= 16 ? 16 : M <= 32 ? 32 : 64, 1, 64}};
     cudaEvent_t e0 = prof_event(ctx), e1 = prof_event(ctx);
@@ -288,9 +289,11 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
     ep.err = ctx->err;
     const int KB = (K + 63) / 64;
     for (const Shape& sh : shapes) {
-        for (int sp : {1, 2, 3, 4, 6, 8, 12, 16}) {
+        for (int spc : {1, 2, -2, 3, -3, 4, -4, 6, -6, 8, -8, 12, -12, 16, -16}) {
+            // negative: the same split count with the last-arriver fixup
+            const int sp = spc < 0 ? -spc : spc;
             if (sp > KB || (sp > 1 && N % 4)) continue;
-            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, sh.bn, sp, sh.wt, sh.bk);
+            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, sh.bn, sp, sh.wt, sh.bk, spc < 0 ? 0 : 1);
             if (p.splits != sp) continue;
             if (p.splits > 1 && ((size_t)p.splits * M * N > ctx->ws_floats ||
                                  (size_t)p.m_tiles * p.n_tiles > ctx->n_tile_counters))
@@ -811,7 +814,7 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     sa.add((void**)&ctx->ids_dev, (size_t)ctx->chunk * 4);
     // Attention key chunks for decode: fixed per context (a sequence's result
     // does not depend on its batch neighbours), sized so that a full batch at
-    // half the context length gives about two CTAs per SM; at most 2048 keys.
+    // half the context length gives about two CTAs per SM; 256 to 2048 keys.
     if (ctx->bf16) {
         const int g = ctx->hq / ctx->hkv;
         const int rt = attn_rows_per_tile(g);
@@ -819,7 +822,9 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         const long long pairs = (long long)B * tiles * ctx->hkv;
         const long long blocks = pairs * std::max(1, (ctx->max_ctx / 2 + 63) / 64);
         long long cb = (blocks + 2LL * ctx->num_sms - 1) / (2LL * ctx->num_sms);
-        cb = std::max(1LL, std::min(cb, 32LL));
+        // at least four blocks per chunk: below that the per-CTA setup and the
+        // merge of many partials outweigh the extra parallelism (small batches)
+        cb = std::max(4LL, std::min(cb, 32LL));
         // at most attn_max_splits() chunks per row tile (the merge keeps its weights on chip)
         const long long ms_cap = attn_max_splits();
         cb = std::max(cb, ((long long)ctx->max_ctx + 64 * ms_cap - 1) / (64 * ms_cap));
