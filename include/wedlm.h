@@ -289,6 +289,14 @@ wedlm_status wedlm_debug_read(wedlm_ctx* ctx, int32_t item, void* host_dst, int6
 wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t pos0, int32_t n,
                             float* host_k, float* host_v);
 
+/* Greedy bf16 steps fuse the entropy pass into the LM head: the GEMM's
+ * epilogue reduces each 32 vocabulary ids to (max, sum, weighted sum, argmax)
+ * partials and logits are never written (sampled steps and fp32 mode keep the
+ * two-pass path).  enable = 1 makes every step write logits and run the
+ * separate entropy pass, so WEDLM_DBG_LOGITS is valid after greedy bf16 steps
+ * too (test hook; synchronises the stream). */
+wedlm_status wedlm_debug_keep_logits(wedlm_ctx* ctx, int32_t enable);
+
 /* Residual-stream capture for per-layer comparisons.  While enabled (1), every
  * decode step keeps x (fp32, the residual stream) entering each layer and
  * after the last one; wedlm_debug_residual copies layer `layer` (0..n_layers,

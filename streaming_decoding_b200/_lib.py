@@ -67,6 +67,7 @@ _SIGS = {
     "wedlm_profile_enable": (c_i32, [c_vp, c_i32]),
     "wedlm_autotune": (c_i32, [c_vp, c_i32]),
     "wedlm_debug_capture": (c_i32, [c_vp, c_i32]),
+    "wedlm_debug_keep_logits": (c_i32, [c_vp, c_i32]),
     "wedlm_debug_residual": (c_i32, [c_vp, c_i32, c_vp, c_i32]),
     "wedlm_gemm_plan": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "wedlm_profile_read": (c_i32, [c_vp, c_vp, c_vp]),

@@ -142,6 +142,10 @@ class Engine:
     def autotune(self, enable: bool = True):
         _check(self.lib.wedlm_autotune(self.ctx, 1 if enable else 0), "wedlm_autotune", self.ctx)
 
+    def keep_logits(self, enable: bool = True):
+        """Write logits every step (two-pass entropy) so debug_read("LOGITS") is valid in bf16 mode."""
+        _check(self.lib.wedlm_debug_keep_logits(self.ctx, 1 if enable else 0), "wedlm_debug_keep_logits", self.ctx)
+
     def debug_capture(self, enable: bool = True):
         """Keep the residual stream at every layer boundary of each decode step (test hook)."""
         _check(self.lib.wedlm_debug_capture(self.ctx, 1 if enable else 0), "wedlm_debug_capture", self.ctx)

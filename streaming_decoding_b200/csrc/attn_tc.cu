@@ -50,7 +50,8 @@ constexpr int BLK_BYTES = 2 * HALF_BYTES;           // one K or V block: 16 KB
 constexpr int BOX_BYTES = kPage * 128;              // one page, one half: 2 KB
 constexpr int NTHREADS = 192;
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;  // S buffer b at TM_S + 64 b
-constexpr int MAX_SPLITS = 32;                       // key chunks per row tile (merge weights in smem)
+constexpr int MAX_SPLITS = 32;  // key chunks per row tile (merge weights in smem)
+constexpr int kMR = 8, kMS = 2;  // merge: rows x chunk partials in flight per lane
 constexpr int SMEM_BYTES = Q_BYTES + 2 * NST * BLK_BYTES + 256 + 1024 /*block maxima*/ + 1024 /*align*/;
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -575,12 +576,12 @@ __global__ void __launch_bounds__(NTHREADS, 2) attn_tc_kernel(const __grid_const
                 // then the rows: a warp takes one row at a time, a lane 4 dims
                 // (coalesced 512-byte reads per chunk partial)
 #pragma unroll 1
-                for (int row0 = warp; row0 < qrows; row0 += 4 * 4) {
-                    float4 acc[4];
-                    int64_t pbr[4];
-                    bool okr[4];
+                for (int row0 = warp; row0 < qrows; row0 += 4 * kMR) {
+                    float4 acc[kMR];
+                    int64_t pbr[kMR];
+                    bool okr[kMR];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < kMR; ++u) {
                         const int row = row0 + 4 * u;
                         okr[u] = row < qrows && r0 + row / g < n;
                         pbr[u] = ((int64_t)(entry * p.stride + r0 + row / g) * p.hq + kvh * g + row % g) *
@@ -588,19 +589,19 @@ __global__ void __launch_bounds__(NTHREADS, 2) attn_tc_kernel(const __grid_const
                         acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                     }
 #pragma unroll 1
-                    for (int s0 = 0; s0 < nsplit; s0 += 4) {
-                        float4 v[4][4];
+                    for (int s0 = 0; s0 < nsplit; s0 += kMS) {
+                        float4 v[kMR][kMS];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
+                        for (int u = 0; u < kMR; ++u)
 #pragma unroll
-                            for (int q = 0; q < 4; ++q)
+                            for (int q = 0; q < kMS; ++q)
                                 v[u][q] = (okr[u] && s0 + q < nsplit)
                                               ? __ldcg(reinterpret_cast<const float4*>(p.part_o + (pbr[u] + s0 + q) * HD) + lane)
                                               : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
+                        for (int u = 0; u < kMR; ++u)
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
+                            for (int q = 0; q < kMS; ++q) {
                                 const float w = (okr[u] && s0 + q < nsplit) ? wsm[(row0 + 4 * u) * MAX_SPLITS + s0 + q] : 0.f;
                                 acc[u].x += w * v[u][q].x;
                                 acc[u].y += w * v[u][q].y;
@@ -609,7 +610,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) attn_tc_kernel(const __grid_const
                             }
                     }
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < kMR; ++u) {
                         if (!okr[u]) continue;
                         const int row = row0 + 4 * u;
                         uint2 o;

@@ -263,6 +263,36 @@ __device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, i
     }
 }
 
+// LM-head epilogue without logits (EPI_ENTROPY): for each of 16 activation
+// rows, this warp's 32 vocab ids (one per lane, id n) reduce to the partial
+// (max, sum e^(z-max), sum e^(z-max)(z-max), lowest argmax) of z = scale * v
+// over valid ids (n < N, n != mask id); lane k stores row k's partial.
+__device__ __forceinline__ void entropy16(const EpiParams& ep, const float (&v)[16], bool valid, int n, int mbase,
+                                          int M, int pidx, int lane) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const float z = valid ? v[k] * ep.scale : -INFINITY;
+        float m = z;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float e = 0.f, t = 0.f;
+        if (valid && m != -INFINITY) {
+            e = expf(z - m);
+            t = e * (z - m);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+            t += __shfl_xor_sync(0xffffffffu, t, o);
+        }
+        int a = (valid && z == m) ? n : INT_MAX;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+        const int row = mbase + k;
+        if (lane == k && row < M) ep.epart[(int64_t)row * ep.npart + pidx] = make_float4(m, e, t, __int_as_float(a));
+    }
+}
+
 // Fused epilogue on weight rows n..n+3 (both row pairs inside this thread) of
 // eight activation rows m = mrow[u], after a split-K reduction.
 __device__ __forceinline__ void epilogue_vec4x8(const EpiParams& ep, int n0, int n, const int (&mrow)[8],
@@ -489,7 +519,23 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             fill_row_meta<BN>(g.ep, m0, g.M, meta, threadIdx.x - 64);
             epi_bar();
             const uint32_t tacc = tmem + b * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
-            if (g.splits == 1) {
+            if (g.splits == 1 && g.ep.kind == EPI_ENTROPY) {
+#pragma unroll 1
+                for (int w = 0; w < WT; ++w) {
+                    const int n = n0 + w * BM + q * 32 + lane;
+                    const bool valid = n < g.N && n != g.ep.mask_id;
+                    const int pidx = (n0 / BM + w) * 4 + q;
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 16) {
+                        float v[16];
+                        tmem_ld16(tacc + (uint32_t)(w * BN + c), v);
+                        entropy16(g.ep, v, valid, n, m0 + c, g.M, pidx, lane);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[b]);
+            } else if (g.splits == 1) {
 #pragma unroll 1
                 for (int w = 0; w < WT; ++w) {
                     const int nw = n0 + w * BM, n = nw + q * 32 + lane;
@@ -763,6 +809,8 @@ bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K, const GemmPlan& p,
                              const EpiParams& ep, cudaStream_t st) {
     if (p.splits > 1 && (!ep.ws || !ep.counters)) return cudaErrorInvalidValue;
+    if (ep.kind == EPI_ENTROPY && (p.splits != 1 || !ep.epart || ep.npart < ((N + 128 * p.wt - 1) / (128 * p.wt)) * p.wt * 4))
+        return cudaErrorInvalidValue;
     GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, ep};
     if (p.bk == 32) {
         if (p.wt == 2 && p.bn == 256) return launch_bn<256, 2, 32>(tmW, tmX, a, p.grid, st);

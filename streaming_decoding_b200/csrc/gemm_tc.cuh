@@ -15,7 +15,11 @@ namespace wedlm {
 //   EPI_QKV_ROPE  rotate q and k head dims (pairs interleaved in adjacent rows) at the
 //                 row's logical position; q -> act[m][hq][128], k and v -> KV pages at
 //                 cache index S + r of the row's sequence
-enum EpiKind : int { EPI_STORE = 0, EPI_QKV_ROPE = 1, EPI_SWIGLU = 2, EPI_RESIDUAL = 3 };
+//   EPI_ENTROPY   (LM head) logits are never stored: for every 32 vocab ids (one
+//                 warp's TMEM lanes) and activation row m, the partial
+//                 (max z, sum e^(z-max), sum e^(z-max)(z-max), lowest argmax) of
+//                 z = scale * Y over ids != mask_id -> epart[m][npart]
+enum EpiKind : int { EPI_STORE = 0, EPI_QKV_ROPE = 1, EPI_SWIGLU = 2, EPI_RESIDUAL = 3, EPI_ENTROPY = 4 };
 
 struct EpiParams {
     int kind = EPI_STORE;
@@ -30,6 +34,10 @@ struct EpiParams {
     SlotState ss{};
     RowMap rm{};
     int check_rows = 0;        // 1: skip rows RowMap marks as padding
+    float4* epart = nullptr;   // EPI_ENTROPY: partials [M][npart], npart = 4 per 128 weight rows
+    int npart = 0;
+    int mask_id = -1;
+    float scale = 1.f;
     float* ws = nullptr;       // split-K partial planes [splits][M][N]
     int* counters = nullptr;   // per-tile tickets; zero before and after every launch
     int* err = nullptr;

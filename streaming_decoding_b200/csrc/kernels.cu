@@ -347,16 +347,21 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(const float* __restr
 constexpr int kNormVec = 8;
 __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float* __restrict__ x, bf16* __restrict__ h,
                                                            const float* __restrict__ g, float eps, int d, RowMap rm) {
-    griddep_wait();
-    griddep_launch();
     __shared__ float red[32];
     const int row = blockIdx.x;
+    const float4* gr = reinterpret_cast<const float4*>(g);
+    const int nv = d >> 2;
+    float4 v[kNormVec], gv[kNormVec];
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {  // the gains are weights: read before the dependency wait
+        const int c = threadIdx.x + i * blockDim.x;
+        gv[i] = c < nv ? __ldg(gr + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    griddep_wait();
+    griddep_launch();
     int slot, r;
     if (!rm.live(row, slot, r)) return;
     const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * d);
-    const float4* gr = reinterpret_cast<const float4*>(g);
-    const int nv = d >> 2;
-    float4 v[kNormVec];
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < kNormVec; ++i) {
@@ -371,9 +376,8 @@ __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float* __restri
     for (int i = 0; i < kNormVec; ++i) {
         const int c = threadIdx.x + i * blockDim.x;
         if (c < nv) {
-            const float4 gg = gr[c];
-            hr[2 * c] = __floats2bfloat162_rn(v[i].x * inv * gg.x, v[i].y * inv * gg.y);
-            hr[2 * c + 1] = __floats2bfloat162_rn(v[i].z * inv * gg.z, v[i].w * inv * gg.w);
+            hr[2 * c] = __floats2bfloat162_rn(v[i].x * inv * gv[i].x, v[i].y * inv * gv[i].y);
+            hr[2 * c + 1] = __floats2bfloat162_rn(v[i].z * inv * gv[i].z, v[i].w * inv * gv[i].w);
         }
     }
 }
@@ -559,6 +563,36 @@ __global__ void __launch_bounds__(256) entropy_partial_kernel(const float* __res
         }
         part[(int64_t)row * chunks + c] = make_float4(t.m, t.s, t.t, __int_as_float(t.a));
         if (sampling) sa.part[(int64_t)row * chunks + c] = make_float2(tq.k, __int_as_float(tq.a));
+    }
+}
+
+// Second level of the fused LM-head entropy: merge the GEMM epilogue's
+// per-32-id partials of a masked row into `chunks` partials (the layout the
+// selection kernel reads).
+__global__ void __launch_bounds__(256) entropy_merge_kernel(const float4* __restrict__ part, int npart,
+                                                            const uint8_t* __restrict__ rowmask, int chunks,
+                                                            float4* __restrict__ out) {
+    griddep_wait();
+    griddep_launch();
+    const int row = blockIdx.y, c = blockIdx.x;
+    if (!rowmask[row]) return;
+    const int seg = (npart + chunks - 1) / chunks;
+    const int p0 = c * seg, p1 = min(npart, p0 + seg);
+    EntAcc e{-INFINITY, 0.f, 0.f, INT_MAX};
+    for (int i = p0 + threadIdx.x; i < p1; i += blockDim.x) {
+        const float4 q = __ldg(part + (int64_t)row * npart + i);
+        e = ent_merge(e, EntAcc{q.x, q.y, q.z, __float_as_int(q.w)});
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e = ent_shfl_merge(e, o);
+    __shared__ EntAcc sh[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) sh[warp] = e;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        EntAcc t = sh[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) t = ent_merge(t, sh[w]);
+        out[(int64_t)row * chunks + c] = make_float4(t.m, t.s, t.t, __int_as_float(t.a));
     }
 }
 
@@ -828,6 +862,11 @@ void launch_entropy_partials(const float* logits, int splits, int64_t sstride, i
     dim3 grid(chunks, rows);
     launch_pdl(entropy_partial_kernel, grid, dim3(256), 0, st, logits, splits, sstride, ld, V, mask_id, scale, rowmask,
                chunks, part, sa);
+}
+
+void launch_entropy_merge(const float4* part, int npart, const uint8_t* rowmask, int rows, int chunks, float4* out,
+                          cudaStream_t st) {
+    launch_pdl(entropy_merge_kernel, dim3(chunks, rows), dim3(256), 0, st, part, npart, rowmask, chunks, out);
 }
 
 void launch_select_commit(const float4* part, const float2* spart, int chunks, SlotState ss, RowState rs,

@@ -71,6 +71,11 @@ void launch_entropy_partials(const float* logits, int splits, int64_t split_stri
                              int mask_id, float scale, const uint8_t* rowmask, int rows, int chunks,
                              float4* part, cudaStream_t st, SampleArgs sa = SampleArgs());
 
+// Fused LM-head entropy, second level: per-32-id partials [rows][npart] of the
+// GEMM epilogue -> [rows][chunks] partials for the selection kernel.
+void launch_entropy_merge(const float4* part, int npart, const uint8_t* rowmask, int rows, int chunks, float4* out,
+                          cudaStream_t st);
+
 // spart: the sampling partials (read only when knobs.temperature > 0).
 void launch_select_commit(const float4* part, const float2* spart, int chunks, SlotState ss, RowState rs,
                           int n_entries, int stride, StepKnobs knobs, int* err, cudaStream_t st);

@@ -139,6 +139,11 @@ struct wedlm_ctx {
     float4* ent_part = nullptr;
     float2* samp_part = nullptr;  // Gumbel-max partials of sampled fills
     float* dbg_resid = nullptr;   // test hook: residual stream before each layer and after the last [L+1][Mdec][d]
+    float4* lm_part = nullptr;    // fused LM-head entropy partials [Mdec][lm_npart]
+    int lm_npart = 0;
+    bool keep_logits = false;     // test hook: write logits (unfused LM head + entropy pass)
+    std::map<int, bool> fuse_choice;  // rows -> fused LM-head entropy is the faster path
+    bool capturing = false;           // a step is being captured into a CUDA graph: no timing runs
     float* attn_po = nullptr;
     float2* attn_pml = nullptr;
     int* attn_tickets = nullptr;   // [maxB][hkv][tiles] merge tickets of the key-chunked attention
@@ -261,9 +266,13 @@ wedlm_status gemm_f32(wedlm_ctx* ctx, int kind, const float* X, const float* W, 
 // launch that follows rewrites anyway (the q / activation scratch, and K/V
 // at the window's own cache positions).  Runs once per (kind, M) on the
 // context's stream; candidates that do not fit the scratch buffers are skipped.
+// Tuning key of a projection: the LM head with the entropy epilogue is tuned
+// apart from the plain LM head (its epilogue costs differ).
+int tune_kind(int kind, const EpiParams& ep) { return ep.kind == EPI_ENTROPY ? kind + 1000 : kind; }
+
 void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WMap* tmW, int M, int N, int K,
                     const EpiParams& ep_real) {
-    const std::pair<int, int> key(kind, M);
+    const std::pair<int, int> key(tune_kind(kind, ep_real), M);
     if (ctx->tuned.count(key)) return;
     ctx->tuned[key] = {plan_gemm_bf16(M, N, K, ctx->num_sms, 1), -1.f};
     EpiParams ep = ep_real;
@@ -329,14 +338,17 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
 wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WMap* tmW, int M, int N, int K,
                        EpiParams ep, bool tune = true) {
     GemmPlan p;
-    if (ctx->autotune && tune) {
+    const bool tuned = ctx->tuned.count({tune_kind(kind, ep), M}) > 0;
+    if (ctx->autotune && tune && (tuned || !ctx->capturing)) {  // no timing runs inside a graph capture
         autotune_shape(ctx, kind, X, tmW, M, N, K, ep);
-        p = ctx->tuned[{kind, M}].plan;
+        p = ctx->tuned[{tune_kind(kind, ep), M}].plan;
     } else {
         const size_t plane = (size_t)M * N;
         const int cap = (int)std::max<size_t>(1, std::min<size_t>(16, ctx->ws_floats / plane));
         p = plan_gemm_bf16(M, N, K, ctx->num_sms, cap);
     }
+    if (ep.kind == EPI_ENTROPY && p.splits != 1)  // the entropy epilogue needs whole K sums
+        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk);
     if (p.splits > 1 && ((size_t)p.n_tiles * p.m_tiles > ctx->n_tile_counters ||
                          (size_t)p.splits * M * N > ctx->ws_floats))
         p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk);
@@ -539,6 +551,51 @@ int max_active_window(const wedlm_ctx* c, int* n_entries) {
 }
 
 // Enqueue one decode step over slots [0, n_entries) with row stride `stride`.
+// LM head over the step's rows and the entropy partials of the masked rows:
+// fused (the GEMM epilogue reduces each 32 vocab ids; one merge kernel) or
+// two-pass (logits written, then one streaming scan, with sampling keys when
+// the step samples).
+wedlm_status lm_head_entropy(wedlm_ctx* ctx, const wedlm_step_params* prm, int M, int stride, bool fused) {
+    wedlm_status s;
+    if (fused) {
+        EpiParams e;
+        e.kind = EPI_ENTROPY;
+        e.epart = ctx->lm_part;
+        e.npart = ctx->lm_npart;
+        e.mask_id = ctx->cfg.mask_id;
+        e.scale = prm->logit_scale;
+        if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, &ctx->tm_lm, M, ctx->V, ctx->d, e))) return s;
+        ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
+        launch_entropy_merge(ctx->lm_part, ctx->lm_npart, ctx->rowmask, M, kEntropyChunks, ctx->ent_part,
+                             ctx->stream);
+        return WEDLM_OK;
+    }
+    if (ctx->bf16) {
+        EpiParams e;
+        e.kind = EPI_STORE;
+        e.out = ctx->logits;
+        if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, &ctx->tm_lm, M, ctx->V, ctx->d, e))) return s;
+    } else {
+        if ((size_t)M * ctx->V > ctx->logits_floats) return fail(ctx, WEDLM_ERR_STATE, "logits buffer too small");
+        ProfScope ps(ctx, WEDLM_PROF_GEMM_LM_HEAD);
+        launch_gemm_f32((const float*)ctx->h, (const float*)ctx->lm_head, ctx->logits, M, ctx->V, ctx->d,
+                        ctx->stream);
+    }
+    ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
+    SampleArgs sa;
+    if (prm->temperature > 0.f) {
+        sa.inv_t = 1.0f / prm->temperature;
+        sa.seed = prm->seed;
+        sa.stride = stride;
+        sa.pos = ctx->rs.pos;
+        sa.steps = ctx->ss.counters;
+        sa.part = ctx->samp_part;
+    }
+    launch_entropy_partials(ctx->logits, 1, (int64_t)M * ctx->V, ctx->V, ctx->V, ctx->cfg.mask_id, prm->logit_scale,
+                            ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream, sa);
+    return WEDLM_OK;
+}
+
 wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_entries, int stride) {
     const int M = n_entries * stride;
     {
@@ -554,33 +611,43 @@ wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, 
     }
     wedlm_status s = run_forward(ctx, 0, n_entries, stride, true);
     if (s) return s;
-    const int lsp = 1;
-    if (ctx->bf16) {
-        EpiParams e;
-        e.kind = EPI_STORE;
-        e.out = ctx->logits;
-        s = gemm_bf16(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, &ctx->tm_lm, M, ctx->V, ctx->d, e);
-    } else {
-        if ((size_t)M * ctx->V > ctx->logits_floats) return fail(ctx, WEDLM_ERR_STATE, "logits buffer too small");
-        ProfScope ps(ctx, WEDLM_PROF_GEMM_LM_HEAD);
-        launch_gemm_f32((const float*)ctx->h, (const float*)ctx->lm_head, ctx->logits, M, ctx->V, ctx->d, ctx->stream);
-        s = WEDLM_OK;
-    }
-    if (s) return s;
-    {
-        ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
-        SampleArgs sa;
-        if (prm->temperature > 0.f) {
-            sa.inv_t = 1.0f / prm->temperature;
-            sa.seed = prm->seed;
-            sa.stride = stride;
-            sa.pos = ctx->rs.pos;
-            sa.steps = ctx->ss.counters;
-            sa.part = ctx->samp_part;
+    // Greedy bf16 steps may fuse the entropy into the LM head (logits never
+    // stored); which of the two is faster at this row count is timed once
+    // (autotuning on) or taken from the row count (off).  Sampling and the
+    // logits test hook always take the two-pass path.
+    const bool fusable = ctx->bf16 && !ctx->keep_logits && prm->temperature == 0.f;
+    bool fused = false;
+    if (fusable) {
+        auto it = ctx->fuse_choice.find(M);
+        if (it == ctx->fuse_choice.end()) {
+            bool choice = M <= 64;
+            if (ctx->autotune && !ctx->capturing) {
+                // both variants once to tune their GEMMs, then once more each, timed
+                if ((s = lm_head_entropy(ctx, prm, M, stride, false)) || (s = lm_head_entropy(ctx, prm, M, stride, true)))
+                    return s;
+                cudaEvent_t e0, e1, e2;
+                cudaEventCreate(&e0);
+                cudaEventCreate(&e1);
+                cudaEventCreate(&e2);
+                cudaEventRecord(e0, ctx->stream);
+                if ((s = lm_head_entropy(ctx, prm, M, stride, false))) return s;
+                cudaEventRecord(e1, ctx->stream);
+                if ((s = lm_head_entropy(ctx, prm, M, stride, true))) return s;
+                cudaEventRecord(e2, ctx->stream);
+                cudaEventSynchronize(e2);
+                float t_two = 0.f, t_fused = 0.f;
+                cudaEventElapsedTime(&t_two, e0, e1);
+                cudaEventElapsedTime(&t_fused, e1, e2);
+                cudaEventDestroy(e0);
+                cudaEventDestroy(e1);
+                cudaEventDestroy(e2);
+                choice = t_fused < t_two;
+            }
+            it = ctx->fuse_choice.emplace(M, choice).first;
         }
-        launch_entropy_partials(ctx->logits, lsp, (int64_t)M * ctx->V, ctx->V, ctx->V, ctx->cfg.mask_id,
-                                prm->logit_scale, ctx->rowmask, M, kEntropyChunks, ctx->ent_part, ctx->stream, sa);
+        fused = it->second;
     }
+    if ((s = lm_head_entropy(ctx, prm, M, stride, fused))) return s;
     StepKnobs kn{prm->lambda, prm->tau, prm->logit_scale, prm->tau_none, prm->blockwise, prm->temperature, prm->seed};
     {
         ProfScope ps(ctx, WEDLM_PROF_SELECT);
@@ -595,7 +662,7 @@ wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, 
         const cudaError_t le = cudaGetLastError();
         if (le != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(le));
     }
-    ctx->logits_splits_last = lsp;
+    ctx->logits_splits_last = 1;
     if (ctx->prof && ctx->ev_marks.size() > 4096) prof_collect(ctx);
     return WEDLM_OK;
 }
@@ -637,7 +704,9 @@ wedlm_status enqueue_step(wedlm_ctx* ctx, const wedlm_step_params* prm, int n_en
     cudaError_t e = cudaStreamBeginCapture(ctx->stream, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return fail(ctx, WEDLM_ERR_CUDA, std::string("begin capture: ") + cudaGetErrorString(e));
     const int64_t l0 = ctx->launches;
+    ctx->capturing = true;
     wedlm_status s = enqueue_step_kernels(ctx, prm, n_entries, stride);
+    ctx->capturing = false;
     e = cudaStreamEndCapture(ctx->stream, &graph);
     if (s) {
         if (graph) cudaGraphDestroy(graph);
@@ -873,6 +942,10 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     xa.add((void**)&ctx->logits, ctx->logits_floats * 4);
     xa.add((void**)&ctx->ent_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float4));
     xa.add((void**)&ctx->samp_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float2));
+    if (ctx->bf16) {
+        ctx->lm_npart = ((V + 255) / 256) * 2 * 4;  // 4 per 128 vocab rows, for 128- or 256-row tiles
+        xa.add((void**)&ctx->lm_part, (size_t)ctx->Mdec * ctx->lm_npart * sizeof(float4));
+    }
     if (ctx->bf16 && ctx->attn_max_splits > 1) {
         const size_t pairs = (size_t)ctx->Mdec * ctx->hq * ctx->attn_max_splits;
         xa.add((void**)&ctx->attn_po, pairs * ctx->hd * 4);
@@ -1210,6 +1283,7 @@ wedlm_status wedlm_autotune(wedlm_ctx* ctx, int32_t enable) {
     if (!ctx) return WEDLM_ERR_INVALID_ARG;
     ctx->autotune = enable != 0;
     ctx->tuned.clear();
+    ctx->fuse_choice.clear();
     drop_graph(ctx);
     ctx->eager_key = wedlm_ctx::StepKey();
     return WEDLM_OK;
@@ -1328,6 +1402,17 @@ wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t
                     (kv ? host_v : host_k)[((size_t)i * hkv + hh) * hd + c] = v;
                 }
     }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_keep_logits(wedlm_ctx* ctx, int32_t enable) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    CK(cudaStreamSynchronize(ctx->stream));
+    if (ctx->keep_logits != (enable != 0)) {
+        drop_graph(ctx);
+        ctx->eager_key = wedlm_ctx::StepKey();  // the next step runs eagerly (it may tune)
+    }
+    ctx->keep_logits = enable != 0;
     return WEDLM_OK;
 }
 

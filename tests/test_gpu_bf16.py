@@ -36,6 +36,7 @@ def test_teacher_forced_logits_and_decisions(model, lam, tau, scale):
     N, W = 20, 16
     prompts = _prompts()
     eng = make_engine(MID, max_batch=3, max_window=16, max_ctx=1024, prefill_chunk=128)
+    eng.keep_logits(True)  # logits are read back below (two-pass entropy)
     for b, p in prompts.items():
         eng.prefill(b, p, N, W)
     prm = step_params(lam, tau, False, scale)
@@ -138,3 +139,37 @@ def test_graph_replay_matches_eager_decoding():
         eng.close()
     assert outs[0][0] == outs[1][0]
     assert outs[0][1] == outs[1][1]
+
+
+def test_fused_lm_head_entropy_matches_two_pass():
+    """Greedy bf16 steps reduce the vocabulary in the LM head's epilogue (per-32-id
+    partials, merged) instead of writing logits and scanning them: every step's
+    H~, fills, commits and the token streams equal those of the two-pass path
+    run on the same inputs (H~ within the decision margin)."""
+    from streaming_decoding_b200 import step_params
+    N, W = 24, 16
+    prompts = _prompts()
+    runs = []
+    for keep in (False, True):
+        eng = make_engine(MID, max_batch=3, max_window=16, max_ctx=1024, prefill_chunk=128)
+        eng.autotune(False)
+        eng.keep_logits(keep)
+        for b, p in prompts.items():
+            eng.prefill(b, p, N, W)
+        prm = step_params(0.05, 6.0, False, 16.0)
+        trace, active = [], 3
+        while active:
+            _, _, active = eng.stream_step(prm)
+            trace.append((eng.debug_read("KN", (3, 3), np.int32).copy(),
+                          eng.debug_read("HTILDE", (3, 16), np.float32).copy(),
+                          eng.debug_read("FILL", (3, 16), np.uint8).copy(),
+                          eng.debug_read("ARGMAX", (3, 16), np.int32).copy()))
+        runs.append((trace, [eng.read_generated(b) for b in prompts]))
+        eng.close()
+    (tf, gf), (tt, gt) = runs
+    assert gf == gt and len(tf) == len(tt)
+    for (kf, hf, ff, af), (kt, ht, ft, at) in zip(tf, tt):
+        assert (kf == kt).all() and (ff == ft).all() and (af == at).all()
+        ok = ~np.isnan(ht)
+        assert (np.isnan(hf) == ~ok).all()
+        assert np.abs(hf[ok] - ht[ok]).max(initial=0.0) < MARGIN

@@ -54,6 +54,7 @@ def test_full_size_batch16_per_layer_against_oracle():
     f0, t0 = eng.get_window(b)
     gen = eng.read_generated(b)
     eng.debug_capture(True)
+    eng.keep_logits(True)  # the logits are read back
     eng.stream_step(prm)
     stride, rows = eng.last_rows()
     assert (stride, rows) == (W, B * W)
