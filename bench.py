@@ -515,20 +515,21 @@ def gemm_sweep():
         for name, (_, _, N, K) in gemm_shapes(dims, M).items():
             W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
             Xk = X[:, :K].contiguous()
-            bns = [0] + ([256, 128] if M > 128 else [16])
+            shapes = [(0, False)] + ([(256, False), (128, False), (256, True), (128, True)] if M > 128
+                                     else [(16, False)])
             res = []
-            for bn in bns:
+            for bn, pair in shapes:
                 for sp in ([0] if bn == 0 else [1, 2, 3, 4, 6, 8]):
                     for _ in range(2):
-                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp)
+                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp, cta_pair=pair)
                     st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                     st.record()
                     for _ in range(10):
-                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp)
+                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp, cta_pair=pair)
                     en.record()
                     en.synchronize()
                     us = st.elapsed_time(en) * 100.0
-                    res.append({"bn": bn, "splits": sp, "us": round(us, 2),
+                    res.append({"bn": bn, "pair": pair, "splits": sp, "us": round(us, 2),
                                 "weight_GBps": round(2 * N * K / us / 1e3, 1),
                                 "TFLOPs": round(2 * M * N * K / us / 1e6, 1)})
             del W

@@ -387,6 +387,14 @@ wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M
 wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
                                     int32_t tile_n, int32_t k_splits, void* stream);
 
+/* wedlm_linear_bf16_plan on CTA-pair tiles: two CTAs of a cluster compute a
+ * tile of 256 weight rows by tile_n activation rows with the two-CTA tensor-core
+ * MMA, each staging its own 128 weight rows and half of the activation rows.
+ * tile_n must be 128 or 256 (WEDLM_ERR_INVALID_ARG otherwise); k_splits as
+ * above (slices reduced by the last one to finish). */
+wedlm_status wedlm_linear_bf16_pair(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                    int32_t tile_n, int32_t k_splits, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

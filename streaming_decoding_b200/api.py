@@ -261,14 +261,15 @@ def entropy_select_noalloc(logits, vocab: int, mask_id: int, filled, n, stride: 
     return ht, am, fill
 
 
-def linear_bf16(X, W, stream=None, tile_n: int = 0, k_splits: int = 0):
+def linear_bf16(X, W, stream=None, tile_n: int = 0, k_splits: int = 0, cta_pair: bool = False):
     """Y = X W^T (fp32) on the tcgen05 GEMM; X [M][K], W [N][K] torch.bfloat16 CUDA tensors.
-    tile_n / k_splits pin the launch shape (0 = automatic)."""
+    tile_n / k_splits pin the launch shape (0 = automatic); cta_pair runs CTA-pair
+    tiles of 256 weight rows (tile_n 128 or 256)."""
     import torch
     M, K = X.shape
     N = W.shape[0]
     Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
     X, W = X.contiguous(), W.contiguous()
-    _check(_lib.load().wedlm_linear_bf16_plan(_ptr(X), _ptr(W), _ptr(Y), M, N, K, tile_n, k_splits,
-                                              _stream_handle(stream)), "wedlm_linear_bf16_plan")
+    fn = "wedlm_linear_bf16_pair" if cta_pair else "wedlm_linear_bf16_plan"
+    _check(getattr(_lib.load(), fn)(_ptr(X), _ptr(W), _ptr(Y), M, N, K, tile_n, k_splits, _stream_handle(stream)), fn)
     return Y

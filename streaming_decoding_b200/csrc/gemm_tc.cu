@@ -24,6 +24,16 @@
 //               cooperative launch) wait for each other and each reduces a
 //               share of the rows, or the slice that finishes last reduces the
 //               tile alone and nobody waits; both sum in fixed split order.
+// CTA pairs (CG = 2, clusters of two): the pair computes a 256-row weight tile
+// with tcgen05.mma.cta_group::2 issued by the even CTA.  Each CTA stages its own
+// 128 weight rows and half of the activation rows; the MMA reads the operands
+// from both CTAs' shared memory and writes each CTA's 128 accumulator lanes in
+// its own TMEM.  Per output a CTA moves half the activation bytes of a
+// single-CTA tile of the same width, which is what limits the main loop: the
+// operand bytes streamed from L2 into each SM per k-block.  Loads of both CTAs
+// complete on the even CTA's ring barrier; its commits release the ring stage
+// and hand over the accumulator in both CTAs; both CTAs' epilogues release the
+// accumulator on the even CTA's barrier.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
 // the device error word and unwinds (freeing TMEM) instead of hanging.
 #include <algorithm>
@@ -45,17 +55,23 @@ constexpr int BK_DEFAULT = 64;  // k-block depth of the 128-byte-swizzle tiles
 // (two when they fit, so a unit's MMAs overlap the previous unit's epilogue).
 // BK = 64 (128-byte rows, 128-byte swizzle) or 32 (64-byte rows, 64-byte
 // swizzle: half the bytes per stage, so twice the stages in flight).
-template <int BN, int WT, int BK> struct PCfg {
+// CG = 2: CTA pair, BN activation rows per pair (BN / 2 staged by each CTA).
+template <int BN, int WT, int BK, int CG> struct PCfg {
+    static_assert(CG == 1 || (CG == 2 && WT == 1 && BK == 64 && BN >= 64), "pair tiles: one weight sub-tile per CTA");
     static constexpr int SUB_A_BYTES = BM * BK * 2;  // one 128-row weight sub-tile of a stage
     static constexpr int A_STAGE_BYTES = WT * SUB_A_BYTES;
-    static constexpr int B_STAGE_BYTES = BN * BK * 2;
+    static constexpr int B_ROWS = BN / CG;  // activation rows this CTA stages
+    static constexpr int B_STAGE_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
     static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 12 ? 12 : (200 * 1024) / STAGE_BYTES;
     static constexpr int ACC_COLS = WT * BN;
     static constexpr int NACC = 2 * ACC_COLS <= 512 ? 2 : 1;
     static constexpr int TMEM_COLS = NACC * ACC_COLS < 32 ? 32 : NACC * ACC_COLS;
     static constexpr int META_BYTES = BN * 16;  // per activation row: live, pos, cache-row offset
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + META_BYTES;
+    // epilogue staging: 32 accumulator columns (activation rows) x 128 weight rows, fp32
+    static constexpr int EPI_COLS = 32;
+    static constexpr int EPI_BYTES = BN >= EPI_COLS ? EPI_COLS * BM * 4 : 0;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ + META_BYTES + EPI_BYTES;
 };
 
 // What the epilogue needs per activation row of the current unit, computed
@@ -95,6 +111,67 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, in
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+// ---- CTA-pair (cluster of two) primitives
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory object in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// Barrier over every thread of both CTAs (each CTA's threads all reach it).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+// TMA load into this CTA's shared memory that completes on an mbarrier of
+// either CTA of the pair (cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* tm, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (arrivals from the peer CTA).
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t parity, int* err) {
+    const long long t0 = clock64();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((it & 1023u) == 1023u) {
+            if (err && *reinterpret_cast<volatile int*>(err) != 0) return false;
+            if (clock64() - t0 > 2000000000LL) {
+                set_error(err, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
 // Shared-memory matrix descriptor of a K-major tile of BK-element rows stored
 // with the matching swizzle: BK = 64 -> 128-byte rows, 128-byte swizzle, 8-row
 // atoms 1024 B apart; BK = 32 -> 64-byte rows, 64-byte swizzle, atoms 512 B apart.
@@ -115,18 +192,56 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+template <int CG>
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
+    if constexpr (CG == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc)
+            : "memory");
 }
 
+// Arrive on `bar` once the MMAs issued so far complete; a pair arrives on the
+// barrier at the same offset in both CTAs (one commit per CTA, by cluster address).
+template <int CG>
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
+    if constexpr (CG == 2) {
+#pragma unroll
+        for (uint32_t r = 0; r < 2; ++r)
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         ::"r"(mapa_rank(smem_u32(bar), r))
+                         : "memory");
+    } else
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                     : "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this warp's 32 TMEM lanes (one
+// load and its wait in one statement, so no use is scheduled before the wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 16 consecutive fp32 accumulator columns of this warp's 32 TMEM lanes.
@@ -368,13 +483,13 @@ __device__ __forceinline__ void epilogue_vec4x8(const EpiParams& ep, int n0, int
     }
 }
 
-template <int BN, int WT, int BK>
+template <int BN, int WT, int BK, int CG>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
                                                          const __grid_constant__ CUtensorMap tmX, const GemmArgs g) {
-    using C = PCfg<BN, WT, BK>;
+    using C = PCfg<BN, WT, BK, CG>;
     constexpr int SUB_A_BYTES = C::SUB_A_BYTES;
     constexpr int NACC = C::NACC;
-    constexpr int TW = BM * WT;  // weight rows per tile
+    constexpr int TW = BM * WT * CG;  // weight rows per tile (of the pair when CG = 2)
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -387,11 +502,16 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
     int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // epilogue warps: this CTA reduces the tile
     RowMeta* meta = reinterpret_cast<RowMeta*>(smem + STAGES * C::STAGE_BYTES + 256);
+    float* epi_stage = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256 + C::META_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = (g.K + BK - 1) / BK;
     const int units = g.n_tiles * g.m_tiles * g.splits;
     int* err = g.ep.err;
+    // Unit schedule: units u0, u0 + ustep, ... (per CTA, or per pair).
+    const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
+    const int u0 = CG == 2 ? (int)cluster_id() : (int)blockIdx.x;
+    const int ustep = CG == 2 ? (int)cluster_count() : (int)gridDim.x;
 
     if (threadIdx.x == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
@@ -402,19 +522,29 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&accf[b], 1);
-            mbar_init(&acce[b], 4);
+            mbar_init(&acce[b], 4 * CG);  // the epilogue warps of every CTA of the pair
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(C::TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (CG == 2) {  // one warp of each CTA of the pair, collectively
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(C::TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(C::TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CG == 2)
+        cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -423,28 +553,39 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             // Weights never depend on the previous kernel: the first ring slots
             // of the first unit get their weight tiles before the dependency
             // wait (overlapping that kernel's tail), the activations after it.
+            // A pair's loads all complete on the even CTA's ring barrier, which
+            // expects the bytes of both CTAs.
+            auto load = [&](void* dst, const CUtensorMap* tm, int x, int y, int s) {
+                if constexpr (CG == 2)
+                    tma_load_2d_pair(dst, tm, x, y, mapa_rank(smem_u32(&full[s]), 0));
+                else
+                    tma_load_2d(dst, tm, x, y, &full[s]);
+            };
+            auto expect = [&](int s) {
+                if (rank == 0) mbar_expect_tx(&full[s], CG * C::STAGE_BYTES);
+            };
             uint32_t it = 0;
             int pre = 0;
-            if ((int)blockIdx.x < units) {
-                const int split = blockIdx.x % g.splits, tile = blockIdx.x / g.splits;
-                const int n0 = (tile / g.m_tiles) * TW;
+            if (u0 < units) {
+                const int split = u0 % g.splits, tile = u0 / g.splits;
+                const int na = (tile / g.m_tiles) * TW + (int)rank * BM;
                 const int kb0 = split * g.kb_per_split;
                 const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
                 pre = min(nkb, STAGES);
                 for (int i = 0; i < pre; ++i) {
-                    mbar_expect_tx(&full[i], C::STAGE_BYTES);
+                    expect(i);
 #pragma unroll
                     for (int w = 0; w < WT; ++w)
-                        tma_load_2d(sA + i * C::A_STAGE_BYTES + w * SUB_A_BYTES, &tmW, (kb0 + i) * BK, n0 + w * BM,
-                                    &full[i]);
+                        load(sA + i * C::A_STAGE_BYTES + w * SUB_A_BYTES, &tmW, (kb0 + i) * BK, na + w * BM, i);
                 }
             }
             griddep_wait();
             griddep_launch();
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            for (int u = u0; u < units && ok; u += ustep) {
                 const int split = u % g.splits, tile = u / g.splits;
-                const int n0 = (tile / g.m_tiles) * TW, m0 = (tile % g.m_tiles) * BN;
+                const int na = (tile / g.m_tiles) * TW + (int)rank * BM;
+                const int mb = (tile % g.m_tiles) * BN + (int)rank * C::B_ROWS;
                 const int kb0 = split * g.kb_per_split;
                 const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
                 for (int i = 0; i < nkb; ++i, ++it) {
@@ -456,13 +597,19 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                             ok = false;
                             break;
                         }
-                        mbar_expect_tx(&full[s], C::STAGE_BYTES);
+                        expect(s);
 #pragma unroll
                         for (int w = 0; w < WT; ++w)
-                            tma_load_2d(sA + s * C::A_STAGE_BYTES + w * SUB_A_BYTES, &tmW, kx, n0 + w * BM, &full[s]);
+                            load(sA + s * C::A_STAGE_BYTES + w * SUB_A_BYTES, &tmW, kx, na + w * BM, s);
                     }
-                    tma_load_2d(sB + s * C::B_STAGE_BYTES, &tmX, kx, m0, &full[s]);
+                    load(sB + s * C::B_STAGE_BYTES, &tmX, kx, mb, s);
                 }
+            }
+            if constexpr (CG == 2) {
+                // Drain: every stage's last release (a commit from the even CTA)
+                // lands before this CTA may exit.
+                for (uint32_t f = it > (uint32_t)STAGES ? it - STAGES : 0u; f < it && ok; ++f)
+                    ok = mbar_wait_bounded(smem_u32(&empty[f % STAGES]), (f / STAGES) & 1u, err);
             }
         } else {
             griddep_wait();
@@ -471,16 +618,18 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     } else if (warp == 1) {
         griddep_wait();
         griddep_launch();
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        if (lane == 0 && rank == 0) {  // a pair's MMAs are issued by its even CTA
+            constexpr uint32_t idesc = idesc_bf16(BM * CG, BN);
             uint32_t it = 0, j = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++j) {
+            for (int u = u0; u < units && ok; u += ustep, ++j) {
                 const int split = u % g.splits;
                 const int kb0 = split * g.kb_per_split;
                 const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
                 const uint32_t b = j % NACC, use = j / NACC;
-                if (!mbar_wait_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err)) break;
+                const bool free_acc = CG == 2 ? mbar_wait_cluster_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err)
+                                              : mbar_wait_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err);
+                if (!free_acc) break;
                 tc_fence_after();
                 const uint32_t d = tmem + b * C::ACC_COLS;
                 for (int i = 0; i < nkb; ++i, ++it) {
@@ -497,21 +646,29 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     for (int kk = 0; kk < BK / 16; ++kk)
 #pragma unroll
                         for (int w = 0; w < WT; ++w)
-                            umma_bf16(d + w * BN, sdesc_k<BK>(a + w * SUB_A_BYTES + kk * 32),
-                                      sdesc_k<BK>(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&empty[s]);
+                            umma_bf16<CG>(d + w * BN, sdesc_k<BK>(a + w * SUB_A_BYTES + kk * 32),
+                                          sdesc_k<BK>(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit<CG>(&empty[s]);
                 }
-                umma_commit(&accf[b]);
+                umma_commit<CG>(&accf[b]);
             }
         }
     } else {
         griddep_wait();
         griddep_launch();
         const int q = warp & 3;
+        // the accumulator is released on the even CTA's barrier
+        auto release = [&](uint32_t b) {
+            if constexpr (CG == 2)
+                mbar_arrive_cluster(mapa_rank(smem_u32(&acce[b]), 0));
+            else
+                mbar_arrive(&acce[b]);
+        };
         uint32_t j = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x, ++j) {
+        for (int u = u0; u < units; u += ustep, ++j) {
             const int split = u % g.splits, tile = u / g.splits;
-            const int n0 = (tile / g.m_tiles) * TW, m0 = (tile % g.m_tiles) * BN;
+            // n0: this CTA's first weight row (its TMEM lanes); m0: the tile's first activation row
+            const int n0 = (tile / g.m_tiles) * TW + (int)rank * BM, m0 = (tile % g.m_tiles) * BN;
             const uint32_t b = j % NACC, use = j / NACC;
             const bool ok = epi_all(mbar_wait_bounded(smem_u32(&accf[b]), use & 1u, err));
             if (!ok) break;
@@ -534,7 +691,57 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acce[b]);
+                if (lane == 0) release(b);
+            } else if (g.splits == 1 && BN >= C::EPI_COLS && (g.N & 3) == 0) {
+                // Through shared memory: 32 accumulator columns at a time are
+                // stored transposed (row = activation row, 128 weight rows; each
+                // store instruction writes 32 consecutive words), then each thread
+                // runs the fused epilogue on float4 runs of weight rows for 8
+                // activation rows: coalesced rows, vector stores, few instructions.
+                const int et = threadIdx.x - 64;
+                const int c4 = 4 * (et & 31);
+                bool released = false;
+#pragma unroll 1
+                for (int w = 0; w < WT; ++w) {
+                    const int nw = n0 + w * BM, nn = nw + c4;
+                    const bool nok = nn < g.N;
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += C::EPI_COLS) {
+                        {
+                            float v[C::EPI_COLS];
+                            tmem_ld32(tacc + (uint32_t)(w * BN + c), v);
+                            if (w == WT - 1 && c + C::EPI_COLS >= BN) {
+                                // the accumulator is fully read: the next unit's MMAs may start
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) release(b);
+                                released = true;
+                            }
+                            float* srow = epi_stage + q * 32 + lane;
+#pragma unroll
+                            for (int k = 0; k < C::EPI_COLS; ++k) srow[k * BM] = v[k];
+                        }
+                        epi_bar();
+                        float4 acc[8];
+                        int mrow[8], krow[8];
+                        bool okr[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const int rl = q + 4 * u;  // row within the staged columns
+                            krow[u] = c + rl;
+                            mrow[u] = m0 + c + rl;
+                            okr[u] = nok && mrow[u] < g.M;
+                            acc[u] = *reinterpret_cast<const float4*>(epi_stage + rl * BM + c4);
+                        }
+                        epilogue_vec4x8(g.ep, nw, nn, mrow, krow, okr, meta, acc, g.N);
+                        epi_bar();
+                    }
+                }
+                if (!released) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) release(b);
+                }
             } else if (g.splits == 1) {
 #pragma unroll 1
                 for (int w = 0; w < WT; ++w) {
@@ -548,7 +755,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acce[b]);
+                if (lane == 0) release(b);
             } else {
                 float* plane = g.ep.ws + (int64_t)split * g.M * g.N;
 #pragma unroll 1
@@ -567,7 +774,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&acce[b]);
+                if (lane == 0) release(b);
                 // Two fixups of the K slices (both sum in fixed split order, so
                 // results are deterministic):
                 //  - distributed (g.coop, cooperative launch: the slices of a tile
@@ -579,7 +786,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 //    the ticket; nobody waits.
                 __threadfence();
                 epi_bar();
-                int* ctr = g.ep.counters + tile;
+                int* ctr = g.ep.counters + tile * CG + rank;
                 int r0 = 0, r1 = BN;
                 if (g.coop) {
                     if (threadIdx.x == 64) {
@@ -662,12 +869,19 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CG == 2)
+        cluster_sync();  // no CTA leaves while the other may still signal or read it
+    else
+        __syncthreads();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
-                     : "memory");
+        if constexpr (CG == 2)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                         : "memory");
     }
 }
 
@@ -683,20 +897,58 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-template <int BN, int WT, int BK>
+template <int BN, int WT, int BK, int CG = 1>
 cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, int grid, cudaStream_t st) {
-    using C = PCfg<BN, WT, BK>;
+    using C = PCfg<BN, WT, BK, CG>;
+    auto kern = gemm_tc_kernel<BN, WT, BK, CG>;
     static int attr_dev = -1;
+    static int max_pairs = 0;
     int dev = 0;
     cudaGetDevice(&dev);
     if (attr_dev != dev) {
-        cudaError_t e =
-            cudaFuncSetAttribute(gemm_tc_kernel<BN, WT, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
+        if (CG == 2) {
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(2);
+            q.blockDim = dim3(192);
+            q.dynamicSmemBytes = C::SMEM_BYTES;
+            cudaLaunchAttribute ca[1];
+            ca[0].id = cudaLaunchAttributeClusterDimension;
+            ca[0].val.clusterDim.x = 2;
+            ca[0].val.clusterDim.y = 1;
+            ca[0].val.clusterDim.z = 1;
+            q.attrs = ca;
+            q.numAttrs = 1;
+            e = cudaOccupancyMaxActiveClusters(&max_pairs, kern, &q);
+            if (e != cudaSuccess) return e;
+            if (max_pairs < 1) return cudaErrorInvalidConfiguration;
+        }
         attr_dev = dev;
     }
+    if (CG == 2) {
+        // Pairs run as clusters of two; the schedule strides over clusters, so
+        // any even grid is correct and no more pairs than fit at once are launched.
+        if (a.splits > 1 && a.coop) return cudaErrorInvalidValue;
+        const int pairs = std::max(1, std::min(grid / 2, max_pairs));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * pairs);
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, a);
+    }
     if (!(a.splits > 1 && a.coop))
-        return launch_pdl(gemm_tc_kernel<BN, WT, BK>, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
+        return launch_pdl(kern, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
     // The slices of a tile wait for one another: launch cooperatively so all CTAs
     // are resident at once (the launch fails instead of deadlocking).
     cudaLaunchConfig_t cfg = {};
@@ -709,7 +961,7 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, WT, BK>, tmW, tmX, a);
+    return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, a);
 }
 
 }  // namespace
@@ -717,19 +969,26 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
 namespace {
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
-GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1, int bk = BK_DEFAULT) {
+GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1, int bk = BK_DEFAULT,
+                   int cg = 1) {
     GemmPlan p;
     p.bn = bn;
     p.wt = wt;
     p.bk = bk;
+    p.cg = cg;
     p.m_tiles = (M + bn - 1) / bn;
-    p.n_tiles = (N + BM * wt - 1) / (BM * wt);
+    p.n_tiles = (N + BM * wt * cg - 1) / (BM * wt * cg);
     const int KB = (K + bk - 1) / bk;
     p.kb_per_split = (KB + splits - 1) / splits;
     p.splits = (KB + p.kb_per_split - 1) / p.kb_per_split;
     // Units are dealt in rounds of `grid`; a multiple of the split count keeps
     // the splits of every tile in one round (they wait for each other).
     const long units = (long)p.m_tiles * p.n_tiles * p.splits;
+    if (cg == 2) {  // CTA pairs; the K-split fixup of pairs is the last-arriver one
+        p.coop = 0;
+        p.grid = 2 * (int)std::min<long>(units, std::max(1, num_sms / 2));
+        return p;
+    }
     const int per_round = std::max(p.splits, (num_sms / p.splits) * p.splits);
     p.grid = (int)std::min<long>(units, per_round);
     return p;
@@ -737,23 +996,25 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
 }  // namespace
 
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                        int force_wt, int force_bk, int force_coop) {
-    GemmPlan p = plan_gemm_bf16_shape(M, N, K, num_sms, max_splits, force_bn, force_splits, force_wt, force_bk);
-    p.coop = force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
+                        int force_wt, int force_bk, int force_coop, int force_cg) {
+    GemmPlan p =
+        plan_gemm_bf16_shape(M, N, K, num_sms, max_splits, force_bn, force_splits, force_wt, force_bk, force_cg);
+    p.coop = p.cg == 2 ? 0 : force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
     return p;
 }
 
 GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                              int force_wt, int force_bk) {
+                              int force_wt, int force_bk, int force_cg) {
     const int KB = (K + BK_DEFAULT - 1) / BK_DEFAULT;
     // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
     const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
     if (force_bn > 0 || force_splits > 0) {
         const int bn = force_bn > 0 ? force_bn : bn_for(M);
-        const int wt = (force_wt == 2 && bn >= 128) ? 2 : 1;
-        const int bk = (force_bk == 32 && bn >= 128) ? 32 : BK_DEFAULT;
+        const int cg = (force_cg == 2 && (bn == 128 || bn == 256)) ? 2 : 1;
+        const int wt = (cg == 1 && force_wt == 2 && bn >= 128) ? 2 : 1;
+        const int bk = (cg == 1 && force_bk == 32 && bn >= 128) ? 32 : BK_DEFAULT;
         return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)), wt,
-                         bk);
+                         bk, cg);
     }
     // Cost in units of one 256-column k-block per CTA: rounds x k-block time x
     // (k-blocks per unit + per-unit overhead + the partial plane's round trip
@@ -809,9 +1070,16 @@ bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K, const GemmPlan& p,
                              const EpiParams& ep, cudaStream_t st) {
     if (p.splits > 1 && (!ep.ws || !ep.counters)) return cudaErrorInvalidValue;
-    if (ep.kind == EPI_ENTROPY && (p.splits != 1 || !ep.epart || ep.npart < ((N + 128 * p.wt - 1) / (128 * p.wt)) * p.wt * 4))
+    const int tw = 128 * p.wt * p.cg;
+    if (ep.kind == EPI_ENTROPY && (p.splits != 1 || !ep.epart || ep.npart < ((N + tw - 1) / tw) * p.wt * p.cg * 4))
         return cudaErrorInvalidValue;
     GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, ep};
+    if (p.cg == 2) {
+        if (p.wt != 1 || p.bk != 64) return cudaErrorInvalidValue;
+        if (p.bn == 256) return launch_bn<256, 1, 64, 2>(tmW, tmX, a, p.grid, st);
+        if (p.bn == 128) return launch_bn<128, 1, 64, 2>(tmW, tmX, a, p.grid, st);
+        return cudaErrorInvalidValue;
+    }
     if (p.bk == 32) {
         if (p.wt == 2 && p.bn == 256) return launch_bn<256, 2, 32>(tmW, tmX, a, p.grid, st);
         if (p.wt == 2 && p.bn == 128) return launch_bn<128, 2, 32>(tmW, tmX, a, p.grid, st);

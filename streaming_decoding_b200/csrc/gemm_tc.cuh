@@ -46,12 +46,16 @@ struct EpiParams {
 // How Y[M][N] = X[M][K] * W[N][K]^T is cut: tiles of 128 * wt weight rows
 // (wt MMAs of M = 128 sharing the activation operand) by bn activation rows
 // (MMA N), K in `splits` slices; units = tiles * splits are dealt round-robin
-// to `grid` persistent CTAs (one per SM).  wt = 2 needs bn >= 128.
+// to `grid` persistent CTAs (one per SM).  wt = 2 needs bn >= 128.  With
+// cg = 2 a tile is 256 weight rows computed by a CTA pair (cta_group::2 MMAs,
+// bn = 128 or 256 split between the two CTAs' shared memory), units are dealt
+// to pairs, and `grid` counts CTAs (two per pair).
 struct GemmPlan {
     int bn = 16;
     int wt = 1;
     int bk = 64;       // k-block depth: 64 (128-byte swizzle) or 32 (64-byte swizzle, bn >= 128)
     int coop = 1;      // K-split fixup: 1 the slices wait and share the reduction, 0 the last one reduces
+    int cg = 1;        // 2: CTA pairs (clusters of two) share 256-row weight tiles; coop is then 0
     int splits = 1;
     int kb_per_split = 1;
     int m_tiles = 1;
@@ -63,11 +67,12 @@ struct GemmPlan {
 // force_bn / force_splits > 0 pin the tile width / split count, force_wt = 2
 // selects 256-row weight tiles (tuning hooks).
 // force_coop: 1 / 0 pick the K-split fixup, -1 the default (distributed for
-// M > 128 rows, last arriver otherwise).
+// M > 128 rows, last arriver otherwise).  force_cg = 2 (with force_bn 128 or
+// 256) selects CTA-pair tiles.
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0,
-                        int force_wt = 0, int force_bk = 0, int force_coop = -1);
+                        int force_wt = 0, int force_bk = 0, int force_coop = -1, int force_cg = 1);
 GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                              int force_wt, int force_bk);
+                              int force_wt, int force_bk, int force_cg = 1);
 
 // 2-D bf16 tensor map [rows][cols], boxes of bk columns (64: 128-byte swizzle,
 // 32: 64-byte swizzle) by box_rows rows.
@@ -77,8 +82,8 @@ bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t c
 bool encode_tmap_bf16(CUtensorMap* tm, const void* base, int rank, const cuuint64_t* gdim, const cuuint64_t* gstride,
                       const cuuint32_t* box);
 
-// tmW: weights [N][K], box rows 128; tmX: activations [>=M][K], box rows plan.bn;
-// both with boxes of plan.bk columns.
+// tmW: weights [N][K], box rows 128; tmX: activations [>=M][K], box rows
+// plan.bn / plan.cg; both with boxes of plan.bk columns.
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int M, int N, int K,
                              const GemmPlan& plan, const EpiParams& ep, cudaStream_t st);
 

@@ -63,22 +63,24 @@ wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M
     return wedlm_linear_bf16_plan(X, W, Y, M, N, K, 0, 0, stream);
 }
 
-wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
-                                    int32_t tile_n, int32_t k_splits, void* stream) {
+static wedlm_status linear_bf16(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                int32_t tile_n, int32_t k_splits, int32_t cg, void* stream) {
     if (M < 1 || N < 1 || K < 8 || K % 8 || !X || !W || !Y) return WEDLM_ERR_INVALID_ARG;
     if (tile_n != 0 && tile_n != 16 && tile_n != 32 && tile_n != 64 && tile_n != 128 && tile_n != 256)
         return WEDLM_ERR_INVALID_ARG;
+    if (cg == 2 && tile_n != 128 && tile_n != 256) return WEDLM_ERR_INVALID_ARG;
     if (k_splits < 0 || k_splits > 16) return WEDLM_ERR_INVALID_ARG;
     if (((uintptr_t)X | (uintptr_t)W) & 15) return WEDLM_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    GemmPlan p = plan_gemm_bf16(M, N, K, sms, 16, tile_n, k_splits);
+    GemmPlan p = plan_gemm_bf16(M, N, K, sms, 16, tile_n, k_splits, 0, 0, -1, cg);
+    if (p.cg != (cg == 2 ? 2 : 1)) return WEDLM_ERR_INVALID_ARG;
     CUtensorMap tw, tx;
     if (!make_tmap_bf16(&tw, W, (uint64_t)N, (uint64_t)K, 128)) return WEDLM_ERR_CUDA;
-    if (!make_tmap_bf16(&tx, X, (uint64_t)M, (uint64_t)K, (uint32_t)p.bn)) return WEDLM_ERR_CUDA;
-    const size_t tiles = (size_t)p.m_tiles * p.n_tiles;
+    if (!make_tmap_bf16(&tx, X, (uint64_t)M, (uint64_t)K, (uint32_t)(p.bn / p.cg))) return WEDLM_ERR_CUDA;
+    const size_t tiles = (size_t)p.m_tiles * p.n_tiles * p.cg;
     int* scratch = nullptr;  // error word, then tile tickets
     float* planes = nullptr;
     if (cudaMallocAsync((void**)&scratch, (1 + tiles) * sizeof(int), st) != cudaSuccess) return WEDLM_ERR_OOM_DEVICE;
@@ -105,6 +107,16 @@ wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int3
     if (herr == kErrTimeout) return WEDLM_ERR_TIMEOUT;
     if (herr) return WEDLM_ERR_DEVICE_ASSERT;
     return WEDLM_OK;
+}
+
+wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                    int32_t tile_n, int32_t k_splits, void* stream) {
+    return linear_bf16(X, W, Y, M, N, K, tile_n, k_splits, 1, stream);
+}
+
+wedlm_status wedlm_linear_bf16_pair(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                    int32_t tile_n, int32_t k_splits, void* stream) {
+    return linear_bf16(X, W, Y, M, N, K, tile_n, k_splits, 2, stream);
 }
 
 }  // extern "C"

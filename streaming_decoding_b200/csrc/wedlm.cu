@@ -16,7 +16,9 @@
 // kernel needs per step lives in device memory, so a step is replayable
 // without host involvement.
 #include <algorithm>
+#include <climits>
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <deque>
@@ -280,16 +282,18 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
         if ((size_t)M * N > ctx->logits_floats) return;
         ep.out = ctx->logits;
     }
-    // (activation rows per tile, 128-row weight sub-tiles per tile, k-block depth)
+    // (activation rows per tile, 128-row weight sub-tiles per tile, k-block
+    // depth, CTAs per tile: 2 = CTA-pair tiles of 256 weight rows)
     struct Shape {
-        int bn, wt, bk;
+        int bn, wt, bk, cg;
     };
     std::vector<Shape> shapes;
     if (M > 128)
-        shapes = {{256, 1, 64}, {128, 1, 64}, {64, 1, 64}, {256, 2, 64}, {128, 2, 64}, {256, 2, 32}, {128, 2, 32},
-                  {256, 1, 32}};
-    else if (M > 64) shapes = {{128, 1, 64}, {64, 1, 64}, {128, 2, 64}, {128, 2, 32}};
-    else shapes = {{M <= 16 ? 16 : M <= 32 ? 32 : 64, 1, 64}};
+        shapes = {{256, 1, 64, 2}, {128, 1, 64, 2}, {256, 1, 64, 1}, {128, 1, 64, 1}, {64, 1, 64, 1},
+                  {256, 2, 64, 1}, {128, 2, 64, 1}, {256, 2, 32, 1}, {128, 2, 32, 1}, {256, 1, 32, 1}};
+    else if (M > 64)
+        shapes = {{128, 1, 64, 2}, {128, 1, 64, 1}, {64, 1, 64, 1}, {128, 2, 64, 1}, {128, 2, 32, 1}};
+    else shapes = {{M <= 16 ? 16 : M <= 32 ? 32 : 64, 1, 64, 1}};
     cudaEvent_t e0 = prof_event(ctx), e1 = prof_event(ctx);
     float best = 1e30f;
     GemmPlan bestp = ctx->tuned[key].plan;
@@ -299,18 +303,25 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
     const int KB = (K + 63) / 64;
     for (const Shape& sh : shapes) {
         for (int spc : {1, 2, -2, 3, -3, 4, -4, 6, -6, 8, -8, 12, -12, 16, -16}) {
-            // negative: the same split count with the last-arriver fixup
+            // negative: the same split count with the last-arriver fixup (the
+            // only one CTA pairs use)
             const int sp = spc < 0 ? -spc : spc;
-            if (sp > KB || (sp > 1 && N % 4)) continue;
-            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, sh.bn, sp, sh.wt, sh.bk, spc < 0 ? 0 : 1);
-            if (p.splits != sp) continue;
+            if (sp > KB || (sp > 1 && N % 4) || (sh.cg == 2 && spc > 1)) continue;
+            GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, sh.bn, sp, sh.wt, sh.bk, spc < 0 ? 0 : 1, sh.cg);
+            if (p.splits != sp || p.cg != sh.cg) continue;
             if (p.splits > 1 && ((size_t)p.splits * M * N > ctx->ws_floats ||
-                                 (size_t)p.m_tiles * p.n_tiles > ctx->n_tile_counters))
+                                 (size_t)p.m_tiles * p.n_tiles * p.cg > ctx->n_tile_counters))
                 continue;
-            const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn, p.bk);
+            const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)(p.bn / p.cg), p.bk);
             if (!tx) continue;
             float t = 1e30f;
-            for (int rep = 0; rep < 4; ++rep) {
+            for (int rep = 0; rep < 5; ++rep) {
+                // In a step every projection's weights arrive cold from HBM (the
+                // other layers' weights stream through L2 in between): rewrite the
+                // logits scratch (larger than L2 at full size; not live while the
+                // projections run) so the weights of the previous repetition are
+                // evicted.
+                cudaMemsetAsync(ctx->logits, 0, ctx->logits_floats * sizeof(float), ctx->stream);
                 cudaEventRecord(e0, ctx->stream);
                 if (launch_gemm_bf16(tmW->of(p.bk), *tx, M, N, K, p, ep, ctx->stream) != cudaSuccess) {
                     cudaGetLastError();
@@ -348,11 +359,11 @@ wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx:
         p = plan_gemm_bf16(M, N, K, ctx->num_sms, cap);
     }
     if (ep.kind == EPI_ENTROPY && p.splits != 1)  // the entropy epilogue needs whole K sums
-        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk);
-    if (p.splits > 1 && ((size_t)p.n_tiles * p.m_tiles > ctx->n_tile_counters ||
+        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk, -1, p.cg);
+    if (p.splits > 1 && ((size_t)p.n_tiles * p.m_tiles * p.cg > ctx->n_tile_counters ||
                          (size_t)p.splits * M * N > ctx->ws_floats))
-        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk);
-    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)p.bn, p.bk);
+        p = plan_gemm_bf16(M, N, K, ctx->num_sms, 1, p.bn, 1, p.wt, p.bk, -1, p.cg);
+    const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)(p.bn / p.cg), p.bk);
     if (!tx) return fail(ctx, WEDLM_ERR_CUDA, "cuTensorMapEncodeTiled failed for activations");
     ep.ws = ctx->ws;
     ep.counters = ctx->tile_counters;
@@ -373,7 +384,8 @@ void gemm_needs(const wedlm_ctx* c, int M, int N, int K, int max_splits, size_t*
     const int sp = std::min(max_splits, KB);
     if (sp > 1 && N % 4 == 0) *ws = std::max(*ws, (size_t)sp * M * N);
     const int bn_min = M > 128 ? 128 : 16;
-    *tiles = std::max(*tiles, (size_t)((M + bn_min - 1) / bn_min) * ((N + 127) / 128));
+    // tickets: one per 128-row weight tile, or two per CTA-pair tile of 256 rows
+    *tiles = std::max(*tiles, (size_t)((M + bn_min - 1) / bn_min) * (2 * ((N + 255) / 256)));
 }
 
 wedlm_status build_weight_maps(wedlm_ctx* ctx) {
@@ -957,6 +969,18 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         return bail(WEDLM_ERR_CUDA);
 
     launch_rope_table(ctx->rope_cs, ctx->max_ctx, ctx->hd / 2, ctx->hd, cfg->rope_theta, ctx->stream);
+    if (ctx->lm_part) {
+        // Partial i always covers vocab ids [32 i, 32 i + 32) whatever the tile
+        // shape; those past the vocabulary, which a narrow-tile plan never
+        // writes, must read as empty (max -inf, sums 0, no argmax).
+        const int32_t no_id = INT32_MAX;
+        float no_id_bits;
+        std::memcpy(&no_id_bits, &no_id, 4);
+        const float4 empty = make_float4(-INFINITY, 0.f, 0.f, no_id_bits);
+        std::vector<float4> fill((size_t)ctx->Mdec * ctx->lm_npart, empty);
+        if (cudaMemcpy(ctx->lm_part, fill.data(), fill.size() * sizeof(float4), cudaMemcpyHostToDevice) != cudaSuccess)
+            return bail(WEDLM_ERR_CUDA);
+    }
     std::vector<int32_t> pt((size_t)B * ctx->pages_per_seq, -1);
     if (cudaMemcpy(ss.page_table, pt.data(), pt.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return bail(WEDLM_ERR_CUDA);
@@ -1294,7 +1318,7 @@ wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t
     if (!ctx) return WEDLM_ERR_INVALID_ARG;
     auto it = ctx->tuned.find({kind, rows});
     if (it == ctx->tuned.end()) return fail(ctx, WEDLM_ERR_STATE, "no plan recorded for this kind and row count");
-    if (tile_w) *tile_w = 128 * it->second.plan.wt;
+    if (tile_w) *tile_w = 128 * it->second.plan.wt * it->second.plan.cg;
     if (tile_n) *tile_n = it->second.plan.bn;
     if (k_splits) *k_splits = it->second.plan.splits;
     if (us) *us = it->second.us;

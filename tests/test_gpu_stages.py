@@ -106,3 +106,31 @@ def test_linear_bf16_matches_fp64_matmul(M, N, K):
     bound = np.abs(synth.bf16_bits_to_f32(X)).astype(np.float64) @ np.abs(synth.bf16_bits_to_f32(W)).astype(np.float64).T
     err = np.abs(Y - ref)
     assert np.all(err <= 1e-4 * bound + 1e-30), float((err / (bound + 1e-30)).max())
+
+
+@pytest.mark.parametrize("M,N,K,tile_n,k_splits", [
+    (256, 6144, 4096, 256, 1),    # QKV-shaped, whole pair tiles
+    (256, 4096, 4096, 256, 3),    # K in slices (last-arriver reduction)
+    (200, 1152, 520, 256, 1),     # ragged rows, a half-empty pair tile (N % 256 = 128), ragged K
+    (256, 1000, 4096, 128, 2),    # two activation tiles per pair tile, ragged N
+    (96, 2048, 1024, 128, 1),     # fewer rows than the tile: the odd CTA's half is padding
+    (512, 768, 256, 256, 1),      # several activation tiles
+])
+def test_linear_bf16_cta_pair_matches_fp64_matmul(M, N, K, tile_n, k_splits):
+    """CTA-pair tiles (two-CTA tensor-core MMA, operands split across the pair's
+    shared memory) against the same fp64 matmul and bound as above."""
+    from streaming_decoding_b200 import linear_bf16
+    X = synth.normal(33, M * 5 + K, 1.0, (M, K), "bf16")
+    W = synth.normal(34, N * 11 + K, 0.02, (N, K), "bf16")
+    Xt = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+    Wt = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=k_splits, cta_pair=True).cpu().numpy().astype(np.float64)
+    x64 = synth.bf16_bits_to_f32(X).astype(np.float64)
+    w64 = synth.bf16_bits_to_f32(W).astype(np.float64)
+    ref = x64 @ w64.T
+    bound = np.abs(x64) @ np.abs(w64).T
+    err = np.abs(Y - ref)
+    assert np.all(err <= 1e-4 * bound + 1e-30), float((err / (bound + 1e-30)).max())
+    # the same plan without pairs agrees to accumulation order
+    Y1 = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=k_splits).cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(Y - Y1) <= 2e-4 * bound + 1e-30)
