@@ -306,13 +306,23 @@ __device__ __forceinline__ void fill_row_meta(const EpiParams& ep, int m0, int M
     }
 }
 
-// Destination of dim `dim` of QKV head `head` for a row (q buffer or pages).
-__device__ __forceinline__ bf16* qkv_dst(const EpiParams& ep, int head, int m, const RowMeta& rm) {
-    if (head < ep.hq) return ep.act + ((int64_t)m * ep.hq + head) * 128;
-    if (rm.kv < 0) return nullptr;
-    const int kv = head < ep.hq + ep.hkv ? 0 : 1;
-    const int h = head - ep.hq - kv * ep.hkv;
-    return ep.kv_pool + rm.kv + (int64_t)(kv * ep.hkv + h) * (kPage * 128);
+// silu(x) * y for the gate/up pair, with the exponential and the division on
+// the special-function unit (no branch: independent elements interleave); its
+// error, about 1e-6 relative, is far below the bf16 rounding of the result.
+__device__ __forceinline__ float silu_mul(float x, float y) { return __fdividef(x, 1.0f + __expf(-x)) * y; }
+
+// Destination row of QKV head `head` for activation row m: the q buffer, or the
+// row's K or V page entry (kv: the row's cache offset, -1 if it has none).
+// Every argument is a register value: the epilogues read all parameters and row
+// metadata before their first global store, since after a store through a
+// generic pointer the compiler would have to reload anything it cannot prove
+// unaliased, which serialises the element loop on load latency.
+__device__ __forceinline__ bf16* qkv_dst(bf16* act, bf16* pool, int hq, int hkv, int head, int m, long long kv) {
+    if (head < hq) return act + ((int64_t)m * hq + head) * 128;
+    if (kv < 0) return nullptr;
+    const int sel = head < hq + hkv ? 0 : 1;
+    const int h = head - hq - sel * hkv;
+    return pool + kv + (int64_t)(sel * hkv + h) * (kPage * 128);
 }
 
 // Fused epilogue on 16 accumulator columns (activation rows mbase..mbase+15,
@@ -320,57 +330,66 @@ __device__ __forceinline__ bf16* qkv_dst(const EpiParams& ep, int head, int m, c
 // (n even, n odd) sit in adjacent lanes.
 __device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, int mbase, int kbase,
                                            const RowMeta* meta, const float (&v)[16], int N, int lane) {
-    int live[16];
+    const int kind = ep.kind;
+    float* const out = ep.out;
+    bf16* const act = ep.act;
+    bool live[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) live[k] = meta[kbase + k].live && n < N;
-    switch (ep.kind) {
+    switch (kind) {
         case EPI_STORE:
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-                if (live[k]) ep.out[(int64_t)(mbase + k) * N + n] = v[k];
+                if (live[k]) out[(int64_t)(mbase + k) * N + n] = v[k];
             break;
         case EPI_RESIDUAL: {
             float x[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) x[k] = live[k] ? ep.out[(int64_t)(mbase + k) * N + n] : 0.f;
+            for (int k = 0; k < 16; ++k) x[k] = live[k] ? out[(int64_t)(mbase + k) * N + n] : 0.f;
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-                if (live[k]) ep.out[(int64_t)(mbase + k) * N + n] = x[k] + v[k];
+                if (live[k]) out[(int64_t)(mbase + k) * N + n] = x[k] + v[k];
             break;
         }
         case EPI_SWIGLU: {
             const int F = N >> 1;
+            bf16 r[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float partner = __shfl_xor_sync(0xffffffffu, v[k], 1);
-                if (!(lane & 1) && live[k])
-                    ep.act[(int64_t)(mbase + k) * F + (n >> 1)] =
-                        __float2bfloat16_rn(v[k] / (1.0f + expf(-v[k])) * partner);
+                r[k] = __float2bfloat16_rn(silu_mul(v[k], partner));
             }
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if (!(lane & 1) && live[k]) act[(int64_t)(mbase + k) * F + (n >> 1)] = r[k];
             break;
         }
         case EPI_QKV_ROPE: {
+            bf16* const pool = ep.kv_pool;
+            const float2* const rope = ep.rope_cs;
+            const int hq = ep.hq, hkv = ep.hkv;
             const int head = n0 >> 7;
             const int t = n - n0;
-            const bool rot = head < ep.hq + ep.hkv;
+            const bool rot = head < hq + hkv;
             const int i = t >> 1, odd = t & 1;
             const int dim = rot ? (odd ? i + 64 : i) : t;
             float2 cs[16];
+            bf16* dst[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                cs[k] = (rot && live[k]) ? __ldg(ep.rope_cs + (int64_t)meta[kbase + k].pos * 64 + i)
-                                         : make_float2(1.f, 0.f);
+            for (int k = 0; k < 16; ++k) {
+                const RowMeta rmk = meta[kbase + k];
+                cs[k] = (rot && live[k]) ? __ldg(rope + (int64_t)rmk.pos * 64 + i) : make_float2(1.f, 0.f);
+                dst[k] = live[k] ? qkv_dst(act, pool, hq, hkv, head, mbase + k, rmk.kv) : nullptr;
+            }
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const float partner = rot ? __shfl_xor_sync(0xffffffffu, v[k], 1) : 0.f;
-                if (!live[k]) continue;
                 float val = v[k];
                 if (rot) {
                     const float a = odd ? partner : val, b = odd ? val : partner;
                     val = odd ? (b * cs[k].x + a * cs[k].y) : (a * cs[k].x - b * cs[k].y);
                 }
-                bf16* dst = qkv_dst(ep, head, mbase + k, meta[kbase + k]);
-                if (dst) dst[dim] = __float2bfloat16_rn(val);
+                if (dst[k]) dst[k][dim] = __float2bfloat16_rn(val);
             }
             break;
         }
@@ -384,9 +403,12 @@ __device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, i
 // over valid ids (n < N, n != mask id); lane k stores row k's partial.
 __device__ __forceinline__ void entropy16(const EpiParams& ep, const float (&v)[16], bool valid, int n, int mbase,
                                           int M, int pidx, int lane) {
+    const float scale = ep.scale;
+    float4* const epart = ep.epart;
+    const int npart = ep.npart;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-        const float z = valid ? v[k] * ep.scale : -INFINITY;
+        const float z = valid ? v[k] * scale : -INFINITY;
         float m = z;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -404,82 +426,173 @@ __device__ __forceinline__ void entropy16(const EpiParams& ep, const float (&v)[
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
         const int row = mbase + k;
-        if (lane == k && row < M) ep.epart[(int64_t)row * ep.npart + pidx] = make_float4(m, e, t, __int_as_float(a));
+        if (lane == k && row < M) epart[(int64_t)row * npart + pidx] = make_float4(m, e, t, __int_as_float(a));
     }
 }
 
 // Fused epilogue on weight rows n..n+3 (both row pairs inside this thread) of
-// eight activation rows m = mrow[u], after a split-K reduction.
+// eight activation rows m = mrow[u] (meta rows krow[u]), in two phases: epi_pre
+// issues every load that does not depend on the accumulator (row metadata, the
+// residual stream, RoPE cos/sin, destination rows) so its latency overlaps the
+// staging of the accumulator; epi_fin does the arithmetic and the vector stores.
+// All parameter reads precede the first store (see qkv_dst).
+struct EpiPre {
+    bool live[8];
+    float4 x[8];          // EPI_RESIDUAL: residual stream values
+    float2 c0[8], c1[8];  // EPI_QKV_ROPE: (cos, sin) of dims (i, i + 64) and (i + 1, i + 65)
+    bf16* dst[8];         // EPI_QKV_ROPE: destination rows
+};
+
+template <int KIND>
+__device__ __forceinline__ void epi_pre(const EpiParams& ep, int n0, int n, const int (&mrow)[8], const int (&krow)[8],
+                                        const bool (&ok)[8], const RowMeta* meta, int N, EpiPre& p) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) p.live[u] = ok[u] && meta[krow[u]].live;
+    if constexpr (KIND == EPI_RESIDUAL) {
+        const float* out = ep.out;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            p.x[u] = p.live[u] ? *reinterpret_cast<const float4*>(out + (int64_t)mrow[u] * N + n)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if constexpr (KIND == EPI_QKV_ROPE) {
+        bf16* const act = ep.act;
+        bf16* const pool = ep.kv_pool;
+        const float2* const rope = ep.rope_cs;
+        const int hq = ep.hq, hkv = ep.hkv;
+        const int head = n0 >> 7;
+        const bool rot = head < hq + hkv;
+        const int i = (n - n0) >> 1;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const RowMeta rmu = meta[krow[u]];
+            const int64_t base = (int64_t)rmu.pos * 64 + i;
+            p.c0[u] = (rot && p.live[u]) ? __ldg(rope + base) : make_float2(1.f, 0.f);
+            p.c1[u] = (rot && p.live[u]) ? __ldg(rope + base + 1) : make_float2(1.f, 0.f);
+            p.dst[u] = p.live[u] ? qkv_dst(act, pool, hq, hkv, head, mrow[u], rmu.kv) : nullptr;
+        }
+    }
+}
+
+template <int KIND>
+__device__ __forceinline__ void epi_fin(const EpiParams& ep, int n0, int n, const int (&mrow)[8], const float4 (&v)[8],
+                                        const EpiPre& p, int N) {
+    if constexpr (KIND == EPI_STORE) {
+        float* const out = ep.out;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (p.live[u]) *reinterpret_cast<float4*>(out + (int64_t)mrow[u] * N + n) = v[u];
+    } else if constexpr (KIND == EPI_RESIDUAL) {
+        float* const out = ep.out;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (p.live[u])
+                *reinterpret_cast<float4*>(out + (int64_t)mrow[u] * N + n) =
+                    make_float4(p.x[u].x + v[u].x, p.x[u].y + v[u].y, p.x[u].z + v[u].z, p.x[u].w + v[u].w);
+    } else if constexpr (KIND == EPI_SWIGLU) {
+        bf16* const act = ep.act;
+        const int F = N >> 1;
+        __nv_bfloat162 r[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) r[u] = __floats2bfloat162_rn(silu_mul(v[u].x, v[u].y), silu_mul(v[u].z, v[u].w));
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (p.live[u]) *reinterpret_cast<__nv_bfloat162*>(act + (int64_t)mrow[u] * F + (n >> 1)) = r[u];
+    } else if constexpr (KIND == EPI_QKV_ROPE) {
+        const int head = n0 >> 7;
+        const int t = n - n0;
+        const bool rot = head < ep.hq + ep.hkv;
+        const int i = t >> 1;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            bf16* const d = p.dst[u];
+            if (!d) continue;
+            if (rot) {
+                // rows (t, t+1) = dims (i, i+64); rows (t+2, t+3) = dims (i+1, i+65)
+                const float d0 = v[u].x * p.c0[u].x - v[u].y * p.c0[u].y;
+                const float d2 = v[u].y * p.c0[u].x + v[u].x * p.c0[u].y;
+                const float d1 = v[u].z * p.c1[u].x - v[u].w * p.c1[u].y;
+                const float d3 = v[u].w * p.c1[u].x + v[u].z * p.c1[u].y;
+                *reinterpret_cast<__nv_bfloat162*>(d + i) = __floats2bfloat162_rn(d0, d1);
+                *reinterpret_cast<__nv_bfloat162*>(d + i + 64) = __floats2bfloat162_rn(d2, d3);
+            } else {
+                *reinterpret_cast<__nv_bfloat162*>(d + t) = __floats2bfloat162_rn(v[u].x, v[u].y);
+                *reinterpret_cast<__nv_bfloat162*>(d + t + 2) = __floats2bfloat162_rn(v[u].z, v[u].w);
+            }
+        }
+    }
+}
+
+// Both phases back to back, dispatched on the epilogue kind at run time.
 __device__ __forceinline__ void epilogue_vec4x8(const EpiParams& ep, int n0, int n, const int (&mrow)[8],
                                                 const int (&krow)[8], const bool (&ok)[8], const RowMeta* meta,
                                                 const float4 (&v)[8], int N) {
-    bool live[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) live[u] = ok[u] && meta[krow[u]].live;
+    EpiPre p;
     switch (ep.kind) {
         case EPI_STORE:
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (live[u]) *reinterpret_cast<float4*>(ep.out + (int64_t)mrow[u] * N + n) = v[u];
+            epi_pre<EPI_STORE>(ep, n0, n, mrow, krow, ok, meta, N, p);
+            epi_fin<EPI_STORE>(ep, n0, n, mrow, v, p, N);
             break;
-        case EPI_RESIDUAL: {
-            float4 x[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                x[u] = live[u] ? *reinterpret_cast<const float4*>(ep.out + (int64_t)mrow[u] * N + n)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (live[u])
-                    *reinterpret_cast<float4*>(ep.out + (int64_t)mrow[u] * N + n) =
-                        make_float4(x[u].x + v[u].x, x[u].y + v[u].y, x[u].z + v[u].z, x[u].w + v[u].w);
+        case EPI_RESIDUAL:
+            epi_pre<EPI_RESIDUAL>(ep, n0, n, mrow, krow, ok, meta, N, p);
+            epi_fin<EPI_RESIDUAL>(ep, n0, n, mrow, v, p, N);
             break;
-        }
-        case EPI_SWIGLU: {
-            const int F = N >> 1;
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (live[u]) {
-                    const float a = v[u].x / (1.0f + expf(-v[u].x)) * v[u].y;
-                    const float b = v[u].z / (1.0f + expf(-v[u].z)) * v[u].w;
-                    *reinterpret_cast<__nv_bfloat162*>(ep.act + (int64_t)mrow[u] * F + (n >> 1)) =
-                        __floats2bfloat162_rn(a, b);
-                }
+        case EPI_SWIGLU:
+            epi_pre<EPI_SWIGLU>(ep, n0, n, mrow, krow, ok, meta, N, p);
+            epi_fin<EPI_SWIGLU>(ep, n0, n, mrow, v, p, N);
             break;
-        }
-        case EPI_QKV_ROPE: {
-            const int head = n0 >> 7;
-            const int t = n - n0;
-            const bool rot = head < ep.hq + ep.hkv;
-            const int i = t >> 1;
-            float2 c0[8], c1[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int64_t base = (int64_t)meta[krow[u]].pos * 64 + i;
-                c0[u] = (rot && live[u]) ? __ldg(ep.rope_cs + base) : make_float2(1.f, 0.f);
-                c1[u] = (rot && live[u]) ? __ldg(ep.rope_cs + base + 1) : make_float2(1.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                if (!live[u]) continue;
-                bf16* dst = qkv_dst(ep, head, mrow[u], meta[krow[u]]);
-                if (!dst) continue;
-                if (rot) {
-                    // rows (t, t+1) = dims (i, i+64); rows (t+2, t+3) = dims (i+1, i+65)
-                    const float d0 = v[u].x * c0[u].x - v[u].y * c0[u].y;
-                    const float d2 = v[u].y * c0[u].x + v[u].x * c0[u].y;
-                    const float d1 = v[u].z * c1[u].x - v[u].w * c1[u].y;
-                    const float d3 = v[u].w * c1[u].x + v[u].z * c1[u].y;
-                    *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(d0, d1);
-                    *reinterpret_cast<__nv_bfloat162*>(dst + i + 64) = __floats2bfloat162_rn(d2, d3);
-                } else {
-                    *reinterpret_cast<__nv_bfloat162*>(dst + t) = __floats2bfloat162_rn(v[u].x, v[u].y);
-                    *reinterpret_cast<__nv_bfloat162*>(dst + t + 2) = __floats2bfloat162_rn(v[u].z, v[u].w);
-                }
-            }
+        case EPI_QKV_ROPE:
+            epi_pre<EPI_QKV_ROPE>(ep, n0, n, mrow, krow, ok, meta, N, p);
+            epi_fin<EPI_QKV_ROPE>(ep, n0, n, mrow, v, p, N);
             break;
-        }
         default: break;
+    }
+}
+
+// Single-slice epilogue through shared memory, for one epilogue kind: 32
+// accumulator columns (activation rows) at a time are stored transposed to
+// `stage` (row = activation row, 128 weight rows; each store instruction writes
+// 32 consecutive words), then each thread finishes float4 runs of weight rows
+// for 8 activation rows: coalesced rows and vector stores.  `release` is called
+// once, right after the last accumulator load.
+template <int KIND, int BN, int WT, typename Release>
+__device__ __forceinline__ void staged_epilogue(const EpiParams& ep, int M, int N, int n0, int m0, uint32_t tacc,
+                                                float* stage, const RowMeta* meta, int q, int lane,
+                                                Release release) {
+    constexpr int COLS = 32;
+    const int c4 = 4 * lane;
+#pragma unroll 1
+    for (int w = 0; w < WT; ++w) {
+        const int nw = n0 + w * BM, nn = nw + c4;
+        const bool nok = nn < N;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += COLS) {
+            int mrow[8], krow[8];
+            bool okr[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int rl = q + 4 * u;  // row within the staged columns
+                krow[u] = c + rl;
+                mrow[u] = m0 + c + rl;
+                okr[u] = nok && mrow[u] < M;
+            }
+            EpiPre p;
+            epi_pre<KIND>(ep, nw, nn, mrow, krow, okr, meta, N, p);
+            {
+                float v[COLS];
+                tmem_ld32(tacc + (uint32_t)(w * BN + c), v);
+                if (w == WT - 1 && c + COLS >= BN) release();
+                float* srow = stage + q * 32 + lane;
+#pragma unroll
+                for (int k = 0; k < COLS; ++k) srow[k * BM] = v[k];
+            }
+            epi_bar();
+            float4 acc[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc[u] = *reinterpret_cast<const float4*>(stage + (q + 4 * u) * BM + c4);
+            epi_fin<KIND>(ep, nw, nn, mrow, acc, p, N);
+            epi_bar();
+        }
     }
 }
 
@@ -693,54 +806,29 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 __syncwarp();
                 if (lane == 0) release(b);
             } else if (g.splits == 1 && BN >= C::EPI_COLS && (g.N & 3) == 0) {
-                // Through shared memory: 32 accumulator columns at a time are
-                // stored transposed (row = activation row, 128 weight rows; each
-                // store instruction writes 32 consecutive words), then each thread
-                // runs the fused epilogue on float4 runs of weight rows for 8
-                // activation rows: coalesced rows, vector stores, few instructions.
-                const int et = threadIdx.x - 64;
-                const int c4 = 4 * (et & 31);
-                bool released = false;
-#pragma unroll 1
-                for (int w = 0; w < WT; ++w) {
-                    const int nw = n0 + w * BM, nn = nw + c4;
-                    const bool nok = nn < g.N;
-#pragma unroll 1
-                    for (int c = 0; c < BN; c += C::EPI_COLS) {
-                        {
-                            float v[C::EPI_COLS];
-                            tmem_ld32(tacc + (uint32_t)(w * BN + c), v);
-                            if (w == WT - 1 && c + C::EPI_COLS >= BN) {
-                                // the accumulator is fully read: the next unit's MMAs may start
-                                tc_fence_before();
-                                __syncwarp();
-                                if (lane == 0) release(b);
-                                released = true;
-                            }
-                            float* srow = epi_stage + q * 32 + lane;
-#pragma unroll
-                            for (int k = 0; k < C::EPI_COLS; ++k) srow[k * BM] = v[k];
-                        }
-                        epi_bar();
-                        float4 acc[8];
-                        int mrow[8], krow[8];
-                        bool okr[8];
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const int rl = q + 4 * u;  // row within the staged columns
-                            krow[u] = c + rl;
-                            mrow[u] = m0 + c + rl;
-                            okr[u] = nok && mrow[u] < g.M;
-                            acc[u] = *reinterpret_cast<const float4*>(epi_stage + rl * BM + c4);
-                        }
-                        epilogue_vec4x8(g.ep, nw, nn, mrow, krow, okr, meta, acc, g.N);
-                        epi_bar();
-                    }
-                }
-                if (!released) {
+                // the accumulator is fully read once the last chunk is loaded: the
+                // next unit's MMAs may start while the stores finish
+                auto rel = [&]() {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) release(b);
+                };
+                switch (g.ep.kind) {
+                    case EPI_STORE:
+                        staged_epilogue<EPI_STORE, BN, WT>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, meta, q, lane, rel);
+                        break;
+                    case EPI_RESIDUAL:
+                        staged_epilogue<EPI_RESIDUAL, BN, WT>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, meta, q, lane,
+                                                              rel);
+                        break;
+                    case EPI_SWIGLU:
+                        staged_epilogue<EPI_SWIGLU, BN, WT>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, meta, q, lane, rel);
+                        break;
+                    case EPI_QKV_ROPE:
+                        staged_epilogue<EPI_QKV_ROPE, BN, WT>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, meta, q, lane,
+                                                              rel);
+                        break;
+                    default: rel(); break;
                 }
             } else if (g.splits == 1) {
 #pragma unroll 1
