@@ -501,53 +501,11 @@ def attention_case(steps: int = 3):
                       "prefill_attention_launches": cfg["B"] * 2}))
 
 
-def gemm_sweep():
-    """Time every projection shape of the batch-16 and batch-1 steps under each
-    (tile width, K split) choice and under the automatic plan (CUDA events)."""
-    import torch
-    from streaming_decoding_b200 import linear_bf16
-    cfg = synth.CONFIGS["qwen3_8b_b16"]
-    dims = cfg["model"]
-    g = torch.Generator(device="cuda").manual_seed(0)
-    out = []
-    for M in (256, 16):
-        X = torch.randn(M, max(dims["F"], dims["d"]), device="cuda", generator=g).to(torch.bfloat16)
-        for name, (_, _, N, K) in gemm_shapes(dims, M).items():
-            W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
-            Xk = X[:, :K].contiguous()
-            shapes = [(0, False)] + ([(256, False), (128, False), (256, True), (128, True)] if M > 128
-                                     else [(16, False)])
-            res = []
-            for bn, pair in shapes:
-                for sp in ([0] if bn == 0 else [1, 2, 3, 4, 6, 8]):
-                    for _ in range(2):
-                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp, cta_pair=pair)
-                    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    st.record()
-                    for _ in range(10):
-                        linear_bf16(Xk, W, tile_n=bn, k_splits=sp, cta_pair=pair)
-                    en.record()
-                    en.synchronize()
-                    us = st.elapsed_time(en) * 100.0
-                    res.append({"bn": bn, "pair": pair, "splits": sp, "us": round(us, 2),
-                                "weight_GBps": round(2 * N * K / us / 1e3, 1),
-                                "TFLOPs": round(2 * M * N * K / us / 1e6, 1)})
-            del W
-            best = min(res[1:], key=lambda r: r["us"])
-            out.append({"M": M, "gemm": name, "N": N, "K": K, "auto": res[0], "best": best, "all": res})
-            print(json.dumps({"M": M, "gemm": name, "auto_us": res[0]["us"], "best": best}), flush=True)
-    with open(os.path.join(ROOT, "gpurun_out", "gemm_sweep.json") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else os.devnull, "w") as f:
-        json.dump(out, f, indent=1)
-
-
 def kernel_case(name: str):
     import torch
     from streaming_decoding_b200 import linear_bf16
     if name == "attention":
         return attention_case()
-    if name == "gemm_sweep":
-        return gemm_sweep()
     cfg = synth.CONFIGS["qwen3_8b_b16"]
     dims = cfg["model"]
     L, M, N, K = gemm_shapes(dims, cfg["B"] * cfg["W"])[name]

@@ -387,13 +387,18 @@ wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M
 wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
                                     int32_t tile_n, int32_t k_splits, void* stream);
 
-/* wedlm_linear_bf16_plan on CTA-pair tiles: two CTAs of a cluster compute a
- * tile of 256 weight rows by tile_n activation rows with the two-CTA tensor-core
- * MMA, each staging its own 128 weight rows and half of the activation rows.
- * tile_n must be 128 or 256 (WEDLM_ERR_INVALID_ARG otherwise); k_splits as
- * above (slices reduced by the last one to finish). */
-wedlm_status wedlm_linear_bf16_pair(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
-                                    int32_t tile_n, int32_t k_splits, void* stream);
+/* wedlm_linear_bf16_plan with the schedule pinned as well; `schedule` is a bit
+ * set (other bits: WEDLM_ERR_INVALID_ARG):
+ *   1  CTA-pair tiles: two CTAs of a cluster compute a tile of 256 weight rows
+ *      by tile_n activation rows with the two-CTA tensor-core MMA, each staging
+ *      its own 128 weight rows and half of the activation rows; tile_n must be
+ *      128 or 256 (WEDLM_ERR_INVALID_ARG otherwise);
+ *   2  hybrid K split: the tiles that fill whole rounds of the persistent grid
+ *      run over all of K, only the tiles of the last partial round are cut into
+ *      k_splits slices (k_splits > 1), reduced by the slice that finishes last.
+ * Results agree with wedlm_linear_bf16 to fp32 accumulation order. */
+wedlm_status wedlm_linear_bf16_sched(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
+                                     int32_t tile_n, int32_t k_splits, int32_t schedule, void* stream);
 
 #ifdef __cplusplus
 }

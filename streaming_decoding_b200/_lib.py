@@ -82,7 +82,7 @@ _SIGS = {
                                              ctypes.POINTER(StepParams), c_vp, c_vp, c_vp, c_vp]),
     "wedlm_linear_bf16": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp]),
     "wedlm_linear_bf16_plan": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]),
-    "wedlm_linear_bf16_pair": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]),
+    "wedlm_linear_bf16_sched": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]),
 }
 
 _lib = None

@@ -85,9 +85,33 @@ struct RowMeta {
 
 struct GemmArgs {
     int M, N, K, kb_per_split, splits, n_tiles, m_tiles;
-    int coop;  // split fixup: 1 distributed (cooperative launch), 0 last arriver
+    int coop;        // split fixup: 1 distributed (cooperative launch), 0 last arriver
+    int full_tiles;  // tiles [0, full_tiles) run whole-K as one unit each; the rest in `splits` K slices
     EpiParams ep;
 };
+
+// One work unit: a tile (n-major over m tiles) and a K slice of it.
+struct Unit {
+    int tile, split, nsplit, kb0, nkb;
+};
+__device__ __forceinline__ Unit unit_of(const GemmArgs& g, int u, int KB) {
+    Unit r;
+    if (u < g.full_tiles) {
+        r.tile = u;
+        r.split = 0;
+        r.nsplit = 1;
+        r.kb0 = 0;
+        r.nkb = KB;
+    } else {
+        const int v = u - g.full_tiles;
+        r.tile = g.full_tiles + v / g.splits;
+        r.split = v % g.splits;
+        r.nsplit = g.splits;
+        r.kb0 = r.split * g.kb_per_split;
+        r.nkb = min(KB, r.kb0 + g.kb_per_split) - r.kb0;
+    }
+    return r;
+}
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -619,7 +643,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = (g.K + BK - 1) / BK;
-    const int units = g.n_tiles * g.m_tiles * g.splits;
+    const int units = g.full_tiles + (g.n_tiles * g.m_tiles - g.full_tiles) * g.splits;
     int* err = g.ep.err;
     // Unit schedule: units u0, u0 + ustep, ... (per CTA, or per pair).
     const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
@@ -680,10 +704,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             uint32_t it = 0;
             int pre = 0;
             if (u0 < units) {
-                const int split = u0 % g.splits, tile = u0 / g.splits;
-                const int na = (tile / g.m_tiles) * TW + (int)rank * BM;
-                const int kb0 = split * g.kb_per_split;
-                const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
+                const Unit un = unit_of(g, u0, KB);
+                const int na = (un.tile / g.m_tiles) * TW + (int)rank * BM;
+                const int kb0 = un.kb0, nkb = un.nkb;
                 pre = min(nkb, STAGES);
                 for (int i = 0; i < pre; ++i) {
                     expect(i);
@@ -696,11 +719,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             griddep_launch();
             bool ok = true;
             for (int u = u0; u < units && ok; u += ustep) {
-                const int split = u % g.splits, tile = u / g.splits;
-                const int na = (tile / g.m_tiles) * TW + (int)rank * BM;
-                const int mb = (tile % g.m_tiles) * BN + (int)rank * C::B_ROWS;
-                const int kb0 = split * g.kb_per_split;
-                const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
+                const Unit un = unit_of(g, u, KB);
+                const int na = (un.tile / g.m_tiles) * TW + (int)rank * BM;
+                const int mb = (un.tile % g.m_tiles) * BN + (int)rank * C::B_ROWS;
+                const int kb0 = un.kb0, nkb = un.nkb;
                 for (int i = 0; i < nkb; ++i, ++it) {
                     const int s = it % STAGES;
                     const int kx = (kb0 + i) * BK;
@@ -736,9 +758,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             uint32_t it = 0, j = 0;
             bool ok = true;
             for (int u = u0; u < units && ok; u += ustep, ++j) {
-                const int split = u % g.splits;
-                const int kb0 = split * g.kb_per_split;
-                const int nkb = min(KB, kb0 + g.kb_per_split) - kb0;
+                const int nkb = unit_of(g, u, KB).nkb;
                 const uint32_t b = j % NACC, use = j / NACC;
                 const bool free_acc = CG == 2 ? mbar_wait_cluster_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err)
                                               : mbar_wait_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err);
@@ -779,7 +799,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         };
         uint32_t j = 0;
         for (int u = u0; u < units; u += ustep, ++j) {
-            const int split = u % g.splits, tile = u / g.splits;
+            const Unit un = unit_of(g, u, KB);
+            const int split = un.split, tile = un.tile, nsplit = un.nsplit;
             // n0: this CTA's first weight row (its TMEM lanes); m0: the tile's first activation row
             const int n0 = (tile / g.m_tiles) * TW + (int)rank * BM, m0 = (tile % g.m_tiles) * BN;
             const uint32_t b = j % NACC, use = j / NACC;
@@ -789,7 +810,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             fill_row_meta<BN>(g.ep, m0, g.M, meta, threadIdx.x - 64);
             epi_bar();
             const uint32_t tacc = tmem + b * C::ACC_COLS + ((uint32_t)(q * 32) << 16);
-            if (g.splits == 1 && g.ep.kind == EPI_ENTROPY) {
+            if (nsplit == 1 && g.ep.kind == EPI_ENTROPY) {
 #pragma unroll 1
                 for (int w = 0; w < WT; ++w) {
                     const int n = n0 + w * BM + q * 32 + lane;
@@ -805,7 +826,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) release(b);
-            } else if (g.splits == 1 && BN >= C::EPI_COLS && (g.N & 3) == 0) {
+            } else if (nsplit == 1 && BN >= C::EPI_COLS && (g.N & 3) == 0) {
                 // the accumulator is fully read once the last chunk is loaded: the
                 // next unit's MMAs may start while the stores finish
                 auto rel = [&]() {
@@ -830,7 +851,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                         break;
                     default: rel(); break;
                 }
-            } else if (g.splits == 1) {
+            } else if (nsplit == 1) {
 #pragma unroll 1
                 for (int w = 0; w < WT; ++w) {
                     const int nw = n0 + w * BM, n = nw + q * 32 + lane;
@@ -880,7 +901,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     if (threadIdx.x == 64) {
                         atomicAdd(ctr, 1);
                         const long long t0 = clock64();
-                        while (*reinterpret_cast<volatile int*>(ctr) < g.splits) {
+                        while (*reinterpret_cast<volatile int*>(ctr) < nsplit) {
                             if (clock64() - t0 > 2000000000LL) {
                                 set_error(err, kErrTimeout);
                                 break;
@@ -890,11 +911,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                         __threadfence();
                     }
                     epi_bar();
-                    const int rows = (BN + g.splits - 1) / g.splits;
+                    const int rows = (BN + nsplit - 1) / nsplit;
                     r0 = split * rows;
                     r1 = min(BN, r0 + rows);
                 } else {
-                    if (threadIdx.x == 64) *last_flag = (atomicAdd(ctr, 1) == g.splits - 1) ? 1 : 0;
+                    if (threadIdx.x == 64) *last_flag = (atomicAdd(ctr, 1) == nsplit - 1) ? 1 : 0;
                     epi_bar();
                     if (!*last_flag) continue;
                     __threadfence();
@@ -912,7 +933,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 #pragma unroll
                         for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
-                        for (int sp0 = 0; sp0 < g.splits; sp0 += 4) {
+                        for (int sp0 = 0; sp0 < nsplit; sp0 += 4) {
                             // up to 4 planes x 8 rows of independent loads in flight
                             float4 t4[4][8];
 #pragma unroll
@@ -921,7 +942,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 #pragma unroll
                                 for (int u = 0; u < 8; ++u) {
                                     const int rr = rb + 4 * u, m = m0 + rr;
-                                    t4[jj][u] = (sp0 + jj < g.splits && nok && rr < r1 && m < g.M)
+                                    t4[jj][u] = (sp0 + jj < nsplit && nok && rr < r1 && m < g.M)
                                                     ? __ldcg(reinterpret_cast<const float4*>(pl + (int64_t)m * g.N + nn))
                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                                 }
@@ -951,7 +972,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 epi_bar();
                 if (threadIdx.x == 64) {
                     if (!g.coop) *ctr = 0;
-                    else if (atomicAdd(ctr, 1) == 2 * g.splits - 1) atomicExch(ctr, 0);
+                    else if (atomicAdd(ctr, 1) == 2 * nsplit - 1) atomicExch(ctr, 0);
                 }
             }
         }
@@ -985,8 +1006,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// Hybrid schedule (hybrid = true): the tiles that fill whole rounds of the
+// launch run whole-K; only the tiles of the last, partial round are cut into
+// a.splits K slices (reduced by the last slice to finish), so that round keeps
+// every CTA busy.
+inline void set_full_tiles(GemmArgs& a, bool hybrid, int per_round) {
+    const int tiles = a.n_tiles * a.m_tiles;
+    a.full_tiles = 0;
+    if (!hybrid || a.splits == 1) return;
+    a.full_tiles = (tiles / per_round) * per_round;
+    if (a.full_tiles == tiles) a.splits = 1;  // no partial round
+}
+
 template <int BN, int WT, int BK, int CG = 1>
-cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, int grid, cudaStream_t st) {
+cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs a, int grid, bool hybrid,
+                      cudaStream_t st) {
     using C = PCfg<BN, WT, BK, CG>;
     auto kern = gemm_tc_kernel<BN, WT, BK, CG>;
     static int attr_dev = -1;
@@ -1019,6 +1053,7 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
         // any even grid is correct and no more pairs than fit at once are launched.
         if (a.splits > 1 && a.coop) return cudaErrorInvalidValue;
         const int pairs = std::max(1, std::min(grid / 2, max_pairs));
+        set_full_tiles(a, hybrid, pairs);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * pairs);
         cfg.blockDim = dim3(192);
@@ -1035,6 +1070,8 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, const Gemm
         cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, a);
     }
+    if (hybrid && a.coop) return cudaErrorInvalidValue;
+    set_full_tiles(a, hybrid, grid);
     if (!(a.splits > 1 && a.coop))
         return launch_pdl(kern, dim3(grid), dim3(192), C::SMEM_BYTES, st, tmW, tmX, a);
     // The slices of a tile wait for one another: launch cooperatively so all CTAs
@@ -1058,12 +1095,13 @@ namespace {
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
 GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1, int bk = BK_DEFAULT,
-                   int cg = 1) {
+                   int cg = 1, bool hybrid = false) {
     GemmPlan p;
     p.bn = bn;
     p.wt = wt;
     p.bk = bk;
     p.cg = cg;
+    p.hybrid = hybrid && splits > 1;
     p.m_tiles = (M + bn - 1) / bn;
     p.n_tiles = (N + BM * wt * cg - 1) / (BM * wt * cg);
     const int KB = (K + bk - 1) / bk;
@@ -1077,6 +1115,11 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
         p.grid = 2 * (int)std::min<long>(units, std::max(1, num_sms / 2));
         return p;
     }
+    if (p.hybrid) {  // whole rounds of full tiles: every SM
+        p.coop = 0;
+        p.grid = (int)std::min<long>(units, num_sms);
+        return p;
+    }
     const int per_round = std::max(p.splits, (num_sms / p.splits) * p.splits);
     p.grid = (int)std::min<long>(units, per_round);
     return p;
@@ -1084,15 +1127,15 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
 }  // namespace
 
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                        int force_wt, int force_bk, int force_coop, int force_cg) {
-    GemmPlan p =
-        plan_gemm_bf16_shape(M, N, K, num_sms, max_splits, force_bn, force_splits, force_wt, force_bk, force_cg);
-    p.coop = p.cg == 2 ? 0 : force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
+                        int force_wt, int force_bk, int force_coop, int force_cg, int force_hybrid) {
+    GemmPlan p = plan_gemm_bf16_shape(M, N, K, num_sms, max_splits, force_bn, force_splits, force_wt, force_bk,
+                                      force_cg, force_hybrid);
+    p.coop = (p.cg == 2 || p.hybrid) ? 0 : force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
     return p;
 }
 
 GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                              int force_wt, int force_bk, int force_cg) {
+                              int force_wt, int force_bk, int force_cg, int force_hybrid) {
     const int KB = (K + BK_DEFAULT - 1) / BK_DEFAULT;
     // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
     const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
@@ -1102,7 +1145,7 @@ GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, 
         const int wt = (cg == 1 && force_wt == 2 && bn >= 128) ? 2 : 1;
         const int bk = (cg == 1 && force_bk == 32 && bn >= 128) ? 32 : BK_DEFAULT;
         return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)), wt,
-                         bk, cg);
+                         bk, cg, force_hybrid != 0);
     }
     // Cost in units of one 256-column k-block per CTA: rounds x k-block time x
     // (k-blocks per unit + per-unit overhead + the partial plane's round trip
@@ -1161,32 +1204,33 @@ cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int
     const int tw = 128 * p.wt * p.cg;
     if (ep.kind == EPI_ENTROPY && (p.splits != 1 || !ep.epart || ep.npart < ((N + tw - 1) / tw) * p.wt * p.cg * 4))
         return cudaErrorInvalidValue;
-    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, ep};
+    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, 0, ep};
+    const bool hy = p.hybrid != 0;
     if (p.cg == 2) {
         if (p.wt != 1 || p.bk != 64) return cudaErrorInvalidValue;
-        if (p.bn == 256) return launch_bn<256, 1, 64, 2>(tmW, tmX, a, p.grid, st);
-        if (p.bn == 128) return launch_bn<128, 1, 64, 2>(tmW, tmX, a, p.grid, st);
+        if (p.bn == 256) return launch_bn<256, 1, 64, 2>(tmW, tmX, a, p.grid, hy, st);
+        if (p.bn == 128) return launch_bn<128, 1, 64, 2>(tmW, tmX, a, p.grid, hy, st);
         return cudaErrorInvalidValue;
     }
     if (p.bk == 32) {
-        if (p.wt == 2 && p.bn == 256) return launch_bn<256, 2, 32>(tmW, tmX, a, p.grid, st);
-        if (p.wt == 2 && p.bn == 128) return launch_bn<128, 2, 32>(tmW, tmX, a, p.grid, st);
-        if (p.wt == 1 && p.bn == 256) return launch_bn<256, 1, 32>(tmW, tmX, a, p.grid, st);
+        if (p.wt == 2 && p.bn == 256) return launch_bn<256, 2, 32>(tmW, tmX, a, p.grid, hy, st);
+        if (p.wt == 2 && p.bn == 128) return launch_bn<128, 2, 32>(tmW, tmX, a, p.grid, hy, st);
+        if (p.wt == 1 && p.bn == 256) return launch_bn<256, 1, 32>(tmW, tmX, a, p.grid, hy, st);
         return cudaErrorInvalidValue;
     }
     if (p.wt == 2) {
         switch (p.bn) {
-            case 128: return launch_bn<128, 2, 64>(tmW, tmX, a, p.grid, st);
-            case 256: return launch_bn<256, 2, 64>(tmW, tmX, a, p.grid, st);
+            case 128: return launch_bn<128, 2, 64>(tmW, tmX, a, p.grid, hy, st);
+            case 256: return launch_bn<256, 2, 64>(tmW, tmX, a, p.grid, hy, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (p.bn) {
-        case 16: return launch_bn<16, 1, 64>(tmW, tmX, a, p.grid, st);
-        case 32: return launch_bn<32, 1, 64>(tmW, tmX, a, p.grid, st);
-        case 64: return launch_bn<64, 1, 64>(tmW, tmX, a, p.grid, st);
-        case 128: return launch_bn<128, 1, 64>(tmW, tmX, a, p.grid, st);
-        case 256: return launch_bn<256, 1, 64>(tmW, tmX, a, p.grid, st);
+        case 16: return launch_bn<16, 1, 64>(tmW, tmX, a, p.grid, hy, st);
+        case 32: return launch_bn<32, 1, 64>(tmW, tmX, a, p.grid, hy, st);
+        case 64: return launch_bn<64, 1, 64>(tmW, tmX, a, p.grid, hy, st);
+        case 128: return launch_bn<128, 1, 64>(tmW, tmX, a, p.grid, hy, st);
+        case 256: return launch_bn<256, 1, 64>(tmW, tmX, a, p.grid, hy, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -134,3 +134,30 @@ def test_linear_bf16_cta_pair_matches_fp64_matmul(M, N, K, tile_n, k_splits):
     # the same plan without pairs agrees to accumulation order
     Y1 = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=k_splits).cpu().numpy().astype(np.float64)
     assert np.all(np.abs(Y - Y1) <= 2e-4 * bound + 1e-30)
+
+
+@pytest.mark.parametrize("M,N,K,tile_n,k_splits,pair", [
+    (256, 10240, 512, 128, 3, False),   # 160 tiles: one full round of 148 CTAs, 12 tiles split
+    (256, 20480, 256, 256, 2, True),    # 80 pair tiles: a full round of pairs, the rest split
+    (200, 10368, 520, 128, 4, False),   # ragged rows and K, a partial round of split tiles
+    (64, 1024, 1024, 128, 3, False),    # fewer tiles than CTAs: every tile split
+])
+def test_linear_bf16_hybrid_split_matches_fp64_matmul(M, N, K, tile_n, k_splits, pair):
+    """Hybrid schedule (whole-K tiles for the full rounds of the persistent grid,
+    K slices only for the last partial round) against the fp64 matmul and bound
+    as above, and against the plain single-slice plan."""
+    from streaming_decoding_b200 import linear_bf16
+    X = synth.normal(35, M * 3 + K, 1.0, (M, K), "bf16")
+    W = synth.normal(36, N * 7 + K, 0.02, (N, K), "bf16")
+    Xt = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+    Wt = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=k_splits, cta_pair=pair, hybrid=True)
+    Y = Y.cpu().numpy().astype(np.float64)
+    x64 = synth.bf16_bits_to_f32(X).astype(np.float64)
+    w64 = synth.bf16_bits_to_f32(W).astype(np.float64)
+    ref = x64 @ w64.T
+    bound = np.abs(x64) @ np.abs(w64).T
+    err = np.abs(Y - ref)
+    assert np.all(err <= 1e-4 * bound + 1e-30), float((err / (bound + 1e-30)).max())
+    Y1 = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=1, cta_pair=pair).cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(Y - Y1) <= 2e-4 * bound + 1e-30)
