@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the batch-1 and regime sweeps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="headline measurement only (for profiler runs)")
+    ap.add_argument("--tile-n", type=int, default=0, help="kernel case: pin the GEMM tile width (0 = automatic)")
+    ap.add_argument("--cta-pair", action="store_true", help="kernel case: CTA-pair GEMM tiles (tile width 128 or 256)")
     ap.add_argument("--kernel-case", default=None,
                     help="run one projection of the batch-16 step (gemm_qkv|gemm_o|gemm_gate_up|gemm_down|"
                          "gemm_lm_head) three times through wedlm_linear_bf16, or 'attention' (3 decode steps of "
@@ -503,7 +505,7 @@ def attention_case(steps: int = 3):
                       "prefill_attention_launches": cfg["B"] * 2}))
 
 
-def kernel_case(name: str):
+def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False):
     import torch
     from streaming_decoding_b200 import linear_bf16
     if name == "attention":
@@ -515,15 +517,16 @@ def kernel_case(name: str):
     X = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
     for _ in range(3):
-        linear_bf16(X, W)
+        linear_bf16(X, W, tile_n=tile_n, cta_pair=cta_pair)
     torch.cuda.synchronize()
-    print(json.dumps({"kernel_case": name, "M": M, "N": N, "K": K, "weight_bytes": 2 * N * K}))
+    print(json.dumps({"kernel_case": name, "M": M, "N": N, "K": K, "weight_bytes": 2 * N * K, "tile_n": tile_n,
+                      "cta_pair": cta_pair}))
 
 
 if __name__ == "__main__":
     args = parse()
     if args.kernel_case:
-        kernel_case(args.kernel_case)
+        kernel_case(args.kernel_case, args.tile_n, args.cta_pair)
     elif args.impl == "reference":
         run_reference(args)
     else:
