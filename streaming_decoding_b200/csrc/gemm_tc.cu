@@ -867,23 +867,37 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 if (lane == 0) release(b);
             } else {
                 float* plane = g.ep.ws + (int64_t)split * g.M * g.N;
+                if constexpr (BN >= C::EPI_COLS) {
+                    // the slice's fp32 partial through the staged path (float4 rows);
+                    // rows the epilogue skips are not written and never read back
+                    EpiParams pe = g.ep;
+                    pe.kind = EPI_STORE;
+                    pe.out = plane;
+                    auto rel = [&]() {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) release(b);
+                    };
+                    staged_epilogue<EPI_STORE, BN, WT>(pe, g.M, g.N, n0, m0, tacc, epi_stage, meta, q, lane, rel);
+                } else {
 #pragma unroll 1
-                for (int w = 0; w < WT; ++w) {
-                    const int n = n0 + w * BM + q * 32 + lane;
+                    for (int w = 0; w < WT; ++w) {
+                        const int n = n0 + w * BM + q * 32 + lane;
 #pragma unroll 1
-                    for (int c = 0; c < BN; c += 16) {
-                        float v[16];
-                        tmem_ld16(tacc + (uint32_t)(w * BN + c), v);
+                        for (int c = 0; c < BN; c += 16) {
+                            float v[16];
+                            tmem_ld16(tacc + (uint32_t)(w * BN + c), v);
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int m = m0 + c + k;
-                            if (m < g.M && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
+                            for (int k = 0; k < 16; ++k) {
+                                const int m = m0 + c + k;
+                                if (m < g.M && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
+                            }
                         }
                     }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) release(b);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) release(b);
                 // Two fixups of the K slices (both sum in fixed split order, so
                 // results are deterministic):
                 //  - distributed (g.coop, cooperative launch: the slices of a tile
