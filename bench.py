@@ -284,6 +284,22 @@ def step_bytes_flops(dims, B, W, S_mean):
     return byt, fl
 
 
+def combine_ranks(dist, ms: float, tokens: float, device) -> tuple:
+    """Whole-job aggregation across ranks: the slowest rank's device time (max)
+    and the committed tokens of all ranks (sum); throughput = sum / max."""
+    import torch
+    t = torch.tensor([ms, tokens], dtype=torch.float64, device=device)
+    mx = t.clone()
+    dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(mx[0]), float(t[1])
+
+
+def rank_prompts(cfg: dict, rank: int):
+    """Each replica decodes its own prompts (weak scaling: fixed work per GPU)."""
+    return synth.prompts(cfg, seed=cfg["prompt_seed"] + 100 * rank)
+
+
 def run_ours(a):
     import torch
     rank = int(os.environ.get("RANK", "0"))
@@ -300,7 +316,7 @@ def run_ours(a):
     dims = cfg["model"]
     pk = peaks()
     rep = Replica(cfg, local, seed=rank)
-    prompts = synth.prompts(cfg, seed=cfg["prompt_seed"] + 100 * rank)
+    prompts = rank_prompts(cfg, rank)
     B, W, N = cfg["B"], cfg["W"], cfg["N"]
     from streaming_decoding_b200 import step_params
     prm = step_params(cfg["lam"], cfg["tau"], False, cfg["logit_scale"])
@@ -318,11 +334,7 @@ def run_ours(a):
     ms_all = ms
     tok_all = committed
     if dist:
-        t = torch.tensor([ms, committed], dtype=torch.float64, device="cuda")
-        mx = t.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        ms_all, tok_all = float(mx[0]), float(t[1])
+        ms_all, tok_all = combine_ranks(dist, ms, committed, "cuda")
     value = tok_all / (ms_all / 1e3)
     S1 = np.mean([rep.eng.stats(b)["committed_len"] for b in range(B)])
 
@@ -338,11 +350,8 @@ def run_ours(a):
     e_ms, e_wall, e_tok, d2h = rep.timed_e2e(prm, e2e_steps)
     e2e_val = e_tok / (e_ms / 1e3)
     if dist:
-        t = torch.tensor([e_ms, e_tok], dtype=torch.float64, device="cuda")
-        mx = t.clone()
-        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        e2e_val = float(t[1]) / (float(mx[0]) / 1e3)
+        e_max, e_sum = combine_ranks(dist, e_ms, e_tok, "cuda")
+        e2e_val = e_sum / (e_max / 1e3)
 
     extra = {"prefill": {"tokens": rep.prefill_tokens, "seconds": round(rep.prefill_s, 3),
                          "tok_per_s": round(rep.prefill_tokens / rep.prefill_s, 1)},
