@@ -221,10 +221,17 @@ def gemm_shapes(dims, M):
 
 
 def src_hash(*names):
+    """Hash of the named CUDA sources' code: comments and trailing blanks are
+    dropped, so an edit that only touches comments keeps a profile valid."""
+    import re
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "streaming_decoding_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "streaming_decoding_b200", "csrc", n), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

@@ -17,23 +17,30 @@
 //               accumulation), releasing ring stages with tcgen05.commit; with
 //               two accumulators the next unit's MMAs overlap the previous
 //               unit's epilogue,
-//   warps 2..5  epilogue: tcgen05.ld 16 columns at a time (warp w owns TMEM
-//               lanes 32*(w%4)..+31), then either the fused epilogue directly
-//               or, for K split over several CTAs, a partial plane and a
-//               ticket; either the slices of a tile (co-resident by
-//               cooperative launch) wait for each other and each reduces a
-//               share of the rows, or the slice that finishes last reduces the
-//               tile alone and nobody waits; both sum in fixed split order.
+//   warps 2..5  epilogue (warp w owns TMEM lanes 32*(w%4)..+31): 32 accumulator
+//               columns at a time are loaded (tcgen05.ld), stored transposed to
+//               shared memory and finished as float4 runs of weight rows for 8
+//               activation rows each (coalesced rows, vector stores; the loads
+//               the fused epilogue needs besides the accumulator are issued
+//               first); the accumulator is released to the MMA thread right
+//               after its last load.  With K split over several units each
+//               slice writes its fp32 partial plane the same way and takes a
+//               ticket; either the slices of a tile (co-resident by cooperative
+//               launch) wait for each other and each reduces a share of the
+//               rows, or the slice that finishes last reduces the tile alone
+//               and nobody waits; both sum in fixed split order.  A hybrid
+//               schedule splits only the tiles of the last partial round.
 // CTA pairs (CG = 2, clusters of two): the pair computes a 256-row weight tile
 // with tcgen05.mma.cta_group::2 issued by the even CTA.  Each CTA stages its own
 // 128 weight rows and half of the activation rows; the MMA reads the operands
 // from both CTAs' shared memory and writes each CTA's 128 accumulator lanes in
-// its own TMEM.  Per output a CTA moves half the activation bytes of a
-// single-CTA tile of the same width, which is what limits the main loop: the
-// operand bytes streamed from L2 into each SM per k-block.  Loads of both CTAs
-// complete on the even CTA's ring barrier; its commits release the ring stage
-// and hand over the accumulator in both CTAs; both CTAs' epilogues release the
-// accumulator on the even CTA's barrier.
+// its own TMEM.  A CTA stages 32 KB per 64-deep k-block for 128 x 256 outputs
+// (a single-CTA 128 x 256 tile stages 48 KB): two thirds of the operand bytes
+// streamed from L2 into the SMs per output (half those of 128 x 128 tiles), and
+// room for a 6-stage ring.
+// Loads of both CTAs complete on the even CTA's ring barrier; its commits
+// release the ring stage and hand over the accumulator in both CTAs; both CTAs'
+// epilogues release the accumulator on the even CTA's barrier.
 // Every mbarrier wait is bounded; on timeout the kernel records an error in
 // the device error word and unwinds (freeing TMEM) instead of hanging.
 #include <algorithm>
