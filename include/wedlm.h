@@ -395,7 +395,11 @@ wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int3
  *      128 or 256 (WEDLM_ERR_INVALID_ARG otherwise);
  *   2  hybrid K split: the tiles that fill whole rounds of the persistent grid
  *      run over all of K, only the tiles of the last partial round are cut into
- *      k_splits slices (k_splits > 1), reduced by the slice that finishes last.
+ *      k_splits slices (k_splits > 1), reduced by the slice that finishes last;
+ *   4  cluster K split: the k_splits (2..4) slices of a tile are the CTAs of
+ *      one thread-block cluster, one tile slice per CTA, and are reduced through
+ *      distributed shared memory (not combinable with 1 or 2; tile_n 128 or 256;
+ *      N % 4 == 0).
  * Results agree with wedlm_linear_bf16 to fp32 accumulation order. */
 wedlm_status wedlm_linear_bf16_sched(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
                                      int32_t tile_n, int32_t k_splits, int32_t schedule, void* stream);

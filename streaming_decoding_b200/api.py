@@ -262,19 +262,21 @@ def entropy_select_noalloc(logits, vocab: int, mask_id: int, filled, n, stride: 
 
 
 def linear_bf16(X, W, stream=None, tile_n: int = 0, k_splits: int = 0, cta_pair: bool = False,
-                hybrid: bool = False):
+                hybrid: bool = False, cluster_k: bool = False):
     """Y = X W^T (fp32) on the tcgen05 GEMM; X [M][K], W [N][K] torch.bfloat16 CUDA tensors.
     tile_n / k_splits pin the launch shape (0 = automatic); cta_pair runs CTA-pair
     tiles of 256 weight rows (tile_n 128 or 256); hybrid splits K only for the
-    tiles of the last partial round of the persistent grid."""
+    tiles of the last partial round of the persistent grid; cluster_k makes the
+    k_splits (2..4) slices of a tile one thread-block cluster reduced through
+    distributed shared memory."""
     import torch
     M, K = X.shape
     N = W.shape[0]
     Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
     X, W = X.contiguous(), W.contiguous()
     lib = _lib.load()
-    if cta_pair or hybrid:
-        sched = (1 if cta_pair else 0) | (2 if hybrid else 0)
+    if cta_pair or hybrid or cluster_k:
+        sched = (1 if cta_pair else 0) | (2 if hybrid else 0) | (4 if cluster_k else 0)
         _check(lib.wedlm_linear_bf16_sched(_ptr(X), _ptr(W), _ptr(Y), M, N, K, tile_n, k_splits, sched,
                                            _stream_handle(stream)), "wedlm_linear_bf16_sched")
     else:

@@ -94,6 +94,8 @@ struct GemmArgs {
     int M, N, K, kb_per_split, splits, n_tiles, m_tiles;
     int coop;        // split fixup: 1 distributed (cooperative launch), 0 last arriver
     int full_tiles;  // tiles [0, full_tiles) run whole-K as one unit each; the rest in `splits` K slices
+    int ks;          // > 1: the `splits` slices of a tile are the CTAs of one cluster (one unit per CTA),
+                     // reduced through distributed shared memory
     EpiParams ep;
 };
 
@@ -222,6 +224,11 @@ __device__ __forceinline__ uint64_t sdesc_k(const void* p) {
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
+
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
 template <int CG>
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -627,6 +634,91 @@ __device__ __forceinline__ void staged_epilogue(const EpiParams& ep, int M, int 
     }
 }
 
+// K slices of one tile computed by the ks CTAs of a cluster (cluster rank =
+// slice), reduced through distributed shared memory instead of partial planes
+// in global memory.  Chunk c (32 accumulator columns) belongs to CTA c % ks;
+// once every CTA's own MMAs are done its operand ring is idle and becomes the
+// receive buffer: each CTA pushes its partial of every chunk it does not own
+// into the owner's ring, then sums the slices of its own chunks in rank order
+// (deterministic) and finishes them like staged_epilogue.  Waits are bounded;
+// false when one gave up (the error word is set).
+template <int KIND, int BN>
+__device__ __forceinline__ bool cluster_epilogue(const EpiParams& ep, int M, int N, int n0, int m0, uint32_t tacc,
+                                                 float* stage, float* recv, uint64_t* rfree, uint64_t* rfull,
+                                                 const RowMeta* meta, int q, int lane, int ks, int rank, int* err) {
+    constexpr int COLS = 32, NCH = BN / COLS, CH_FLOATS = COLS * BM;
+    const int per_owner = (NCH + ks - 1) / ks;
+    // this CTA's ring is idle: every other CTA may write into it
+    if (threadIdx.x == 64)
+        for (int r = 0; r < ks; ++r)
+            if (r != rank) mbar_arrive_cluster(mapa_rank(smem_u32(rfree), (uint32_t)r));
+    if (!epi_all(mbar_wait_cluster_bounded(smem_u32(rfree), 0, err))) return false;
+    // push this slice's partial of every chunk another CTA owns
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+        const int o = c % ks;
+        if (o == rank) continue;
+        float v[COLS];
+        tmem_ld32(tacc + (uint32_t)(c * COLS), v);
+        const int slot = rank < o ? rank : rank - 1;  // this CTA's index among o's senders
+        const uint32_t dst =
+            mapa_rank(smem_u32(recv + (size_t)(slot * per_owner + c / ks) * CH_FLOATS + q * 32 + lane), (uint32_t)o);
+#pragma unroll
+        for (int k = 0; k < COLS; ++k) st_cluster_f32(dst + (uint32_t)(k * BM * 4), v[k]);
+    }
+    fence_acq_rel_cluster();
+    __syncwarp();
+    if (lane == 0)
+        for (int o = 0; o < ks; ++o)
+            if (o != rank) mbar_arrive_cluster(mapa_rank(smem_u32(rfull), (uint32_t)o));
+    if (!epi_all(mbar_wait_cluster_bounded(smem_u32(rfull), 0, err))) return false;
+    // this CTA's chunks: all slices summed in rank order, then the fused epilogue
+    const int c4 = 4 * lane, nn = n0 + c4;
+    const bool nok = nn < N;
+#pragma unroll 1
+    for (int c = rank; c < NCH; c += ks) {
+        int mrow[8], krow[8];
+        bool okr[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int rl = q + 4 * u;
+            krow[u] = c * COLS + rl;
+            mrow[u] = m0 + c * COLS + rl;
+            okr[u] = nok && mrow[u] < M;
+        }
+        EpiPre p;
+        epi_pre<KIND>(ep, n0, nn, mrow, krow, okr, meta, N, p);
+        {
+            float v[COLS], a[COLS];
+            tmem_ld32(tacc + (uint32_t)(c * COLS), v);
+#pragma unroll
+            for (int k = 0; k < COLS; ++k) a[k] = 0.f;
+#pragma unroll 1
+            for (int r = 0; r < ks; ++r) {
+                if (r == rank) {
+#pragma unroll
+                    for (int k = 0; k < COLS; ++k) a[k] += v[k];
+                } else {
+                    const int slot = r < rank ? r : r - 1;
+                    const float* src = recv + (size_t)(slot * per_owner + c / ks) * CH_FLOATS + q * 32 + lane;
+#pragma unroll
+                    for (int k = 0; k < COLS; ++k) a[k] += src[k * BM];
+                }
+            }
+            float* srow = stage + q * 32 + lane;
+#pragma unroll
+            for (int k = 0; k < COLS; ++k) srow[k * BM] = a[k];
+        }
+        epi_bar();
+        float4 acc[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = *reinterpret_cast<const float4*>(stage + (q + 4 * u) * BM + c4);
+        epi_fin<KIND>(ep, n0, nn, mrow, acc, p, N);
+        epi_bar();
+    }
+    return true;
+}
+
 template <int BN, int WT, int BK, int CG>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW,
                                                          const __grid_constant__ CUtensorMap tmX, const GemmArgs g) {
@@ -643,7 +735,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     uint64_t* empty = full + STAGES;
     uint64_t* accf = empty + STAGES;
     uint64_t* acce = accf + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
+    uint64_t* rfree = acce + 2;  // cluster K split: the other CTAs' rings are idle
+    uint64_t* rfull = rfree + 1; // cluster K split: the other slices of this CTA's chunks have arrived
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rfull + 1);
     int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // epilogue warps: this CTA reduces the tile
     RowMeta* meta = reinterpret_cast<RowMeta*>(smem + STAGES * C::STAGE_BYTES + 256);
     float* epi_stage = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256 + C::META_BYTES);
@@ -668,6 +762,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 4 * CG);  // the epilogue warps of every CTA of the pair
         }
+        mbar_init(rfree, g.ks > 1 ? g.ks - 1 : 1);
+        mbar_init(rfull, g.ks > 1 ? 4 * (g.ks - 1) : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -685,8 +781,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         }
     }
     tc_fence_before();
-    if constexpr (CG == 2)
-        cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
+    if (CG == 2 || g.ks > 1)
+        cluster_sync();  // every CTA's barriers are initialised before another signals them
     else
         __syncthreads();
     tc_fence_after();
@@ -872,6 +968,35 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) release(b);
+            } else if (g.ks > 1) {
+                bool ok2 = true;
+                if constexpr (WT == 1 && CG == 1 && BN >= 128) {
+                    const int rank = (int)cluster_rank();
+                    float* recv = reinterpret_cast<float*>(sA);
+                    switch (g.ep.kind) {
+                        case EPI_STORE:
+                            ok2 = cluster_epilogue<EPI_STORE, BN>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, recv, rfree,
+                                                                  rfull, meta, q, lane, g.ks, rank, err);
+                            break;
+                        case EPI_RESIDUAL:
+                            ok2 = cluster_epilogue<EPI_RESIDUAL, BN>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, recv,
+                                                                     rfree, rfull, meta, q, lane, g.ks, rank, err);
+                            break;
+                        case EPI_SWIGLU:
+                            ok2 = cluster_epilogue<EPI_SWIGLU, BN>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, recv, rfree,
+                                                                   rfull, meta, q, lane, g.ks, rank, err);
+                            break;
+                        case EPI_QKV_ROPE:
+                            ok2 = cluster_epilogue<EPI_QKV_ROPE, BN>(g.ep, g.M, g.N, n0, m0, tacc, epi_stage, recv,
+                                                                     rfree, rfull, meta, q, lane, g.ks, rank, err);
+                            break;
+                        default: break;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) release(b);
+                if (!ok2) break;
             } else {
                 float* plane = g.ep.ws + (int64_t)split * g.M * g.N;
                 if constexpr (BN >= C::EPI_COLS) {
@@ -999,8 +1124,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         }
     }
     tc_fence_before();
-    if constexpr (CG == 2)
-        cluster_sync();  // no CTA leaves while the other may still signal or read it
+    if (CG == 2 || g.ks > 1)
+        cluster_sync();  // no CTA leaves while another may still signal or read it
     else
         __syncthreads();
     if (warp == 1) {
@@ -1091,6 +1216,24 @@ cudaError_t launch_bn(const CUtensorMap& tmW, const CUtensorMap& tmX, GemmArgs a
         cfg.numAttrs = 2;
         return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, a);
     }
+    if (a.ks > 1) {
+        if (grid % a.ks) return cudaErrorInvalidValue;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(192);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = a.ks;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, a);
+    }
     if (hybrid && a.coop) return cudaErrorInvalidValue;
     set_full_tiles(a, hybrid, grid);
     if (!(a.splits > 1 && a.coop))
@@ -1116,7 +1259,7 @@ namespace {
 int bn_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256; }
 
 GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt = 1, int bk = BK_DEFAULT,
-                   int cg = 1, bool hybrid = false) {
+                   int cg = 1, bool hybrid = false, bool cluster_k = false) {
     GemmPlan p;
     p.bn = bn;
     p.wt = wt;
@@ -1131,6 +1274,13 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
     // Units are dealt in rounds of `grid`; a multiple of the split count keeps
     // the splits of every tile in one round (they wait for each other).
     const long units = (long)p.m_tiles * p.n_tiles * p.splits;
+    if (cluster_k && p.splits > 1 && cg == 1 && wt == 1) {  // one unit per CTA, a tile's slices one cluster
+        p.ks = p.splits;
+        p.coop = 0;
+        p.hybrid = 0;
+        p.grid = (int)units;
+        return p;
+    }
     if (cg == 2) {  // CTA pairs; the K-split fixup of pairs is the last-arriver one
         p.coop = 0;
         p.grid = 2 * (int)std::min<long>(units, std::max(1, num_sms / 2));
@@ -1148,15 +1298,15 @@ GemmPlan make_plan(int M, int N, int K, int num_sms, int bn, int splits, int wt 
 }  // namespace
 
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                        int force_wt, int force_bk, int force_coop, int force_cg, int force_hybrid) {
+                        int force_wt, int force_bk, int force_coop, int force_cg, int force_hybrid, int force_cluster_k) {
     GemmPlan p = plan_gemm_bf16_shape(M, N, K, num_sms, max_splits, force_bn, force_splits, force_wt, force_bk,
-                                      force_cg, force_hybrid);
-    p.coop = (p.cg == 2 || p.hybrid) ? 0 : force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
+                                      force_cg, force_hybrid, force_cluster_k);
+    p.coop = (p.cg == 2 || p.hybrid || p.ks > 1) ? 0 : force_coop >= 0 ? (force_coop ? 1 : 0) : (M > 128 ? 1 : 0);
     return p;
 }
 
 GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                              int force_wt, int force_bk, int force_cg, int force_hybrid) {
+                              int force_wt, int force_bk, int force_cg, int force_hybrid, int force_cluster_k) {
     const int KB = (K + BK_DEFAULT - 1) / BK_DEFAULT;
     // the split-K reduction reads float4 runs of a row, so N must be a multiple of 4
     const int smax = (N % 4) ? 1 : std::max(1, std::min({max_splits, KB, 16}));
@@ -1165,8 +1315,9 @@ GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, 
         const int cg = (force_cg == 2 && (bn == 128 || bn == 256)) ? 2 : 1;
         const int wt = (cg == 1 && force_wt == 2 && bn >= 128) ? 2 : 1;
         const int bk = (cg == 1 && force_bk == 32 && bn >= 128) ? 32 : BK_DEFAULT;
-        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, smax)), wt,
-                         bk, cg, force_hybrid != 0);
+        const bool ck = force_cluster_k != 0 && cg == 1 && wt == 1 && bk == BK_DEFAULT && bn >= 128;
+        return make_plan(M, N, K, num_sms, bn, std::max(1, std::min(force_splits > 0 ? force_splits : 1, ck ? 4 : smax)),
+                         ck ? 1 : wt, bk, cg, force_hybrid != 0 && !ck, ck);
     }
     // Cost in units of one 256-column k-block per CTA: rounds x k-block time x
     // (k-blocks per unit + per-unit overhead + the partial plane's round trip
@@ -1225,8 +1376,17 @@ cudaError_t launch_gemm_bf16(const CUtensorMap& tmW, const CUtensorMap& tmX, int
     const int tw = 128 * p.wt * p.cg;
     if (ep.kind == EPI_ENTROPY && (p.splits != 1 || !ep.epart || ep.npart < ((N + tw - 1) / tw) * p.wt * p.cg * 4))
         return cudaErrorInvalidValue;
-    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, 0, ep};
+    GemmArgs a{M, N, K, p.kb_per_split, p.splits, p.n_tiles, p.m_tiles, p.coop, 0, p.ks, ep};
     const bool hy = p.hybrid != 0;
+    if (p.ks > 1) {
+        // cluster K split: one unit per CTA, a tile's slices are one cluster
+        if (p.splits != p.ks || p.wt != 1 || p.cg != 1 || p.bk != 64 || (N & 3) || ep.kind == EPI_ENTROPY ||
+            p.grid != p.n_tiles * p.m_tiles * p.ks)
+            return cudaErrorInvalidValue;
+        if (p.bn == 256) return launch_bn<256, 1, 64>(tmW, tmX, a, p.grid, false, st);
+        if (p.bn == 128) return launch_bn<128, 1, 64>(tmW, tmX, a, p.grid, false, st);
+        return cudaErrorInvalidValue;
+    }
     if (p.cg == 2) {
         if (p.wt != 1 || p.bk != 64) return cudaErrorInvalidValue;
         if (p.bn == 256) return launch_bn<256, 1, 64, 2>(tmW, tmX, a, p.grid, hy, st);

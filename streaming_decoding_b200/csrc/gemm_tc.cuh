@@ -57,6 +57,8 @@ struct GemmPlan {
     int coop = 1;      // K-split fixup: 1 the slices wait and share the reduction, 0 the last one reduces
     int cg = 1;        // 2: CTA pairs (clusters of two) share 256-row weight tiles; coop is then 0
     int hybrid = 0;    // 1: only the tiles of the last partial round are split (splits slices); coop is then 0
+    int ks = 1;        // > 1: a tile's `splits` slices are the CTAs of one cluster, one unit per CTA, reduced
+                       // through distributed shared memory (bn 128 or 256, wt 1, cg 1)
     int splits = 1;
     int kb_per_split = 1;
     int m_tiles = 1;
@@ -71,12 +73,14 @@ struct GemmPlan {
 // M > 128 rows, last arriver otherwise).  force_cg = 2 (with force_bn 128 or
 // 256) selects CTA-pair tiles.
 // force_hybrid = 1 (with force_splits > 1): the whole rounds of tiles run whole-K
-// and only the last partial round is split.
+// and only the last partial round is split.  force_cluster_k = 1 (with
+// force_splits 2..4, force_bn 128 or 256): cluster K split.
 GemmPlan plan_gemm_bf16(int M, int N, int K, int num_sms, int max_splits, int force_bn = 0, int force_splits = 0,
                         int force_wt = 0, int force_bk = 0, int force_coop = -1, int force_cg = 1,
-                        int force_hybrid = 0);
+                        int force_hybrid = 0, int force_cluster_k = 0);
 GemmPlan plan_gemm_bf16_shape(int M, int N, int K, int num_sms, int max_splits, int force_bn, int force_splits,
-                              int force_wt, int force_bk, int force_cg = 1, int force_hybrid = 0);
+                              int force_wt, int force_bk, int force_cg = 1, int force_hybrid = 0,
+                              int force_cluster_k = 0);
 
 // 2-D bf16 tensor map [rows][cols], boxes of bk columns (64: 128-byte swizzle,
 // 32: 64-byte swizzle) by box_rows rows.

@@ -64,7 +64,8 @@ wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M
 }
 
 static wedlm_status linear_bf16(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
-                                int32_t tile_n, int32_t k_splits, int32_t cg, int32_t hybrid, void* stream) {
+                                int32_t tile_n, int32_t k_splits, int32_t cg, int32_t hybrid, int32_t cluster_k,
+                                void* stream) {
     if (M < 1 || N < 1 || K < 8 || K % 8 || !X || !W || !Y) return WEDLM_ERR_INVALID_ARG;
     if (tile_n != 0 && tile_n != 16 && tile_n != 32 && tile_n != 64 && tile_n != 128 && tile_n != 256)
         return WEDLM_ERR_INVALID_ARG;
@@ -75,7 +76,9 @@ static wedlm_status linear_bf16(const void* X, const void* W, float* Y, int32_t 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    GemmPlan p = plan_gemm_bf16(M, N, K, sms, 16, tile_n, k_splits, 0, 0, -1, cg, hybrid);
+    if (cluster_k && (cg == 2 || hybrid || (tile_n != 128 && tile_n != 256) || k_splits < 2 || k_splits > 4 || N % 4))
+        return WEDLM_ERR_INVALID_ARG;
+    GemmPlan p = plan_gemm_bf16(M, N, K, sms, 16, tile_n, k_splits, 0, 0, -1, cg, hybrid, cluster_k);
     if (p.cg != (cg == 2 ? 2 : 1)) return WEDLM_ERR_INVALID_ARG;
     CUtensorMap tw, tx;
     if (!make_tmap_bf16(&tw, W, (uint64_t)N, (uint64_t)K, 128)) return WEDLM_ERR_CUDA;
@@ -111,13 +114,14 @@ static wedlm_status linear_bf16(const void* X, const void* W, float* Y, int32_t 
 
 wedlm_status wedlm_linear_bf16_plan(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
                                     int32_t tile_n, int32_t k_splits, void* stream) {
-    return linear_bf16(X, W, Y, M, N, K, tile_n, k_splits, 1, 0, stream);
+    return linear_bf16(X, W, Y, M, N, K, tile_n, k_splits, 1, 0, 0, stream);
 }
 
 wedlm_status wedlm_linear_bf16_sched(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K,
                                      int32_t tile_n, int32_t k_splits, int32_t schedule, void* stream) {
-    if (schedule & ~3) return WEDLM_ERR_INVALID_ARG;
-    return linear_bf16(X, W, Y, M, N, K, tile_n, k_splits, (schedule & 1) ? 2 : 1, (schedule & 2) ? 1 : 0, stream);
+    if (schedule & ~7) return WEDLM_ERR_INVALID_ARG;
+    return linear_bf16(X, W, Y, M, N, K, tile_n, k_splits, (schedule & 1) ? 2 : 1, (schedule & 2) ? 1 : 0,
+                       (schedule & 4) ? 1 : 0, stream);
 }
 
 }  // extern "C"

@@ -330,16 +330,18 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
     };
     std::vector<std::pair<float, GemmPlan>> timed;
     for (const Shape& sh : shapes) {
-        for (int spc : {1, 2, -2, 3, -3, 4, -4, 6, -6, 8, -8, 12, -12, 16, -16, 102, 103, 104, 106}) {
+        for (int spc : {1, 2, -2, 3, -3, 4, -4, 6, -6, 8, -8, 12, -12, 16, -16, 102, 103, 104, 106, 202, 203, 204}) {
             // negative: the same split count with the last-arriver fixup (the
-            // only one CTA pairs use); above 100: hybrid schedule, only the last
-            // partial round split in (spc - 100) slices
-            const bool hy = spc > 100;
-            const int sp = hy ? spc - 100 : spc < 0 ? -spc : spc;
+            // only one CTA pairs use); 10x: hybrid schedule, only the last
+            // partial round split in x slices; 20x: x slices as the CTAs of one
+            // cluster, reduced through distributed shared memory
+            const bool hy = spc > 100 && spc < 200, ck = spc > 200;
+            const int sp = ck ? spc - 200 : hy ? spc - 100 : spc < 0 ? -spc : spc;
             if (sp > KB || (sp > 1 && N % 4) || (sh.cg == 2 && spc > 1 && !hy)) continue;
+            if (ck && (sh.cg != 1 || sh.wt != 1 || sh.bk != 64 || sh.bn < 128 || ep.kind == EPI_ENTROPY)) continue;
             GemmPlan p = plan_gemm_bf16(M, N, K, ctx->num_sms, 16, sh.bn, sp, sh.wt, sh.bk, (spc < 0 || hy) ? 0 : 1,
-                                        sh.cg, hy ? 1 : 0);
-            if (p.splits != sp || p.cg != sh.cg || (p.hybrid != 0) != hy) continue;
+                                        sh.cg, hy ? 1 : 0, ck ? 1 : 0);
+            if (p.splits != sp || p.cg != sh.cg || (p.hybrid != 0) != hy || (p.ks > 1) != ck) continue;
             if (p.splits > 1 && ((size_t)p.splits * M * N > ctx->ws_floats ||
                                  (size_t)p.m_tiles * p.n_tiles * p.cg > ctx->n_tile_counters))
                 continue;

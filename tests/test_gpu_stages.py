@@ -161,3 +161,32 @@ def test_linear_bf16_hybrid_split_matches_fp64_matmul(M, N, K, tile_n, k_splits,
     assert np.all(err <= 1e-4 * bound + 1e-30), float((err / (bound + 1e-30)).max())
     Y1 = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=1, cta_pair=pair).cpu().numpy().astype(np.float64)
     assert np.all(np.abs(Y - Y1) <= 2e-4 * bound + 1e-30)
+
+
+@pytest.mark.parametrize("M,N,K,tile_n,k_splits", [
+    (256, 4096, 12288, 256, 4),   # the down projection's shape, four slices per cluster
+    (256, 4096, 4096, 128, 2),
+    (200, 1000, 520, 256, 3),     # ragged rows, N and K (9 k-blocks in 3 slices)
+    (96, 2048, 1024, 128, 4),     # fewer rows than the tile
+])
+def test_linear_bf16_cluster_k_split_matches_fp64_matmul(M, N, K, tile_n, k_splits):
+    """K slices of a tile as the CTAs of one cluster, reduced through distributed
+    shared memory, against the fp64 matmul and bound as above, and against the
+    plain single-slice plan."""
+    from streaming_decoding_b200 import linear_bf16
+    X = synth.normal(37, M * 13 + K, 1.0, (M, K), "bf16")
+    W = synth.normal(38, N * 5 + K, 0.02, (N, K), "bf16")
+    Xt = torch.from_numpy(X.view(np.int16)).cuda().view(torch.bfloat16)
+    Wt = torch.from_numpy(W.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=k_splits, cluster_k=True).cpu().numpy().astype(np.float64)
+    x64 = synth.bf16_bits_to_f32(X).astype(np.float64)
+    w64 = synth.bf16_bits_to_f32(W).astype(np.float64)
+    ref = x64 @ w64.T
+    bound = np.abs(x64) @ np.abs(w64).T
+    err = np.abs(Y - ref)
+    assert np.all(err <= 1e-4 * bound + 1e-30), float((err / (bound + 1e-30)).max())
+    Y1 = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=1).cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(Y - Y1) <= 2e-4 * bound + 1e-30)
+    # deterministic: the slices are summed in a fixed order
+    Y2 = linear_bf16(Xt, Wt, tile_n=tile_n, k_splits=k_splits, cluster_k=True).cpu().numpy().astype(np.float64)
+    assert np.array_equal(Y, Y2)
