@@ -369,7 +369,8 @@ def run_ours(a):
              "step_roofline_frac": round(step_floor_ms / (ms / a.steps), 4),
              "profile_ms_per_step": {k: round(v[0] / 10, 4) for k, v in prof.items() if v[1]},
              "e2e_wall_s": round(e_wall, 3),
-             "gemm_plans_rows%d" % (B * W): {k: rep.eng.gemm_plan(k, B * W) for k in gemm_shapes(dims, M)}}
+             "gemm_plans_rows%d" % (B * W): {k: rep.eng.gemm_plan(k, B * W) for k in gemm_shapes(dims, M)},
+             "gemm_schedules_rows%d" % (B * W): {k: rep.eng.gemm_schedule(k, B * W) for k in gemm_shapes(dims, M)}}
     if not a.quick and not a.no_extra and world == 1:
         extra.update(sweeps(rep, cfg, a))
     cpu = None

@@ -256,6 +256,14 @@ wedlm_status wedlm_autotune(wedlm_ctx* ctx, int32_t enable);
 wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* tile_w, int32_t* tile_n,
                              int32_t* k_splits, float* us);
 
+/* The schedule of the plan wedlm_gemm_plan reports, as a bit set: 1 CTA-pair
+ * tiles, 2 hybrid K split (only the last partial round split), 4 cluster K
+ * split (slices reduced through distributed shared memory), 8 K slices
+ * reduced by the co-resident slices of a tile (otherwise, when split, by the
+ * slice that finishes last), 16 two 128-row weight sub-tiles per CTA, 32
+ * 32-deep k-blocks.  WEDLM_ERR_STATE if no plan is recorded. */
+wedlm_status wedlm_gemm_schedule(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* schedule);
+
 /* Enable (1) or disable (0) per-kernel timing; enabling clears the totals. */
 wedlm_status wedlm_profile_enable(wedlm_ctx* ctx, int32_t on);
 

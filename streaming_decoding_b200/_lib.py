@@ -70,6 +70,7 @@ _SIGS = {
     "wedlm_debug_keep_logits": (c_i32, [c_vp, c_i32]),
     "wedlm_debug_residual": (c_i32, [c_vp, c_i32, c_vp, c_i32]),
     "wedlm_gemm_plan": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "wedlm_gemm_schedule": (c_i32, [c_vp, c_i32, c_i32, c_vp]),
     "wedlm_profile_read": (c_i32, [c_vp, c_vp, c_vp]),
     "wedlm_debug_read": (c_i32, [c_vp, c_i32, c_vp, c_i64]),
     "wedlm_debug_kv": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_vp, c_vp]),

@@ -164,6 +164,17 @@ class Engine:
                                       ctypes.byref(tn), ctypes.byref(ks), ctypes.byref(us))
         return (tw.value, tn.value, ks.value, round(us.value, 2)) if st == 0 else None
 
+    def gemm_schedule(self, kind: str, rows: int):
+        """Names of the schedule features of the recorded plan (CTA pairs, hybrid or
+        cluster K split, ...), or None."""
+        sc = ctypes.c_int32()
+        st = self.lib.wedlm_gemm_schedule(self.ctx, C["WEDLM_PROF_" + kind.upper()], rows, ctypes.byref(sc))
+        if st != 0:
+            return None
+        names = {1: "cta_pair", 2: "hybrid_split", 4: "cluster_split", 8: "co_resident_fixup",
+                 16: "two_weight_subtiles", 32: "bk32"}
+        return [n for bit, n in names.items() if sc.value & bit]
+
     def profile_enable(self, on: bool = True):
         _check(self.lib.wedlm_profile_enable(self.ctx, 1 if on else 0), "wedlm_profile_enable", self.ctx)
 

@@ -1343,6 +1343,17 @@ wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t
     return WEDLM_OK;
 }
 
+wedlm_status wedlm_gemm_schedule(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* schedule) {
+    if (!ctx || !schedule) return WEDLM_ERR_INVALID_ARG;
+    auto it = ctx->tuned.find({kind, rows});
+    if (it == ctx->tuned.end()) return fail(ctx, WEDLM_ERR_STATE, "no plan recorded for this kind and row count");
+    const GemmPlan& p = it->second.plan;
+    *schedule = (p.cg == 2 ? 1 : 0) | (p.hybrid ? 2 : 0) | (p.ks > 1 ? 4 : 0) |
+                (p.splits > 1 && p.coop && p.ks <= 1 && !p.hybrid ? 8 : 0) | (p.wt == 2 ? 16 : 0) |
+                (p.bk == 32 ? 32 : 0);
+    return WEDLM_OK;
+}
+
 wedlm_status wedlm_kernel_launches(const wedlm_ctx* ctx, int64_t* out) {
     if (!ctx || !out) return WEDLM_ERR_INVALID_ARG;
     *out = ctx->launches;
