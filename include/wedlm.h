@@ -216,6 +216,8 @@ typedef struct wedlm_seq_stats {
     int32_t active;         /* 1 while S < end */
 } wedlm_seq_stats;
 
+/* Copy the counters of `slot` into host `*out` (synchronises the stream).
+ * WEDLM_ERR_INVALID_ARG for a slot outside [0, max_batch) or a NULL `out`. */
 wedlm_status wedlm_get_stats(wedlm_ctx* ctx, int32_t slot, wedlm_seq_stats* out);
 
 /* Number of kernels this context has launched since creation (each launch

@@ -107,3 +107,25 @@ def test_null_arguments_are_rejected():
     assert lib.wedlm_linear_bf16(None, None, None, 16, 16, 7, None) == C["WEDLM_ERR_INVALID_ARG"]
     lib.wedlm_destroy(None)
     assert lib.wedlm_last_error(None) == b""
+
+
+
+def test_every_declaration_is_documented():
+    """Each function the header declares is preceded by a doc comment, its own
+    or that of the group of declarations it closes (argument meaning, layout,
+    ownership and errors live there)."""
+    import re
+    lines = open(os.path.join(ROOT, "include", "wedlm.h")).read().split("\n")
+    decl = re.compile(r"^[A-Za-z_][\w\s\*]*?\b(wedlm_\w+)\s*\(")
+    undocumented = []
+    for i, line in enumerate(lines):
+        m = decl.match(line)
+        if not m or line.startswith(("typedef", "#")):
+            continue
+        j = i - 1
+        while j >= 0 and (not lines[j].strip() or lines[j].startswith("#define")):
+            j -= 1
+        # a declaration right after another one shares that one's comment
+        if not (lines[j].rstrip().endswith("*/") or lines[j].rstrip().endswith(");")):
+            undocumented.append(m.group(1))
+    assert not undocumented, undocumented
