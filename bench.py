@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--quick", action="store_true", help="headline measurement only (for profiler runs)")
     ap.add_argument("--tile-n", type=int, default=0, help="kernel case: pin the GEMM tile width (0 = automatic)")
     ap.add_argument("--cta-pair", action="store_true", help="kernel case: CTA-pair GEMM tiles (tile width 128 or 256)")
+    ap.add_argument("--micro-cell", default=None,
+                    help="attn_micro: run one cell 'S,B' (attention, then the entropy pass at s=4) and exit "
+                         "(single-kernel captures)")
     ap.add_argument("--kernel-case", default=None,
                     help="run one projection of the batch-16 step (gemm_qkv|gemm_o|gemm_gate_up|gemm_down|"
                          "gemm_lm_head) three times through wedlm_linear_bf16, or 'attention' (3 decode steps of "
@@ -185,25 +188,23 @@ class Replica:
         return ms, self.committed(B) - c0, self.eng.kernel_launches() - l0
 
     def timed_e2e(self, params, steps):
-        """Same metric through the synchronous public call with pinned host buffers."""
+        """Same metric through the synchronous public call (wedlm_stream_step,
+        one call per step, each returning that step's committed tokens in pinned
+        host buffers), timed on the host wall clock."""
         torch = self.torch
         B, W = self.cfg["B"], self.cfg["W"]
         committed = torch.zeros((B, W), dtype=torch.int32).pin_memory().numpy()
         counts = torch.zeros(B, dtype=torch.int32).pin_memory().numpy()
         active = torch.zeros(1, dtype=torch.int32).pin_memory().numpy()
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         total = 0
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        start.record(self.stream)
         for _ in range(steps):
             self.eng.stream_step_into(params, committed, counts, active)
             total += int(counts.sum())
-        end.record(self.stream)
-        end.synchronize()
         wall = time.perf_counter() - t0
         d2h = (2 * B + B * W + 1) * 4
-        return start.elapsed_time(end), wall, total, d2h
+        return wall, total, d2h
 
     def profile(self, params, steps):
         self.eng.profile_enable(True)
@@ -280,6 +281,23 @@ def roofline(prof, dims, M, pk, workload):
     return out, bytes_tot, flops_tot
 
 
+def attention_roofline(prof, dims, B, W, S_mean, pk, steps):
+    """The decode attention's own fraction of HBM: K and V of every committed
+    position read once per sequence and layer (plus q and the output), over the
+    attention kernel's event-timed duration."""
+    ms, nl = prof.get("attention", (0.0, 0))
+    if nl == 0:
+        return None
+    hq, hkv, hd, L = dims["hq"], dims["hkv"], dims["hd"], dims["L"]
+    per_layer = B * (S_mean + W) * 2 * hkv * hd * 2 + 2 * B * W * hq * hd * 2
+    sec = ms / 1e3 / steps / L
+    ach = per_layer / sec / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm"], "unit": "GB/s",
+            "frac": round(ach / pk["hbm"], 4), "kernel": "attn_tc_kernel", "us_per_layer": round(sec * 1e6, 2),
+            "algorithmic_bytes_per_launch": round(per_layer),
+            "peak_source": f"{pk['src']} (hbm_gbs)"}
+
+
 def step_bytes_flops(dims, B, W, S_mean):
     """Algorithmic bytes and flops of one decode step (weights once, committed KV
     once per sequence and layer, logits once)."""
@@ -352,12 +370,18 @@ def run_ours(a):
     sb, sf = step_bytes_flops(dims, B, W, (S0 + S1) / 2)
     step_floor_ms = max(sb / (pk["hbm"] * 1e9), sf / (pk["tc_sus"] * 1e12)) * 1e3
 
-    # end to end through the public synchronous call
-    e2e_steps = max(20, a.steps // 3)
-    e_ms, e_wall, e_tok, d2h = rep.timed_e2e(prm, e2e_steps)
-    e2e_val = e_tok / (e_ms / 1e3)
+    # end to end through the public synchronous call: the same decode segment
+    # (prompts admitted again, the same warm-up steps, the same step count),
+    # host wall clock around the step calls
+    rep.admit(prompts, N, W)
+    rep.eng.stream_step_async(prm, a.warmup)
+    torch.cuda.synchronize()
     if dist:
-        e_max, e_sum = combine_ranks(dist, e_ms, e_tok, "cuda")
+        dist.barrier()
+    e_wall, e_tok, d2h = rep.timed_e2e(prm, a.steps)
+    e2e_val = e_tok / e_wall
+    if dist:
+        e_max, e_sum = combine_ranks(dist, e_wall * 1e3, e_tok, "cuda")
         e2e_val = e_sum / (e_max / 1e3)
 
     extra = {"prefill": {"tokens": rep.prefill_tokens, "seconds": round(rep.prefill_s, 3),
@@ -368,11 +392,16 @@ def run_ours(a):
              "step_ms_floor_algorithmic": round(step_floor_ms, 3),
              "step_roofline_frac": round(step_floor_ms / (ms / a.steps), 4),
              "profile_ms_per_step": {k: round(v[0] / 10, 4) for k, v in prof.items() if v[1]},
+             "attention_roofline": attention_roofline(prof, dims, B, W, (S0 + S1) / 2, pk, 10),
              "e2e_wall_s": round(e_wall, 3),
+             "e2e_committed_per_step": round(e_tok / a.steps, 3),
              "gemm_plans_rows%d" % (B * W): {k: rep.eng.gemm_plan(k, B * W) for k in gemm_shapes(dims, M)},
              "gemm_schedules_rows%d" % (B * W): {k: rep.eng.gemm_schedule(k, B * W) for k in gemm_shapes(dims, M)}}
     if not a.quick and not a.no_extra and world == 1:
-        extra.update(sweeps(rep, cfg, a))
+        if a.workload == "qwen3_8b_b16":
+            extra.update(sweeps(rep, cfg, a))
+        elif "lams" in cfg:
+            extra.update(knob_sweep(rep, cfg, a, prompts))
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.quick:
         cpu = cpu_baseline(cfg, budget_s=25.0)
@@ -393,8 +422,11 @@ def run_ours(a):
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": d2h,
-                    "api": "wedlm_stream_step (synchronous), pinned host outputs",
-                    "note": "decode steps take no host input (window and KV state stay on the device)"},
+                    "api": "wedlm_stream_step (synchronous, one call per step), pinned host outputs, host wall clock",
+                    "segment": "the same prompts, warm-up and step count as value",
+                    "note": "h2d_bytes_per_step is 0 because a decode step takes no host input: the window, "
+                            "the KV cache and every per-step size stay on the device; each step copies its "
+                            "committed tokens, counts and committed lengths back (d2h_bytes_per_step)"},
             "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "extra": extra}
@@ -440,6 +472,111 @@ def sweeps(rep, cfg, a):
                       "committed_per_step": round(com / n, 3)}
     out["decoders_batch16_x%g" % scale] = cmp_
     return out
+
+
+def knob_sweep(rep, cfg, a, prompts):
+    """lambda x tau sweep of a workload that lists them: the batch is admitted
+    once and each setting then decodes a stretch of steps in turn (the context
+    grows by the tokens committed in between)."""
+    from streaming_decoding_b200 import step_params
+    rep.admit(prompts, cfg["N"], cfg["W"])
+    out = {}
+    n = max(5, min(a.steps, 20))
+    for lam in cfg["lams"]:
+        for tau in cfg["taus"]:
+            prm = step_params(lam, tau, False, cfg["logit_scale"])
+            rep.eng.stream_step_async(prm, 2)
+            ms, com, _ = rep.timed_async(prm, n, cfg["B"])
+            out[f"lambda{lam:g}_tau{tau:g}"] = {"tok_per_s": round(com / (ms / 1e3), 2),
+                                               "ms_per_step": round(ms / n, 4),
+                                               "committed_per_step": round(com / n, 3)}
+    return {"lambda_tau_sweep": out, "lambda_tau_sweep_steps": n}
+
+
+# ------------------------------------------------------- C2 microbench --
+def run_micro(a):
+    """Single-layer decode-step microbench: the decode attention over random
+    page tables at committed lengths S x batch sizes B (W = 16 window rows, 32 /
+    8 heads, head_dim 128), and the vocabulary-151936 entropy + selection pass
+    over N(0, s^2) logits of the masked half of each window.  Each cell is
+    timed with CUDA events around single launches, after an L2 flush (a 256
+    MB write) before every launch; achieved GB/s counts the algorithmic bytes
+    (K and V of every position once, q and the output; the masked rows'
+    logits once)."""
+    import torch
+    from streaming_decoding_b200 import (attention_bf16, attention_error, attention_workspace, entropy_select_async,
+                                         step_params)
+    cfg = synth.CONFIGS["attn_micro"]
+    m = cfg["model"]
+    hq, hkv, V, W = m["hq"], m["hkv"], m["V"], cfg["W"]
+    pk = peaks()
+    torch.cuda.set_device(0)
+    g = torch.Generator(device="cuda").manual_seed(cfg["prompt_seed"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    iters = max(5, min(a.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    cells_S, cells_B, stds = cfg["S"], cfg["B"], cfg["logit_std"]
+    if a.micro_cell:
+        S1, B1 = (int(v) for v in a.micro_cell.split(","))
+        cells_S, cells_B, stds = (S1,), (B1,), (4.0,)
+    att = []
+    for S in cells_S:
+        for B in cells_B:
+            pps = (S + W + 15) // 16
+            pool = torch.randn(B * pps, 2, hkv, 16, 128, device="cuda", generator=g, dtype=torch.bfloat16)
+            table = torch.randperm(B * pps, device="cuda", generator=g).to(torch.int32).view(B, pps)
+            q = torch.randn(B * W, hq, 128, device="cuda", generator=g, dtype=torch.bfloat16)
+            Sd = torch.full((B,), S, dtype=torch.int32, device="cuda")
+            nd = torch.full((B,), W, dtype=torch.int32, device="cuda")
+            ws = attention_workspace(B, W, hq, hkv, S + W)
+            out = torch.empty_like(q)
+            ms = timed(lambda: attention_bf16(q, pool, table, Sd, nd, W, hq, hkv, S + W, ws, out=out))
+            torch.cuda.synchronize()
+            assert attention_error(ws) == 0
+            byt = B * (S + W) * hkv * 128 * 2 * 2 + 2 * B * W * hq * 128 * 2
+            att.append({"S": S, "B": B, "us": round(ms * 1e3, 2), "GB_s": round(byt / (ms / 1e3) / 1e9, 1),
+                        "frac": round(byt / (ms / 1e3) / 1e9 / pk["hbm"], 4)})
+            del pool, table, q, ws, out
+    ent = []
+    nf = cfg["n_filled"]
+    prm = step_params(0.1, 0.3, False, 1.0)
+    for s_ in stds:
+        for B in cells_B:
+            filled, _ = synth.window_state(2002, int(s_), B, W, nf, V, V - 1)
+            fd = torch.from_numpy(filled).cuda()
+            nd = torch.full((B,), W, dtype=torch.int32, device="cuda")
+            z = torch.randn(B * W, V, device="cuda", generator=g) * s_
+            outs = entropy_select_async(z, V, V - 1, fd, nd, W, prm)
+            ws = outs[3]
+            ms = timed(lambda: entropy_select_async(z, V, V - 1, fd, nd, W, prm, workspace=ws, out=outs[:3]))
+            byt = B * (W - nf) * V * 4
+            ent.append({"s": s_, "B": B, "us": round(ms * 1e3, 2), "GB_s": round(byt / (ms / 1e3) / 1e9, 1),
+                        "frac": round(byt / (ms / 1e3) / 1e9 / pk["hbm"], 4)})
+            del z
+    big = max(att, key=lambda c: (c["S"], c["B"]))
+    line = {"metric": "decode attention GB/s (largest cell)", "value": big["GB_s"], "unit": "GB/s", "n_gpus": 1,
+            "steps": iters, "warmup": 3, "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic (torch.randn K/V, q and logits; random page tables)",
+            "config": {"workload": "attn_micro: one layer, 32/8 heads, head_dim 128, W 16 (8 slots filled), "
+                                   "16-token pages; S x B grid; entropy over vocab 151936",
+                       "l2": "flushed before every launch (256 MB write)"},
+            "peak": {"hbm_gbs": pk["hbm"], "source": pk["src"]},
+            "attention": att, "entropy": ent}
+    print(json.dumps(line))
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -544,6 +681,8 @@ if __name__ == "__main__":
     args = parse()
     if args.kernel_case:
         kernel_case(args.kernel_case, args.tile_n, args.cta_pair)
+    elif args.workload == "attn_micro" and args.impl == "ours":
+        run_micro(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

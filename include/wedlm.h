@@ -57,6 +57,7 @@ typedef int32_t wedlm_status;
 #define WEDLM_ERR_STATE          -6  /* call not valid in the current state */
 #define WEDLM_ERR_UNSUPPORTED    -7  /* shape or dtype this build does not run */
 #define WEDLM_ERR_TIMEOUT        -8  /* a bounded device wait gave up */
+#define WEDLM_ERR_NONFINITE      -9  /* a masked slot's logits held a NaN or an infinity */
 
 #define WEDLM_DTYPE_F32   0
 #define WEDLM_DTYPE_BF16  1
@@ -188,7 +189,13 @@ typedef struct wedlm_step_params {
  *                 step at out_committed[b * max_window + 0 .. count-1]
  *   out_counts    [max_batch]: tokens committed by each slot this step
  *   out_active    [1]: slots still decoding after this step
- * Synchronises the context's stream before returning. */
+ * Synchronises the context's stream before returning.
+ * Non-finite logits: a masked slot whose logits hold a NaN or an infinity
+ * (a corrupted weight, an overflow) is never filled; its H~ reads as NaN and
+ * its argmax as -1 in the debug items, the other slots are decided among
+ * themselves (if none is valid, nothing is filled), the step's commit run is
+ * committed as usual, and the call returns WEDLM_ERR_NONFINITE (after
+ * wedlm_stream_step_async: the next call that reads the device error word). */
 wedlm_status wedlm_stream_step(wedlm_ctx* ctx, const wedlm_step_params* params,
                                int32_t* out_committed, int32_t* out_counts, int32_t* out_active);
 
@@ -266,6 +273,18 @@ wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t
  * 32-deep k-blocks.  WEDLM_ERR_STATE if no plan is recorded. */
 wedlm_status wedlm_gemm_schedule(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* schedule);
 
+/* Test hook: record a GEMM launch shape for (kind, rows) as if the autotuner
+ * had chosen it, so every epilogue can be checked under every schedule:
+ * tile_n activation rows per tile (16..256), k_splits slices of K (1..16) and
+ * `schedule` in the bits of wedlm_gemm_schedule (1 CTA pairs, 2 hybrid split,
+ * 4 cluster split, 8 co-resident fixup, 16 two weight sub-tiles, 32 32-deep
+ * k-blocks) plus 64 = the LM head's fused-entropy epilogue (kind LM_HEAD,
+ * k_splits 1).  WEDLM_ERR_INVALID_ARG when the shape cannot be built as asked
+ * or its K-split scratch does not fit the context.  Synchronises the stream;
+ * the next step runs eagerly. */
+wedlm_status wedlm_debug_set_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t tile_n, int32_t k_splits,
+                                  int32_t schedule);
+
 /* Enable (1) or disable (0) per-kernel timing; enabling clears the totals. */
 wedlm_status wedlm_profile_enable(wedlm_ctx* ctx, int32_t on);
 
@@ -304,7 +323,9 @@ wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t
  * partials and logits are never written (sampled steps and fp32 mode keep the
  * two-pass path).  enable = 1 makes every step write logits and run the
  * separate entropy pass, so WEDLM_DBG_LOGITS is valid after greedy bf16 steps
- * too (test hook; synchronises the stream). */
+ * too; enable = 2 makes every greedy bf16 step take the fused epilogue
+ * (whatever the timing choice at its row count would be); 0 restores the
+ * default (test hook; synchronises the stream). */
 wedlm_status wedlm_debug_keep_logits(wedlm_ctx* ctx, int32_t enable);
 
 /* Residual-stream capture for per-layer comparisons.  While enabled (1), every
@@ -323,6 +344,20 @@ wedlm_status wedlm_debug_get_window(wedlm_ctx* ctx, int32_t slot, uint8_t* fille
                                     int32_t cap, int32_t* n);
 wedlm_status wedlm_debug_set_window(wedlm_ctx* ctx, int32_t slot, const uint8_t* filled,
                                     const int32_t* tokens, int32_t n);
+
+/* Copy the first `bytes` of a weight tensor's device storage to host memory,
+ * as stored: WQ / WK / WV read the layer's fused [(hq + 2 hkv) * hd][d] block
+ * and WG / WU the fused [2 ffn][d] block, in the row order the bf16 epilogues
+ * use (RoPE partners / gate-up pairs in adjacent rows); other tensors as
+ * loaded.  Synchronises the stream. */
+wedlm_status wedlm_debug_read_weight(wedlm_ctx* ctx, int32_t tensor, int32_t layer, void* host_dst, int64_t bytes);
+
+/* Fault injection on the host side: overwrite entry `index` of slot `slot`'s
+ * device page table with `page`, unchecked (a value outside [0, num_pages)
+ * makes the kernels' own bounds checks fire: the step skips those accesses
+ * and returns WEDLM_ERR_DEVICE_ASSERT).  *old_page receives the previous
+ * entry (may be NULL).  Synchronises the stream. */
+wedlm_status wedlm_debug_set_page(wedlm_ctx* ctx, int32_t slot, int32_t index, int32_t page, int32_t* old_page);
 
 /* Stand-alone launches of single stages on caller-provided DEVICE buffers
  * (no context; the caller owns all memory; stream may be NULL).
@@ -349,7 +384,12 @@ wedlm_status wedlm_reorder_window(const uint8_t* filled, const int32_t* n, const
  *   argmax_j = lowest id attaining the max (never mask_id),
  *   htilde[b*stride+j] = H_j + lambda * j  (NaN for filled slots or j >= n[b]).
  * fill[b*stride+j] = 1 for slots chosen by the threshold / argmin rule, else 0;
- * argmax[b*stride+j] = argmax_j (or -1).  Device buffers, caller-owned. */
+ * argmax[b*stride+j] = argmax_j (or -1).  Device buffers, caller-owned.
+ * A masked slot whose logits hold a NaN or an infinity is invalid: htilde NaN,
+ * argmax -1, fill 0; the window's other slots are decided among themselves
+ * (none valid: nothing filled) and the call returns WEDLM_ERR_NONFINITE with
+ * every output written.  Synchronous; takes its scratch from cudaMallocAsync
+ * on `stream`. */
 wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t mask_id,
                                   const uint8_t* filled, const int32_t* n, int32_t n_seq, int32_t stride,
                                   const wedlm_step_params* params,
@@ -359,9 +399,11 @@ wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t ma
  * paper has no counterpart.)  It exists for callers that must not allocate
  * device memory: for example a runtime that has already reserved the device
  * for its own memory pool, where any further allocation fails or fragments
- * that pool, or a latency-critical thread that cannot risk the device
- * synchronisation an allocation may cause.  Same arguments, outputs and
- * device-pointer rules as wedlm_entropy_select; it allocates nothing.
+ * that pool, or a thread that must not take the allocator's locks or risk
+ * the device-wide synchronisation an allocation may cause.  Same arguments,
+ * outputs and device-pointer rules as wedlm_entropy_select; it allocates
+ * nothing.  Like wedlm_entropy_select it is synchronous: it waits for
+ * `stream` (only that stream, nothing device-wide) before returning.
  *
  * Its scratch is a fixed array inside the library image (about 1 MiB: room
  * for WEDLM_NOALLOC_MAX_ROWS rows), present on every GPU that loads the
@@ -369,17 +411,68 @@ wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t ma
  *   - n_seq * stride must be <= WEDLM_NOALLOC_MAX_ROWS; larger requests
  *     return WEDLM_ERR_INVALID_ARG without launching anything.
  *   - The first call on a device (with that device current) looks up the
- *     array's device address once; make that first call before any stream
- *     capture.
+ *     array's device address once and keeps it for the life of the process;
+ *     make that first call before any stream capture.  cudaDeviceReset
+ *     destroys the context that address belongs to: after a reset in the
+ *     same process, do not call this function again on that device.
  *   - Every call on a device shares the one array, and it keeps the previous
  *     call's contents (each call rewrites what it reads).  Calls whose work
  *     overlaps on the GPU (different streams or host threads without ordering
  *     between them) race on it and must be serialised by the caller. */
 #define WEDLM_NOALLOC_MAX_ROWS 4096
+/* (Non-finite logits: as for wedlm_entropy_select, WEDLM_ERR_NONFINITE.) */
 wedlm_status wedlm_entropy_select_noalloc(const float* logits, int32_t vocab, int32_t mask_id,
                                           const uint8_t* filled, const int32_t* n, int32_t n_seq, int32_t stride,
                                           const wedlm_step_params* params,
                                           float* htilde, int32_t* argmax, uint8_t* fill, void* stream);
+
+/* wedlm_entropy_select on caller-provided scratch, asynchronously: the call
+ * enqueues its kernels on `stream` and returns; the outputs are valid once the
+ * stream has been synchronised.  workspace: DEVICE memory, 256-byte aligned,
+ * at least wedlm_entropy_select_workspace_bytes(n_seq, stride) bytes; its first
+ * int32 is the call's device error word (cleared by the call itself; 3 = a
+ * masked slot's logits held a NaN or an infinity, the slot treated as in
+ * wedlm_entropy_select).  Nothing else in it needs initialising. */
+wedlm_status wedlm_entropy_select_workspace_bytes(int32_t n_seq, int32_t stride, int64_t* bytes);
+wedlm_status wedlm_entropy_select_async(const float* logits, int32_t vocab, int32_t mask_id,
+                                        const uint8_t* filled, const int32_t* n, int32_t n_seq, int32_t stride,
+                                        const wedlm_step_params* params, float* htilde, int32_t* argmax,
+                                        uint8_t* fill, void* workspace, int64_t workspace_bytes, void* stream);
+
+/* Reordered-causal GQA attention of window rows against a paged KV cache, on
+ * the bf16 tensor-core path (summary, section Method: after Topological
+ * Reordering the window runs a plain causal forward conditioned on the
+ * persistent KV cache).  This is the kernel the decode step runs per layer.
+ * All pointers are DEVICE memory owned by the caller, 256-byte aligned.
+ *   q          bf16 [n_seq * stride][n_heads][128]: query rows after RoPE;
+ *              row b * stride + r is physical window row r of sequence b.
+ *   kv_pool    bf16 [num_pages][2 (K, V)][n_kv_heads][16 tokens][128]: one
+ *              layer's page pool (K and V after RoPE for K).
+ *   page_table int32 [n_seq][pages_per_seq]: page of each 16-token block.
+ *   S, n       int32 [n_seq]: committed length and window rows of sequence b.
+ *              Window row r's own K/V must already sit at cache position
+ *              S[b] + r (the decode step's QKV epilogue writes them there).
+ *   out        bf16 [n_seq * stride][n_heads][128]: softmax(q K^T / sqrt(128)) V
+ *              of each row r < n[b] over cache positions 0 .. S[b] + r (rows
+ *              r >= n[b] are not written).
+ * max_ctx bounds S[b] + n[b] (it sizes the key chunks and the workspace);
+ * n_heads % n_kv_heads == 0; stride <= 1024.
+ * workspace: at least wedlm_attention_workspace_bytes(...) bytes; its first
+ * int32 is a device error word (1: a page id outside [0, num_pages) or more
+ * keys than max_ctx allows; 2: a bounded wait gave up).  The workspace must
+ * be zeroed (e.g. cudaMemsetAsync) before its first use; each call leaves it
+ * reusable as long as the error word stays 0.  After a nonzero error word,
+ * zero the whole workspace again.  Asynchronous: the call enqueues the kernel
+ * on `stream` and returns; out and the error word are valid once the stream
+ * has been synchronised.  WEDLM_ERR_INVALID_ARG for bad sizes, pointers or a
+ * too small workspace, WEDLM_ERR_CUDA if the launch fails. */
+wedlm_status wedlm_attention_workspace_bytes(int32_t n_seq, int32_t stride, int32_t n_heads, int32_t n_kv_heads,
+                                             int32_t max_ctx, int64_t* bytes);
+wedlm_status wedlm_attention_bf16(const void* q, const void* kv_pool, int32_t num_pages, int32_t n_heads,
+                                  int32_t n_kv_heads, const int32_t* page_table, int32_t pages_per_seq,
+                                  const int32_t* S, const int32_t* n, int32_t n_seq, int32_t stride,
+                                  int32_t max_ctx, void* out, void* workspace, int64_t workspace_bytes,
+                                  void* stream);
 
 /* Dense projection on the bf16 tensor-core path: Y = X * W^T with X bf16
  * [M][K], W bf16 [N][K] (nn.Linear layout), Y fp32 [M][N], all DEVICE

@@ -19,8 +19,8 @@ Everything is computed in float64 with numpy; weights arrive as float32 or as
 bf16 bit patterns (uint16) and are widened exactly.  Readings of points the
 pages leave open are marked R1..R16 (the same numbering as the design notes):
   R1  the commit run is the run of slots already filled when the forward starts;
-      their K/V come from this forward (Summary/Method: "its KV states depend
-      only on earlier tokens under the causal mask").
+      their K/V come from this forward (Summary/Method: with a causal mask those
+      K/V are functions of earlier tokens alone, so they can be cached at once).
   R2  the logits of a mask row predict that row's own slot.
   R3  entropy is Shannon entropy in nats of softmax(logit_scale * logits).
   R4  H~_j = H_j + lambda * j with j the slot's offset from the window start

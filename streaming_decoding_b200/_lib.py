@@ -81,6 +81,15 @@ _SIGS = {
                                      c_vp, c_vp, c_vp, c_vp]),
     "wedlm_entropy_select_noalloc": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_i32,
                                              ctypes.POINTER(StepParams), c_vp, c_vp, c_vp, c_vp]),
+    "wedlm_entropy_select_workspace_bytes": (c_i32, [c_i32, c_i32, ctypes.POINTER(c_i64)]),
+    "wedlm_entropy_select_async": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_i32, c_i32, ctypes.POINTER(StepParams),
+                                           c_vp, c_vp, c_vp, c_vp, c_i64, c_vp]),
+    "wedlm_debug_set_page": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_vp]),
+    "wedlm_debug_read_weight": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_i64]),
+    "wedlm_debug_set_plan": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_i32, c_i32]),
+    "wedlm_attention_workspace_bytes": (c_i32, [c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(c_i64)]),
+    "wedlm_attention_bf16": (c_i32, [c_vp, c_vp, c_i32, c_i32, c_i32, c_vp, c_i32, c_vp, c_vp, c_i32, c_i32, c_i32,
+                                     c_vp, c_vp, c_i64, c_vp]),
     "wedlm_linear_bf16": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_vp]),
     "wedlm_linear_bf16_plan": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]),
     "wedlm_linear_bf16_sched": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_vp]),

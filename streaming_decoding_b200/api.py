@@ -143,8 +143,12 @@ class Engine:
         _check(self.lib.wedlm_autotune(self.ctx, 1 if enable else 0), "wedlm_autotune", self.ctx)
 
     def keep_logits(self, enable: bool = True):
-        """Write logits every step (two-pass entropy) so debug_read("LOGITS") is valid in bf16 mode."""
+        """Test hook: True writes logits every step (two-pass LM head + entropy)."""
         _check(self.lib.wedlm_debug_keep_logits(self.ctx, 1 if enable else 0), "wedlm_debug_keep_logits", self.ctx)
+
+    def force_fused_entropy(self, enable: bool = True):
+        """Test hook: greedy bf16 steps always take the fused LM-head entropy epilogue."""
+        _check(self.lib.wedlm_debug_keep_logits(self.ctx, 2 if enable else 0), "wedlm_debug_keep_logits", self.ctx)
 
     def debug_capture(self, enable: bool = True):
         """Keep the residual stream at every layer boundary of each decode step (test hook)."""
@@ -221,6 +225,36 @@ class Engine:
         _check(self.lib.wedlm_debug_set_window(self.ctx, slot, f.ctypes.data, t.ctypes.data, len(f)),
                "wedlm_debug_set_window", self.ctx)
 
+    SCHEDULE_BITS = {"cta_pair": 1, "hybrid_split": 2, "cluster_split": 4, "co_resident_fixup": 8,
+                     "two_weight_subtiles": 16, "bk32": 32, "fused_entropy": 64}
+
+    def set_plan(self, kind: str, rows: int, tile_n: int, k_splits: int = 1, schedule=()):
+        """Test hook: pin the GEMM launch shape of a projection kind at `rows` (see
+        wedlm_debug_set_plan); `schedule` is a list of names.  Returns False if the
+        shape cannot be built as asked."""
+        bits = 0
+        for name in schedule:
+            bits |= self.SCHEDULE_BITS[name]
+        st = self.lib.wedlm_debug_set_plan(self.ctx, C["WEDLM_PROF_" + kind.upper()], rows, tile_n, k_splits, bits)
+        if st == C["WEDLM_ERR_INVALID_ARG"]:
+            return False
+        _check(st, "wedlm_debug_set_plan", self.ctx)
+        return True
+
+    def read_weight(self, kind: int, layer: int, nbytes: int) -> np.ndarray:
+        """Test hook: the first `nbytes` of a weight tensor's device storage (uint8)."""
+        out = np.empty(nbytes, np.uint8)
+        _check(self.lib.wedlm_debug_read_weight(self.ctx, kind, layer, out.ctypes.data, nbytes),
+               "wedlm_debug_read_weight", self.ctx)
+        return out
+
+    def set_page(self, slot: int, index: int, page: int) -> int:
+        """Overwrite one device page-table entry, unchecked (fault-injection hook); returns the old entry."""
+        old = ctypes.c_int32()
+        _check(self.lib.wedlm_debug_set_page(self.ctx, slot, index, page, ctypes.byref(old)),
+               "wedlm_debug_set_page", self.ctx)
+        return int(old.value)
+
 
 def _stream_handle(stream) -> int:
     if stream is None:
@@ -270,6 +304,63 @@ def entropy_select_noalloc(logits, vocab: int, mask_id: int, filled, n, stride: 
                                                     stride, ctypes.byref(params), _ptr(ht), _ptr(am), _ptr(fill),
                                                     _stream_handle(stream)), "wedlm_entropy_select_noalloc")
     return ht, am, fill
+
+
+def entropy_select_async(logits, vocab: int, mask_id: int, filled, n, stride: int, params: StepParams,
+                         workspace=None, out=None, stream=None):
+    """Asynchronous entropy selection on caller scratch (wedlm_entropy_select_async).
+    Returns (htilde, argmax, fill, workspace); the first int32 of the workspace is
+    the call's device error word (read it after synchronising)."""
+    import torch
+    n_seq = filled.shape[0]
+    dev = logits.device
+    lib = _lib.load()
+    if workspace is None:
+        nb = ctypes.c_int64()
+        _check(lib.wedlm_entropy_select_workspace_bytes(n_seq, stride, ctypes.byref(nb)),
+               "wedlm_entropy_select_workspace_bytes")
+        workspace = torch.zeros(int(nb.value), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = (torch.empty((n_seq, stride), dtype=torch.float32, device=dev),
+               torch.empty((n_seq, stride), dtype=torch.int32, device=dev),
+               torch.empty((n_seq, stride), dtype=torch.uint8, device=dev))
+    ht, am, fill = out
+    _check(lib.wedlm_entropy_select_async(_ptr(logits), vocab, mask_id, _ptr(filled), _ptr(n), n_seq, stride,
+                                          ctypes.byref(params), _ptr(ht), _ptr(am), _ptr(fill), _ptr(workspace),
+                                          workspace.numel(), _stream_handle(stream)), "wedlm_entropy_select_async")
+    return ht, am, fill, workspace
+
+
+def attention_workspace(n_seq: int, stride: int, n_heads: int, n_kv_heads: int, max_ctx: int, device="cuda"):
+    """A zeroed workspace for attention_bf16 (uint8 CUDA tensor)."""
+    import torch
+    nb = ctypes.c_int64()
+    _check(_lib.load().wedlm_attention_workspace_bytes(n_seq, stride, n_heads, n_kv_heads, max_ctx, ctypes.byref(nb)),
+           "wedlm_attention_workspace_bytes")
+    return torch.zeros(int(nb.value), dtype=torch.uint8, device=device)
+
+
+def attention_bf16(q, kv_pool, page_table, S, n, stride: int, n_heads: int, n_kv_heads: int, max_ctx: int,
+                   workspace, out=None, stream=None):
+    """Asynchronous reordered-causal paged attention (wedlm_attention_bf16).
+    q [n_seq*stride, n_heads, 128] bf16; kv_pool [pages, 2, n_kv_heads, 16, 128]
+    bf16; page_table [n_seq, pages_per_seq] int32; S, n [n_seq] int32; workspace
+    from attention_workspace().  Returns `out`; read attention_error(workspace)
+    after synchronising."""
+    import torch
+    n_seq = page_table.shape[0]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_lib.load().wedlm_attention_bf16(_ptr(q), _ptr(kv_pool), kv_pool.shape[0], n_heads, n_kv_heads,
+                                            _ptr(page_table), page_table.shape[1], _ptr(S), _ptr(n), n_seq, stride,
+                                            max_ctx, _ptr(out), _ptr(workspace), workspace.numel(),
+                                            _stream_handle(stream)), "wedlm_attention_bf16")
+    return out
+
+
+def attention_error(workspace) -> int:
+    """The device error word of an attention workspace (synchronise first)."""
+    return int(workspace[:4].view(dtype=__import__("torch").int32)[0].item())
 
 
 def linear_bf16(X, W, stream=None, tile_n: int = 0, k_splits: int = 0, cta_pair: bool = False,

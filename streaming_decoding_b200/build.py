@@ -29,7 +29,12 @@ def nvcc() -> str:
 
 
 def _flags(verbose_ptxas: bool):
-    f = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
+    # -dlcm=cg: plain global loads bypass L1.  Kernels of a step start early
+    # (programmatic dependent launch) and read slot state, row metadata and
+    # activations that the kernel just before them writes, and a context's
+    # buffers may reuse addresses another context freed; an L1 line filled
+    # before such a write could otherwise be read stale (common.cuh).
+    f = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-Xptxas", "-dlcm=cg",
          "-I" + os.path.join(ROOT, "include")] + ARCH
     if verbose_ptxas:
         f += ["-Xptxas", "-v"]
@@ -47,6 +52,13 @@ def _stale(obj: str, src: str) -> bool:
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
+    # objects built with other flags are rebuilt
+    stamp = os.path.join(BUILD, "flags.txt")
+    flags_now = " ".join(_flags(False))
+    if not os.path.exists(stamp) or open(stamp).read() != flags_now:
+        force = True
+        with open(stamp, "w") as f:
+            f.write(flags_now)
     jobs = []
     objs = []
     for s in SOURCES:

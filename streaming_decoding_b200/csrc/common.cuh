@@ -39,9 +39,18 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Global memory is never read through the non-coherent read-only path (no
+// __ldg, no const __restrict__ kernel parameters): a context's buffers may
+// reuse the addresses of buffers another context freed earlier in the
+// process, and kernels started early by programmatic dependent launch do not
+// begin from clean caches, so a stale line of the old contents could be
+// returned.  Plain loads are compiled to bypass L1 (-dlcm=cg, see build.py)
+// and are served coherently from L2; bulk data moves by TMA, also through L2.
+
 // Device error word codes (mirrors of the wedlm_status values they map to).
-constexpr int kErrBounds = 1;   // a bounds check refused an access
-constexpr int kErrTimeout = 2;  // a bounded wait gave up
+constexpr int kErrBounds = 1;     // a bounds check refused an access
+constexpr int kErrTimeout = 2;    // a bounded wait gave up
+constexpr int kErrNonFinite = 3;  // a masked slot's logits held a NaN or an infinity
 
 __device__ __forceinline__ void set_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
@@ -151,7 +160,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits at most ~limit_cycles (about one second at B200 clocks); gives up early
-// once any CTA has recorded an error, so a failing launch drains quickly.
+// once any CTA has recorded a timeout (a stall somewhere), so a launch that
+// cannot finish drains quickly.  Bounds and non-finite errors are only
+// recorded: the work that follows them completes normally.
+__device__ __forceinline__ bool stalled(int* err) {
+    return err && *reinterpret_cast<volatile int*>(err) == kErrTimeout;
+}
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* err,
                                                   long long limit_cycles = 2000000000LL) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -159,7 +174,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 1023u) == 0) {
-            if (err && *reinterpret_cast<volatile int*>(err) != 0) return false;
+            if (stalled(err)) return false;
             if (clock64() - t0 > limit_cycles) {
                 set_error(err, kErrTimeout);
                 return false;

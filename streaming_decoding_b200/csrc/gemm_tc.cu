@@ -85,8 +85,8 @@ template <int BN, int WT, int BK, int CG> struct PCfg {
 // once per unit into shared memory so the element loops issue their global
 // loads in batches (no load waits behind a store of the previous element).
 struct RowMeta {
-    int live;      // row < M and not padding
-    int pos;       // logical position (RoPE)
+    int live;      // row < M (and < the device row count) and not padding
+    int pos;       // logical position (RoPE); with a row map, the row the result goes to
     long long kv;  // element offset of (layer, page, K, head 0, token) in the pool; -1 if out of range
 };
 
@@ -196,7 +196,7 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint32_t bar, uint32_t
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if ((it & 1023u) == 1023u) {
-            if (err && *reinterpret_cast<volatile int*>(err) != 0) return false;
+            if (stalled(err)) return false;
             if (clock64() - t0 > 2000000000LL) {
                 set_error(err, kErrTimeout);
                 return false;
@@ -312,25 +312,33 @@ __device__ __forceinline__ bool epi_all(bool v) {
 }
 
 // Fill meta[0..BN) for activation rows m0..m0+BN-1 (the 128 epilogue threads).
+// Live activation rows of a launch: M, or fewer when the rows are counted on
+// the device (read after the dependency wait: the previous kernel writes it).
+__device__ __forceinline__ int live_rows(const EpiParams& ep, int M) {
+    return ep.m_count ? min(M, __ldcg(ep.m_count)) : M;
+}
+
 template <int BN>
 __device__ __forceinline__ void fill_row_meta(const EpiParams& ep, int m0, int M, RowMeta* meta, int et) {
+    const int Ml = live_rows(ep, M);
     for (int k = et; k < BN; k += 128) {
         const int m = m0 + k;
         RowMeta rmeta{0, 0, -1};
         int slot = 0, r = m;
-        if (m < M && (!ep.check_rows || ep.rm.live(m, slot, r))) {
+        if (m < Ml && (!ep.check_rows || ep.rm.live(m, slot, r))) {
             rmeta.live = 1;
+            if (ep.row_map) rmeta.pos = __ldcg(ep.row_map + m);
             if (ep.kind == EPI_QKV_ROPE) {
-                const int pos = __ldg(ep.rs.pos + m);
+                const int pos = __ldcg(ep.rs.pos + m);
                 if (pos < 0 || pos >= ep.rope_max_pos) {
                     set_error(ep.err, kErrBounds);
                     rmeta.live = 0;
                 } else {
                     rmeta.pos = pos;
-                    const int p = __ldg(ep.ss.S + slot) + r;
+                    const int p = __ldcg(ep.ss.S + slot) + r;
                     const int pidx = p / kPage;
                     const int page = pidx < ep.ss.pages_per_seq
-                                         ? __ldg(ep.ss.page_table + (int64_t)slot * ep.ss.pages_per_seq + pidx)
+                                         ? __ldcg(ep.ss.page_table + (int64_t)slot * ep.ss.pages_per_seq + pidx)
                                          : -1;
                     if (page < 0 || page >= ep.kvl.num_pages) {
                         set_error(ep.err, kErrBounds);
@@ -378,7 +386,7 @@ __device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, i
         case EPI_STORE:
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-                if (live[k]) out[(int64_t)(mbase + k) * N + n] = v[k];
+                if (live[k]) out[(int64_t)(ep.row_map ? meta[kbase + k].pos : mbase + k) * N + n] = v[k];
             break;
         case EPI_RESIDUAL: {
             float x[16];
@@ -416,7 +424,7 @@ __device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, i
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const RowMeta rmk = meta[kbase + k];
-                cs[k] = (rot && live[k]) ? __ldg(rope + (int64_t)rmk.pos * 64 + i) : make_float2(1.f, 0.f);
+                cs[k] = (rot && live[k]) ? __ldcg(rope + (int64_t)rmk.pos * 64 + i) : make_float2(1.f, 0.f);
                 dst[k] = live[k] ? qkv_dst(act, pool, hq, hkv, head, mbase + k, rmk.kv) : nullptr;
             }
 #pragma unroll
@@ -439,8 +447,8 @@ __device__ __forceinline__ void epilogue16(const EpiParams& ep, int n0, int n, i
 // rows, this warp's 32 vocab ids (one per lane, id n) reduce to the partial
 // (max, sum e^(z-max), sum e^(z-max)(z-max), lowest argmax) of z = scale * v
 // over valid ids (n < N, n != mask id); lane k stores row k's partial.
-__device__ __forceinline__ void entropy16(const EpiParams& ep, const float (&v)[16], bool valid, int n, int mbase,
-                                          int M, int pidx, int lane) {
+__device__ __forceinline__ void entropy16(const EpiParams& ep, const float (&v)[16], bool valid, int n, int kbase,
+                                          const RowMeta* meta, int m0, int pidx, int lane) {
     const float scale = ep.scale;
     float4* const epart = ep.epart;
     const int npart = ep.npart;
@@ -463,8 +471,9 @@ __device__ __forceinline__ void entropy16(const EpiParams& ep, const float (&v)[
         int a = (valid && z == m) ? n : INT_MAX;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
-        const int row = mbase + k;
-        if (lane == k && row < M) epart[(int64_t)row * npart + pidx] = make_float4(m, e, t, __int_as_float(a));
+        const RowMeta rk = meta[kbase + k];
+        const int row = ep.row_map ? rk.pos : m0 + kbase + k;
+        if (lane == k && rk.live) epart[(int64_t)row * npart + pidx] = make_float4(m, e, t, __int_as_float(a));
     }
 }
 
@@ -505,8 +514,8 @@ __device__ __forceinline__ void epi_pre(const EpiParams& ep, int n0, int n, cons
         for (int u = 0; u < 8; ++u) {
             const RowMeta rmu = meta[krow[u]];
             const int64_t base = (int64_t)rmu.pos * 64 + i;
-            p.c0[u] = (rot && p.live[u]) ? __ldg(rope + base) : make_float2(1.f, 0.f);
-            p.c1[u] = (rot && p.live[u]) ? __ldg(rope + base + 1) : make_float2(1.f, 0.f);
+            p.c0[u] = (rot && p.live[u]) ? __ldcg(rope + base) : make_float2(1.f, 0.f);
+            p.c1[u] = (rot && p.live[u]) ? __ldcg(rope + base + 1) : make_float2(1.f, 0.f);
             p.dst[u] = p.live[u] ? qkv_dst(act, pool, hq, hkv, head, mrow[u], rmu.kv) : nullptr;
         }
     }
@@ -613,6 +622,7 @@ __device__ __forceinline__ void staged_epilogue(const EpiParams& ep, int M, int 
                 krow[u] = c + rl;
                 mrow[u] = m0 + c + rl;
                 okr[u] = nok && mrow[u] < M;
+                if (KIND == EPI_STORE && ep.row_map && okr[u] && meta[krow[u]].live) mrow[u] = meta[krow[u]].pos;
             }
             EpiPre p;
             epi_pre<KIND>(ep, nw, nn, mrow, krow, okr, meta, N, p);
@@ -685,6 +695,7 @@ __device__ __forceinline__ bool cluster_epilogue(const EpiParams& ep, int M, int
             krow[u] = c * COLS + rl;
             mrow[u] = m0 + c * COLS + rl;
             okr[u] = nok && mrow[u] < M;
+            if (KIND == EPI_STORE && ep.row_map && okr[u] && meta[krow[u]].live) mrow[u] = meta[krow[u]].pos;
         }
         EpiPre p;
         epi_pre<KIND>(ep, n0, nn, mrow, krow, okr, meta, N, p);
@@ -737,7 +748,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     uint64_t* acce = accf + 2;
     uint64_t* rfree = acce + 2;  // cluster K split: the other CTAs' rings are idle
     uint64_t* rfull = rfree + 1; // cluster K split: the other slices of this CTA's chunks have arrived
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rfull + 1);
+    uint64_t* mma_drain = rfull + 1;  // every MMA issued has completed (before TMEM is released)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
     int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);  // epilogue warps: this CTA reduces the tile
     RowMeta* meta = reinterpret_cast<RowMeta*>(smem + STAGES * C::STAGE_BYTES + 256);
     float* epi_stage = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + 256 + C::META_BYTES);
@@ -764,6 +776,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         }
         mbar_init(rfree, g.ks > 1 ? g.ks - 1 : 1);
         mbar_init(rfull, g.ks > 1 ? 4 * (g.ks - 1) : 1);
+        mbar_init(mma_drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -848,6 +861,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                 // lands before this CTA may exit.
                 for (uint32_t f = it > (uint32_t)STAGES ? it - STAGES : 0u; f < it && ok; ++f)
                     ok = mbar_wait_bounded(smem_u32(&empty[f % STAGES]), (f / STAGES) & 1u, err);
+            } else {
+                // Drain: the loads of the last stages issued land before this CTA
+                // may exit (they complete whether or not anything consumed them).
+                for (uint32_t f = it > (uint32_t)STAGES ? it - STAGES : 0u; f < it; ++f)
+                    mbar_wait_bounded(smem_u32(&full[f % STAGES]), (f / STAGES) & 1u, nullptr, 200000000LL);
             }
         } else {
             griddep_wait();
@@ -857,11 +875,19 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         griddep_wait();
         griddep_launch();
         if (lane == 0 && rank == 0) {  // a pair's MMAs are issued by its even CTA
-            constexpr uint32_t idesc = idesc_bf16(BM * CG, BN);
+            constexpr uint32_t idesc_full = idesc_bf16(BM * CG, BN);
+            const int Ml = live_rows(g.ep, g.M);
             uint32_t it = 0, j = 0;
             bool ok = true;
             for (int u = u0; u < units && ok; u += ustep, ++j) {
-                const int nkb = unit_of(g, u, KB).nkb;
+                const Unit un = unit_of(g, u, KB);
+                const int nkb = un.nkb;
+                // rows counted on the device: a tile past them issues no MMA, a
+                // single-CTA tile narrows its MMA to the live rows (multiple of 16)
+                const int live = Ml - (un.tile % g.m_tiles) * BN;
+                const bool skip = live <= 0;
+                const uint32_t idesc = (CG == 1 && live > 0 && live < BN)
+                                           ? idesc_bf16(BM, (live + 15) & ~15) : idesc_full;
                 const uint32_t b = j % NACC, use = j / NACC;
                 const bool free_acc = CG == 2 ? mbar_wait_cluster_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err)
                                               : mbar_wait_bounded(smem_u32(&acce[b]), (use & 1u) ^ 1u, err);
@@ -878,17 +904,25 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     tc_fence_after();
                     const uint8_t* a = sA + s * C::A_STAGE_BYTES;
                     const uint8_t* bb = sB + s * C::B_STAGE_BYTES;
+                    if (!skip) {
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
+                        for (int kk = 0; kk < BK / 16; ++kk)
 #pragma unroll
-                        for (int w = 0; w < WT; ++w)
-                            umma_bf16<CG>(d + w * BN, sdesc_k<BK>(a + w * SUB_A_BYTES + kk * 32),
-                                          sdesc_k<BK>(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                            for (int w = 0; w < WT; ++w)
+                                umma_bf16<CG>(d + w * BN, sdesc_k<BK>(a + w * SUB_A_BYTES + kk * 32),
+                                              sdesc_k<BK>(bb + kk * 32), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
                     umma_commit<CG>(&empty[s]);
                 }
                 umma_commit<CG>(&accf[b]);
             }
+            // TMEM is released after the final barrier: every MMA issued (also
+            // after a failed wait) must have completed by then
+            umma_commit<CG>(mma_drain);
+            mbar_wait_bounded(smem_u32(mma_drain), 0, nullptr, 200000000LL);
         }
+        if (CG == 2 && lane == 0 && rank == 1)  // the pair's commit reaches this CTA's barrier too
+            mbar_wait_bounded(smem_u32(mma_drain), 0, nullptr, 200000000LL);
     } else {
         griddep_wait();
         griddep_launch();
@@ -923,7 +957,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     for (int c = 0; c < BN; c += 16) {
                         float v[16];
                         tmem_ld16(tacc + (uint32_t)(w * BN + c), v);
-                        entropy16(g.ep, v, valid, n, m0 + c, g.M, pidx, lane);
+                        entropy16(g.ep, v, valid, n, c, meta, m0, pidx, lane);
                     }
                 }
                 tc_fence_before();
@@ -1005,6 +1039,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                     EpiParams pe = g.ep;
                     pe.kind = EPI_STORE;
                     pe.out = plane;
+                    pe.row_map = nullptr;  // planes are indexed by the tile's own rows
                     auto rel = [&]() {
                         tc_fence_before();
                         __syncwarp();
@@ -1022,7 +1057,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 #pragma unroll
                             for (int k = 0; k < 16; ++k) {
                                 const int m = m0 + c + k;
-                                if (m < g.M && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
+                                if (meta[c + k].live && n < g.N) plane[(int64_t)m * g.N + n] = v[k];
                             }
                         }
                     }
@@ -1111,6 +1146,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                             krow[u] = rr < BN ? rr : 0;
                             mrow[u] = m0 + rr;
                             okr[u] = nok && rr < r1 && mrow[u] < g.M;
+                            if (g.ep.kind == EPI_STORE && g.ep.row_map && okr[u] && meta[krow[u]].live)
+                                mrow[u] = meta[krow[u]].pos;
                         }
                         epilogue_vec4x8(g.ep, nw, nn, mrow, krow, okr, meta, acc, g.N);
                     }

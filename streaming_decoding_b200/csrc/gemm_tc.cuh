@@ -38,6 +38,12 @@ struct EpiParams {
     int npart = 0;
     int mask_id = -1;
     float scale = 1.f;
+    // Activation rows counted on the device (LM head over the packed masked
+    // rows): rows >= *m_count are neither computed nor stored (the MMA width of
+    // a tile shrinks to cover the live rows when the plan has no CTA pairs),
+    // and an EPI_STORE / EPI_ENTROPY result of row m goes to row row_map[m].
+    const int* m_count = nullptr;
+    const int32_t* row_map = nullptr;
     float* ws = nullptr;       // split-K partial planes [splits][M][N]
     int* counters = nullptr;   // per-tile tickets; zero before and after every launch
     int* err = nullptr;

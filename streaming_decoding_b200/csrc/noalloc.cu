@@ -12,7 +12,9 @@
 // The array lives in every GPU that loads the library until the process
 // exits.  In host code its name is only a host-side stand-in for the symbol,
 // never a device address, so the device address is fetched with
-// cudaGetSymbolAddress once per device (with that device current) and cached.
+// cudaGetSymbolAddress once per device (with that device current) and cached
+// for the life of the process (a cudaDeviceReset would invalidate it; the
+// header tells callers not to use this entry point after one).
 #include <mutex>
 
 #include "kernels.cuh"
@@ -24,9 +26,11 @@ namespace {
 constexpr int kChunks = 16;
 constexpr size_t kPartBytes = (size_t)WEDLM_NOALLOC_MAX_ROWS * kChunks * sizeof(float4);
 constexpr size_t kMaskBytes = (size_t)WEDLM_NOALLOC_MAX_ROWS;
+constexpr size_t kErrBytes = 256;
 
-// Scratch shared by every call on a device: the partials, then the row flags.
-static __device__ __align__(256) unsigned char g_select_scratch[kPartBytes + kMaskBytes];
+// Scratch shared by every call on a device: the partials, the row flags, then
+// the call's error word.
+static __device__ __align__(256) unsigned char g_select_scratch[kPartBytes + kMaskBytes + kErrBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
@@ -64,15 +68,20 @@ extern "C" wedlm_status wedlm_entropy_select_noalloc(const float* logits, int32_
     if (s) return s;
     float4* part = reinterpret_cast<float4*>(base);
     uint8_t* rowmask = base + kPartBytes;
+    int* errw = reinterpret_cast<int*>(base + kPartBytes + kMaskBytes);
     cudaStream_t st = (cudaStream_t)stream;
     const int rows = n_seq * stride;
     StepKnobs kn{params->lambda, params->tau, params->logit_scale, params->tau_none};
-    // Every row flag is rewritten below and every partial of a flagged row is
-    // written before it is read, so nothing left by an earlier call is used.
+    // Every row flag is rewritten below, every partial of a flagged row is
+    // written before it is read and the error word is cleared first, so
+    // nothing left by an earlier call is used.
+    cudaMemsetAsync(errw, 0, sizeof(int), st);
     launch_rowmask_from_filled(filled, n, n_seq, stride, rowmask, st);
     launch_entropy_partials(logits, 1, 0, vocab, vocab, mask_id, params->logit_scale, rowmask, rows, kChunks, part, st);
-    launch_select_only(part, kChunks, filled, n, n_seq, stride, kn, htilde, argmax, fill, st);
+    launch_select_only(part, kChunks, filled, n, n_seq, stride, kn, htilde, argmax, fill, errw, st);
+    int herr = 0;
+    cudaMemcpyAsync(&herr, errw, sizeof(int), cudaMemcpyDeviceToHost, st);
     if (cudaGetLastError() != cudaSuccess) return WEDLM_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return WEDLM_ERR_CUDA;
-    return WEDLM_OK;
+    return herr == kErrNonFinite ? WEDLM_ERR_NONFINITE : herr ? WEDLM_ERR_DEVICE_ASSERT : WEDLM_OK;
 }

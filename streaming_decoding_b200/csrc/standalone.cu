@@ -1,6 +1,7 @@
 // Stand-alone launches of single stages on caller-provided device buffers.
 // They run exactly the kernels the decode step runs, so the tests can check
 // each stage against the CPU oracle in isolation.
+#include <algorithm>
 #include <string>
 
 #include "gemm_tc.cuh"
@@ -33,30 +34,153 @@ wedlm_status wedlm_reorder_window(const uint8_t* filled, const int32_t* n, const
     return sync_status(st);
 }
 
+// Entropy selection on caller-provided scratch: `part` [rows][kChunks]
+// partials, `rowmask` [rows] flags, `err` one device int (zeroed here).
+static void enqueue_entropy_select(const float* logits, int32_t vocab, int32_t mask_id, const uint8_t* filled,
+                                   const int32_t* n, int32_t n_seq, int32_t stride, const wedlm_step_params* params,
+                                   float* htilde, int32_t* argmax, uint8_t* fill, float4* part, uint8_t* rowmask,
+                                   int* err, cudaStream_t st) {
+    const int rows = n_seq * stride;
+    StepKnobs kn{params->lambda, params->tau, params->logit_scale, params->tau_none};
+    cudaMemsetAsync(err, 0, sizeof(int), st);
+    launch_rowmask_from_filled(filled, n, n_seq, stride, rowmask, st);
+    launch_entropy_partials(logits, 1, 0, vocab, vocab, mask_id, params->logit_scale, rowmask, rows, kChunks, part, st);
+    launch_select_only(part, kChunks, filled, n, n_seq, stride, kn, htilde, argmax, fill, err, st);
+}
+
+static bool entropy_args_ok(int32_t vocab, int32_t mask_id, int32_t n_seq, int32_t stride,
+                            const wedlm_step_params* params) {
+    return n_seq >= 0 && stride >= 1 && stride <= kMaxWindow && vocab >= 2 && mask_id >= -1 && mask_id < vocab &&
+           params && params->logit_scale > 0.f;
+}
+
+static size_t entropy_ws_bytes(int32_t n_seq, int32_t stride) {
+    const size_t rows = (size_t)n_seq * stride;
+    return 256 + (rows * kChunks * sizeof(float4) + 255) / 256 * 256 + (rows + 255) / 256 * 256;
+}
+
 wedlm_status wedlm_entropy_select(const float* logits, int32_t vocab, int32_t mask_id, const uint8_t* filled,
                                   const int32_t* n, int32_t n_seq, int32_t stride, const wedlm_step_params* params,
                                   float* htilde, int32_t* argmax, uint8_t* fill, void* stream) {
-    if (n_seq < 0 || stride < 1 || stride > kMaxWindow || vocab < 2 || mask_id < -1 || mask_id >= vocab || !params)
-        return WEDLM_ERR_INVALID_ARG;
-    if (!(params->logit_scale > 0.f)) return WEDLM_ERR_INVALID_ARG;
+    if (!entropy_args_ok(vocab, mask_id, n_seq, stride, params)) return WEDLM_ERR_INVALID_ARG;
     if (n_seq == 0) return WEDLM_OK;
     if (!logits || !filled || !n || !htilde || !argmax || !fill) return WEDLM_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
+    const size_t bytes = entropy_ws_bytes(n_seq, stride);
+    char* ws = nullptr;
+    if (cudaMallocAsync((void**)&ws, bytes, st) != cudaSuccess) return WEDLM_ERR_OOM_DEVICE;
+    const size_t rows = (size_t)n_seq * stride;
+    float4* part = reinterpret_cast<float4*>(ws + 256);
+    uint8_t* rowmask = reinterpret_cast<uint8_t*>(ws + 256 + (rows * kChunks * sizeof(float4) + 255) / 256 * 256);
+    enqueue_entropy_select(logits, vocab, mask_id, filled, n, n_seq, stride, params, htilde, argmax, fill, part,
+                           rowmask, reinterpret_cast<int*>(ws), st);
+    int herr = 0;
+    cudaMemcpyAsync(&herr, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+    cudaFreeAsync(ws, st);
+    wedlm_status s = sync_status(st);
+    if (s) return s;
+    return herr == kErrNonFinite ? WEDLM_ERR_NONFINITE : herr ? WEDLM_ERR_DEVICE_ASSERT : WEDLM_OK;
+}
+
+wedlm_status wedlm_entropy_select_workspace_bytes(int32_t n_seq, int32_t stride, int64_t* bytes) {
+    if (!bytes || n_seq < 0 || stride < 1 || stride > kMaxWindow) return WEDLM_ERR_INVALID_ARG;
+    *bytes = (int64_t)entropy_ws_bytes(n_seq, stride);
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_entropy_select_async(const float* logits, int32_t vocab, int32_t mask_id, const uint8_t* filled,
+                                        const int32_t* n, int32_t n_seq, int32_t stride,
+                                        const wedlm_step_params* params, float* htilde, int32_t* argmax,
+                                        uint8_t* fill, void* workspace, int64_t workspace_bytes, void* stream) {
+    if (!entropy_args_ok(vocab, mask_id, n_seq, stride, params)) return WEDLM_ERR_INVALID_ARG;
+    if (n_seq == 0) return WEDLM_OK;
+    if (!logits || !filled || !n || !htilde || !argmax || !fill || !workspace) return WEDLM_ERR_INVALID_ARG;
+    if (workspace_bytes < (int64_t)entropy_ws_bytes(n_seq, stride) || ((uintptr_t)workspace & 255))
+        return WEDLM_ERR_INVALID_ARG;
+    char* ws = static_cast<char*>(workspace);
+    const size_t rows = (size_t)n_seq * stride;
+    enqueue_entropy_select(logits, vocab, mask_id, filled, n, n_seq, stride, params, htilde, argmax, fill,
+                           reinterpret_cast<float4*>(ws + 256),
+                           reinterpret_cast<uint8_t*>(ws + 256 + (rows * kChunks * sizeof(float4) + 255) / 256 * 256),
+                           reinterpret_cast<int*>(ws), (cudaStream_t)stream);
+    return cudaGetLastError() == cudaSuccess ? WEDLM_OK : WEDLM_ERR_CUDA;
+}
+
+// Workspace of the stand-alone attention: [0, 256) the device error word;
+// then the merge tickets, the (m, l) partials and the O partials of the key
+// chunks, each piece 256-byte aligned.
+struct AttnWs {
+    int kv_chunk = 0, max_splits = 0, tiles = 0;
+    size_t off_tickets = 0, off_ml = 0, off_o = 0, bytes = 0;
+};
+
+static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+static bool attn_ws_layout(int n_seq, int stride, int hq, int hkv, int max_ctx, AttnWs* w) {
+    if (n_seq < 1 || stride < 1 || stride > kMaxWindow * 16 || hq < 1 || hkv < 1 || hq % hkv || hq / hkv > 128 ||
+        max_ctx < 1)
+        return false;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int g = hq / hkv;
+    w->kv_chunk = attn_kv_chunk_for(n_seq, stride, hq, hkv, max_ctx, sms);
+    w->max_splits = (max_ctx + w->kv_chunk - 1) / w->kv_chunk;
+    if (w->max_splits > attn_max_splits()) return false;
+    const int rt = attn_rows_per_tile(g);
+    w->tiles = (stride + rt - 1) / rt;
+    const size_t rows = (size_t)n_seq * stride;
+    w->off_tickets = 256;
+    w->off_ml = w->off_tickets + round256((size_t)n_seq * hkv * std::max(w->tiles, 1) * sizeof(int));
+    const size_t parts = w->max_splits > 1 ? rows * hq * w->max_splits : 0;
+    w->off_o = w->off_ml + round256(parts * sizeof(float2));
+    w->bytes = w->off_o + round256(parts * 128 * sizeof(float));
+    return true;
+}
+
+wedlm_status wedlm_attention_workspace_bytes(int32_t n_seq, int32_t stride, int32_t n_heads, int32_t n_kv_heads,
+                                             int32_t max_ctx, int64_t* bytes) {
+    AttnWs w;
+    if (!bytes || !attn_ws_layout(n_seq, stride, n_heads, n_kv_heads, max_ctx, &w)) return WEDLM_ERR_INVALID_ARG;
+    *bytes = (int64_t)w.bytes;
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_attention_bf16(const void* q, const void* kv_pool, int32_t num_pages, int32_t n_heads,
+                                  int32_t n_kv_heads, const int32_t* page_table, int32_t pages_per_seq,
+                                  const int32_t* S, const int32_t* n, int32_t n_seq, int32_t stride, int32_t max_ctx,
+                                  void* out, void* workspace, int64_t workspace_bytes, void* stream) {
+    AttnWs w;
+    if (!attn_ws_layout(n_seq, stride, n_heads, n_kv_heads, max_ctx, &w)) return WEDLM_ERR_INVALID_ARG;
+    if (!q || !kv_pool || !page_table || !S || !n || !out || !workspace || num_pages < 1 || pages_per_seq < 1)
+        return WEDLM_ERR_INVALID_ARG;
+    if (workspace_bytes < (int64_t)w.bytes) return WEDLM_ERR_INVALID_ARG;
+    if (((uintptr_t)q | (uintptr_t)kv_pool | (uintptr_t)out | (uintptr_t)workspace) & 255) return WEDLM_ERR_INVALID_ARG;
+    const int hq = n_heads, hkv = n_kv_heads;
+    KVLayout kvl;
+    kvl.layer_stride = (int64_t)num_pages * 2 * hkv * kPage * 128;
+    kvl.hkv = hkv;
+    kvl.hd = 128;
+    kvl.num_pages = num_pages;
+    CUtensorMap tm_kv, tm_q, tm_qd;
     const int rows = n_seq * stride;
-    uint8_t* rowmask = nullptr;
-    float4* part = nullptr;
-    if (cudaMallocAsync((void**)&rowmask, rows, st) != cudaSuccess) return WEDLM_ERR_OOM_DEVICE;
-    if (cudaMallocAsync((void**)&part, (size_t)rows * kChunks * sizeof(float4), st) != cudaSuccess) {
-        cudaFreeAsync(rowmask, st);
-        return WEDLM_ERR_OOM_DEVICE;
-    }
-    StepKnobs kn{params->lambda, params->tau, params->logit_scale, params->tau_none};
-    launch_rowmask_from_filled(filled, n, n_seq, stride, rowmask, st);
-    launch_entropy_partials(logits, 1, 0, vocab, vocab, mask_id, params->logit_scale, rowmask, rows, kChunks, part, st);
-    launch_select_only(part, kChunks, filled, n, n_seq, stride, kn, htilde, argmax, fill, st);
-    cudaFreeAsync(part, st);
-    cudaFreeAsync(rowmask, st);
-    return sync_status(st);
+    if (!make_kv_tmap(&tm_kv, (const bf16*)kv_pool, kvl, 1) ||
+        !make_q_tmap(&tm_q, (const bf16*)q, rows, hq, hkv, false) ||
+        !make_q_tmap(&tm_qd, (const bf16*)q, rows, hq, hkv, true))
+        return WEDLM_ERR_CUDA;
+    SlotState ss{};
+    ss.S = const_cast<int32_t*>(S);
+    ss.n = const_cast<int32_t*>(n);
+    ss.page_table = const_cast<int32_t*>(page_table);
+    ss.pages_per_seq = pages_per_seq;
+    RowMap rm{0, stride, n};
+    char* ws = static_cast<char*>(workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    const cudaError_t e =
+        launch_attn_bf16(tm_kv, tm_q, tm_qd, kvl, 0, hq, hkv, (bf16*)out, (float*)(ws + w.off_o),
+                         (float2*)(ws + w.off_ml), (int*)(ws + w.off_tickets), n_seq, stride, w.kv_chunk,
+                         w.max_splits, ss, rm, (int*)ws, st);
+    return e == cudaSuccess ? WEDLM_OK : WEDLM_ERR_CUDA;
 }
 
 wedlm_status wedlm_linear_bf16(const void* X, const void* W, float* Y, int32_t M, int32_t N, int32_t K, void* stream) {

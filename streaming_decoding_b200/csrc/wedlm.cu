@@ -34,6 +34,7 @@ using namespace wedlm;
 namespace {
 
 constexpr int kEntropyChunks = 16;
+constexpr size_t kEvictBytes = (size_t)256 << 20;  // > 2x the 126 MB L2
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -138,12 +139,17 @@ struct wedlm_ctx {
     StepKey graph_key, eager_key;
     float* logits = nullptr;
     size_t logits_floats = 0;
+    void* evict = nullptr;        // zeroed buffer larger than L2, swept before every tuning launch
+    float* evict_sink = nullptr;
     float4* ent_part = nullptr;
     float2* samp_part = nullptr;  // Gumbel-max partials of sampled fills
     float* dbg_resid = nullptr;   // test hook: residual stream before each layer and after the last [L+1][Mdec][d]
     float4* lm_part = nullptr;    // fused LM-head entropy partials [Mdec][lm_npart]
+    int32_t* lm_rows = nullptr;   // [Mdec] physical row of each packed masked row (LM-head input)
+    int32_t* lm_count = nullptr;  // [1] masked rows of the current step
     int lm_npart = 0;
     bool keep_logits = false;     // test hook: write logits (unfused LM head + entropy pass)
+    bool force_fused = false;     // test hook: greedy bf16 steps always take the fused LM-head entropy
     std::map<int, bool> fuse_choice;  // rows -> fused LM-head entropy is the faster path
     bool capturing = false;           // a step is being captured into a CUDA graph: no timing runs
     float* attn_po = nullptr;
@@ -303,15 +309,15 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
     const int KB = (K + 63) / 64;
     // Time one plan: `reps` launches (the first discarded), each after an L2
     // eviction: in a step every projection's weights arrive cold from HBM (the
-    // other layers' weights stream through L2 in between), so the logits scratch
-    // (larger than L2 at full size; not live while the projections run) is
-    // rewritten before each launch.  Minimum or median of the timed launches.
+    // other layers' weights stream through L2 in between), so a buffer twice
+    // the size of L2 is read before each launch.  Minimum or median of the
+    // timed launches.
     auto time_plan = [&](const GemmPlan& p, int reps, bool median) -> float {
         const CUtensorMap* tx = xmap(ctx, X, (uint64_t)ctx->Mmax, (uint64_t)K, (uint32_t)(p.bn / p.cg), p.bk);
         if (!tx) return 1e30f;
         std::vector<float> ts;
         for (int rep = 0; rep < reps; ++rep) {
-            cudaMemsetAsync(ctx->logits, 0, ctx->logits_floats * sizeof(float), ctx->stream);
+            launch_l2_evict(ctx->evict, kEvictBytes, ctx->evict_sink, ctx->num_sms, ctx->stream);
             cudaEventRecord(e0, ctx->stream);
             if (launch_gemm_bf16(tmW->of(p.bk), *tx, M, N, K, p, ep, ctx->stream) != cudaSuccess) {
                 cudaGetLastError();
@@ -367,8 +373,10 @@ void autotune_shape(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WM
 wedlm_status gemm_bf16(wedlm_ctx* ctx, int kind, const void* X, const wedlm_ctx::WMap* tmW, int M, int N, int K,
                        EpiParams ep, bool tune = true) {
     GemmPlan p;
-    const bool tuned = ctx->tuned.count({tune_kind(kind, ep), M}) > 0;
-    if (ctx->autotune && tune && (tuned || !ctx->capturing)) {  // no timing runs inside a graph capture
+    const auto rec = ctx->tuned.find({tune_kind(kind, ep), M});
+    if (rec != ctx->tuned.end() && tune) {  // a recorded (tuned or pinned) plan
+        p = rec->second.plan;
+    } else if (ctx->autotune && tune && !ctx->capturing) {  // no timing runs inside a graph capture
         autotune_shape(ctx, kind, X, tmW, M, N, K, ep);
         p = ctx->tuned[{tune_kind(kind, ep), M}].plan;
     } else {
@@ -438,6 +446,8 @@ wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
     if (ctx->attn_tickets)
         CK(cudaMemsetAsync(ctx->attn_tickets, 0, ctx->n_attn_tickets * sizeof(int), ctx->stream));
     if (code == kErrTimeout) return fail(ctx, WEDLM_ERR_TIMEOUT, "a bounded device wait timed out");
+    if (code == kErrNonFinite)
+        return fail(ctx, WEDLM_ERR_NONFINITE, "a masked slot's logits held a NaN or an infinity (slot not filled)");
     return fail(ctx, WEDLM_ERR_DEVICE_ASSERT, "a device bounds check fired");
 }
 
@@ -513,7 +523,6 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
     bf16* qb = (bf16*)ctx->q;
     bf16* ao = (bf16*)ctx->attn_out;
     bf16* act = (bf16*)ctx->act;
-    const int rt = attn_rows_per_tile(ctx->hq / ctx->hkv);
     EpiParams base;
     base.check_rows = 1;
     base.rm = rm;
@@ -537,9 +546,12 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
         const int ms = decode ? ctx->attn_max_splits : 1;
         {
             ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
-            launch_attn_bf16(ctx->tm_kv, ctx->tm_q, ctx->tm_q_dual, ctx->kvl, l, ctx->hq, ctx->hkv, ao,
-                             ctx->attn_po, ctx->attn_pml, ctx->attn_tickets, n_entries, stride, kc, ms, ctx->ss, rm,
-                             ctx->err, ctx->stream);
+            const cudaError_t ae =
+                launch_attn_bf16(ctx->tm_kv, ctx->tm_q, ctx->tm_q_dual, ctx->kvl, l, ctx->hq, ctx->hkv, ao,
+                                 ctx->attn_po, ctx->attn_pml, ctx->attn_tickets, n_entries, stride, kc, ms, ctx->ss, rm,
+                                 ctx->err, ctx->stream);
+            if (ae != cudaSuccess)
+                return fail(ctx, WEDLM_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(ae));
         }
         e.kind = EPI_RESIDUAL;
         e.out = ctx->x;
@@ -555,10 +567,20 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
         e.out = ctx->x;
         if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_DOWN, act, &ctx->tm_d[l], M, ctx->d, ctx->F, e, decode))) return s;
         capture_residual(ctx, l + 1, M, decode);
-        const float* gnext = (l + 1 < ctx->L) ? ctx->attn_norm[l + 1] : ctx->final_norm;
-        {
+        if (l + 1 == ctx->L) {
+            // final norm: the LM head reads the masked rows only, packed (a
+            // prefill has no LM head)
+            if (!decode) break;
+            MaskedRows mr;
+            mr.nf = ctx->ss.nf;
+            mr.row_map = ctx->lm_rows;
+            mr.count = ctx->lm_count;
+            mr.n_entries = n_entries;
             ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
-            launch_rmsnorm_bf16(ctx->x, h, gnext, eps, M, ctx->d, rm, ctx->stream);
+            launch_rmsnorm_bf16(ctx->x, h, ctx->final_norm, eps, M, ctx->d, rm, ctx->stream, mr);
+        } else {
+            ProfScope ps(ctx, WEDLM_PROF_RESIDUAL_NORM);
+            launch_rmsnorm_bf16(ctx->x, h, ctx->attn_norm[l + 1], eps, M, ctx->d, rm, ctx->stream);
         }
     }
     return WEDLM_OK;
@@ -594,6 +616,8 @@ wedlm_status lm_head_entropy(wedlm_ctx* ctx, const wedlm_step_params* prm, int M
         e.npart = ctx->lm_npart;
         e.mask_id = ctx->cfg.mask_id;
         e.scale = prm->logit_scale;
+        e.m_count = ctx->lm_count;  // the packed masked rows (final norm)
+        e.row_map = ctx->lm_rows;
         if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, &ctx->tm_lm, M, ctx->V, ctx->d, e))) return s;
         ProfScope ps(ctx, WEDLM_PROF_ENTROPY);
         launch_entropy_merge(ctx->lm_part, ctx->lm_npart, ctx->rowmask, M, kEntropyChunks, ctx->ent_part,
@@ -604,6 +628,8 @@ wedlm_status lm_head_entropy(wedlm_ctx* ctx, const wedlm_step_params* prm, int M
         EpiParams e;
         e.kind = EPI_STORE;
         e.out = ctx->logits;
+        e.m_count = ctx->lm_count;  // the packed masked rows (final norm)
+        e.row_map = ctx->lm_rows;
         if ((s = gemm_bf16(ctx, WEDLM_PROF_GEMM_LM_HEAD, ctx->h, &ctx->tm_lm, M, ctx->V, ctx->d, e))) return s;
     } else {
         if ((size_t)M * ctx->V > ctx->logits_floats) return fail(ctx, WEDLM_ERR_STATE, "logits buffer too small");
@@ -649,7 +675,10 @@ wedlm_status enqueue_step_kernels(wedlm_ctx* ctx, const wedlm_step_params* prm, 
     bool fused = false;
     if (fusable) {
         auto it = ctx->fuse_choice.find(M);
-        if (it == ctx->fuse_choice.end()) {
+        if (ctx->force_fused) {
+            it = ctx->fuse_choice.emplace(M, true).first;
+            it->second = true;
+        } else if (it == ctx->fuse_choice.end()) {
             bool choice = M <= 64;
             if (ctx->autotune && !ctx->capturing) {
                 // both variants once to tune their GEMMs, then once more each, timed
@@ -773,6 +802,7 @@ const char* wedlm_status_str(wedlm_status s) {
         case WEDLM_ERR_STATE: return "invalid state for this call";
         case WEDLM_ERR_UNSUPPORTED: return "unsupported shape or dtype";
         case WEDLM_ERR_TIMEOUT: return "bounded device wait timed out";
+        case WEDLM_ERR_NONFINITE: return "non-finite logits in a masked slot";
         default: return "unknown status";
     }
 }
@@ -910,26 +940,18 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     sa.add((void**)&ctx->rs.tok, (size_t)Mmax * 4);
     sa.add((void**)&ctx->rs.perm, (size_t)Mmax * 4);
     sa.add((void**)&ctx->rowmask, (size_t)Mmax);
+    sa.add((void**)&ctx->lm_rows, (size_t)ctx->Mdec * 4);
+    sa.add((void**)&ctx->lm_count, 4);
     sa.add((void**)&ctx->ids_dev, (size_t)ctx->chunk * 4);
     // Attention key chunks for decode: fixed per context (a sequence's result
-    // does not depend on its batch neighbours), sized so that a full batch at
-    // half the context length gives about two CTAs per SM; 256 to 2048 keys.
+    // does not depend on its batch neighbours).
     if (ctx->bf16) {
         const int g = ctx->hq / ctx->hkv;
         const int rt = attn_rows_per_tile(g);
         const int tiles = (maxW + rt - 1) / rt;
-        const long long pairs = (long long)B * tiles * ctx->hkv;
-        const long long blocks = pairs * std::max(1, (ctx->max_ctx / 2 + 63) / 64);
-        long long cb = (blocks + 2LL * ctx->num_sms - 1) / (2LL * ctx->num_sms);
-        // at least four blocks per chunk: below that the per-CTA setup and the
-        // merge of many partials outweigh the extra parallelism (small batches)
-        cb = std::max(4LL, std::min(cb, 32LL));
-        // at most attn_max_splits() chunks per row tile (the merge keeps its weights on chip)
-        const long long ms_cap = attn_max_splits();
-        cb = std::max(cb, ((long long)ctx->max_ctx + 64 * ms_cap - 1) / (64 * ms_cap));
-        ctx->attn_kv_chunk = (int)(cb * 64);
+        ctx->attn_kv_chunk = attn_kv_chunk_for(B, maxW, ctx->hq, ctx->hkv, ctx->max_ctx, ctx->num_sms);
         ctx->attn_max_splits = (ctx->max_ctx + ctx->attn_kv_chunk - 1) / ctx->attn_kv_chunk;
-        ctx->n_attn_tickets = (size_t)pairs;
+        ctx->n_attn_tickets = (size_t)B * tiles * ctx->hkv;
         sa.add((void**)&ctx->attn_tickets, ctx->n_attn_tickets * sizeof(int));
     }
     if (sa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
@@ -971,6 +993,10 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     ctx->logits_floats = (size_t)ctx->Mdec * (size_t)V;
     xa.add((void**)&ctx->logits, ctx->logits_floats * 4);
     xa.add((void**)&ctx->ent_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float4));
+    if (ctx->bf16) {
+        xa.add(&ctx->evict, kEvictBytes);
+        xa.add((void**)&ctx->evict_sink, sizeof(float));
+    }
     xa.add((void**)&ctx->samp_part, (size_t)ctx->Mdec * kEntropyChunks * sizeof(float2));
     if (ctx->bf16) {
         ctx->lm_npart = ((V + 255) / 256) * 2 * 4;  // 4 per 128 vocab rows, for 128- or 256-row tiles
@@ -1343,6 +1369,42 @@ wedlm_status wedlm_gemm_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t
     return WEDLM_OK;
 }
 
+wedlm_status wedlm_debug_set_plan(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t tile_n, int32_t k_splits,
+                                  int32_t schedule) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (!ctx->bf16) return fail(ctx, WEDLM_ERR_UNSUPPORTED, "GEMM plans exist in bf16 mode only");
+    int N = 0, K = 0;
+    switch (kind) {
+        case WEDLM_PROF_GEMM_QKV: N = ctx->Nqkv; K = ctx->d; break;
+        case WEDLM_PROF_GEMM_O: N = ctx->d; K = ctx->hq * ctx->hd; break;
+        case WEDLM_PROF_GEMM_GATE_UP: N = 2 * ctx->F; K = ctx->d; break;
+        case WEDLM_PROF_GEMM_DOWN: N = ctx->d; K = ctx->F; break;
+        case WEDLM_PROF_GEMM_LM_HEAD: N = ctx->V; K = ctx->d; break;
+        default: return fail(ctx, WEDLM_ERR_INVALID_ARG, "kind is not a GEMM kind");
+    }
+    if (rows < 1 || rows > ctx->Mmax || k_splits < 1 || k_splits > 16 || (schedule & ~127) ||
+        (tile_n != 16 && tile_n != 32 && tile_n != 64 && tile_n != 128 && tile_n != 256))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad rows, tile_n, k_splits or schedule");
+    const bool entropy = (schedule & 64) != 0;
+    if (entropy && (kind != WEDLM_PROF_GEMM_LM_HEAD || k_splits != 1))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "the entropy epilogue is the LM head's, over whole K");
+    const int cg = (schedule & 1) ? 2 : 1, hy = (schedule & 2) ? 1 : 0, ck = (schedule & 4) ? 1 : 0;
+    const int coop = (schedule & 8) ? 1 : 0, wt = (schedule & 16) ? 2 : 1, bk = (schedule & 32) ? 32 : 64;
+    GemmPlan p = plan_gemm_bf16(rows, N, K, ctx->num_sms, 16, tile_n, k_splits, wt, bk, coop, cg, hy, ck);
+    const bool same = p.bn == tile_n && p.splits == k_splits && p.cg == cg && p.wt == wt && p.bk == bk &&
+                      (p.ks > 1) == (ck != 0) && (p.hybrid != 0) == (hy != 0) &&
+                      (k_splits == 1 || cg == 2 || hy || ck || p.coop == coop);
+    if (!same) return fail(ctx, WEDLM_ERR_INVALID_ARG, "the launch shape cannot be built as asked");
+    if (p.splits > 1 && ((size_t)p.splits * rows * N > ctx->ws_floats ||
+                         (size_t)p.m_tiles * p.n_tiles * p.cg > ctx->n_tile_counters))
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "the plan's K-split scratch does not fit");
+    CK(cudaStreamSynchronize(ctx->stream));
+    ctx->tuned[{entropy ? kind + 1000 : kind, rows}] = {p, -2.f};
+    drop_graph(ctx);
+    ctx->eager_key = wedlm_ctx::StepKey();
+    return WEDLM_OK;
+}
+
 wedlm_status wedlm_gemm_schedule(wedlm_ctx* ctx, int32_t kind, int32_t rows, int32_t* schedule) {
     if (!ctx || !schedule) return WEDLM_ERR_INVALID_ARG;
     auto it = ctx->tuned.find({kind, rows});
@@ -1461,11 +1523,12 @@ wedlm_status wedlm_debug_kv(wedlm_ctx* ctx, int32_t slot, int32_t layer, int32_t
 wedlm_status wedlm_debug_keep_logits(wedlm_ctx* ctx, int32_t enable) {
     if (!ctx) return WEDLM_ERR_INVALID_ARG;
     CK(cudaStreamSynchronize(ctx->stream));
-    if (ctx->keep_logits != (enable != 0)) {
-        drop_graph(ctx);
-        ctx->eager_key = wedlm_ctx::StepKey();  // the next step runs eagerly (it may tune)
-    }
-    ctx->keep_logits = enable != 0;
+    if (enable < 0 || enable > 2) return fail(ctx, WEDLM_ERR_INVALID_ARG, "enable must be 0, 1 or 2");
+    drop_graph(ctx);
+    ctx->eager_key = wedlm_ctx::StepKey();  // the next step runs eagerly (it may tune)
+    if (ctx->force_fused && enable != 2) ctx->fuse_choice.clear();  // choose afresh
+    ctx->keep_logits = enable == 1;
+    ctx->force_fused = enable == 2;
     return WEDLM_OK;
 }
 
@@ -1512,6 +1575,43 @@ wedlm_status wedlm_debug_get_window(wedlm_ctx* ctx, int32_t slot, uint8_t* fille
         CK(cudaMemcpy(filled, ctx->ss.filled + (size_t)slot * ctx->maxW, m, cudaMemcpyDeviceToHost));
         CK(cudaMemcpy(tokens, ctx->ss.token + (size_t)slot * ctx->maxW, (size_t)m * 4, cudaMemcpyDeviceToHost));
     }
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_read_weight(wedlm_ctx* ctx, int32_t tensor, int32_t layer, void* host_dst, int64_t bytes) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (!host_dst || bytes < 0) return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad destination");
+    if (tensor_slot(ctx, tensor, layer) < 0) return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad tensor id or layer");
+    const size_t elt = ctx->elt, d = ctx->d, qd = (size_t)ctx->hq * ctx->hd, kd = (size_t)ctx->hkv * ctx->hd;
+    const char* src = nullptr;
+    size_t avail = 0;
+    switch (tensor) {
+        case WEDLM_T_EMBED: src = (const char*)ctx->embed; avail = (size_t)ctx->V * d * elt; break;
+        case WEDLM_T_LM_HEAD: src = (const char*)ctx->lm_head; avail = (size_t)ctx->V * d * elt; break;
+        case WEDLM_T_FINAL_NORM: src = (const char*)ctx->final_norm; avail = d * 4; break;
+        case WEDLM_T_ATTN_NORM: src = (const char*)ctx->attn_norm[layer]; avail = d * 4; break;
+        case WEDLM_T_FFN_NORM: src = (const char*)ctx->ffn_norm[layer]; avail = d * 4; break;
+        case WEDLM_T_WQ: case WEDLM_T_WK: case WEDLM_T_WV:
+            src = (const char*)ctx->wqkv[layer]; avail = (qd + 2 * kd) * d * elt; break;
+        case WEDLM_T_WO: src = (const char*)ctx->wo[layer]; avail = d * qd * elt; break;
+        case WEDLM_T_WG: case WEDLM_T_WU: src = (const char*)ctx->wgu[layer]; avail = 2 * (size_t)ctx->F * d * elt; break;
+        case WEDLM_T_WD: src = (const char*)ctx->wd[layer]; avail = d * ctx->F * elt; break;
+        default: return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad tensor id");
+    }
+    if ((size_t)bytes > avail) return fail(ctx, WEDLM_ERR_INVALID_ARG, "too many bytes for this tensor");
+    CK(cudaStreamSynchronize(ctx->stream));
+    CK(cudaMemcpy(host_dst, src, (size_t)bytes, cudaMemcpyDeviceToHost));
+    return WEDLM_OK;
+}
+
+wedlm_status wedlm_debug_set_page(wedlm_ctx* ctx, int32_t slot, int32_t index, int32_t page, int32_t* old_page) {
+    if (!ctx) return WEDLM_ERR_INVALID_ARG;
+    if (slot < 0 || slot >= ctx->maxB || index < 0 || index >= ctx->pages_per_seq)
+        return fail(ctx, WEDLM_ERR_INVALID_ARG, "bad slot or page index");
+    CK(cudaStreamSynchronize(ctx->stream));
+    int32_t* entry = ctx->ss.page_table + (size_t)slot * ctx->pages_per_seq + index;
+    if (old_page) CK(cudaMemcpy(old_page, entry, 4, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(entry, &page, 4, cudaMemcpyHostToDevice));
     return WEDLM_OK;
 }
 

@@ -186,3 +186,26 @@ def window_state(seed: int, stream: int, n_seq: int, W: int, n_filled: int | Non
     toks = token_ids(seed, stream + 1, vocab, n_seq * W, exclude=mask_id).reshape(n_seq, W)
     toks = np.where(filled == 1, toks, mask_id).astype(np.int32)
     return filled, toks
+
+
+def paged_kv(seed: int, lengths, hkv: int, hd: int = 128, std: float = 1.0, spare_pages: int = 3):
+    """A one-layer paged KV pool with seeded random page tables.
+
+    Returns (pool, page_table): pool holds bf16 bits (uint16) [num_pages][2 (K, V)]
+    [hkv][16][hd] of N(0, std^2)-shaped values; page_table [n_seq][pages_per_seq]
+    (int32, -1 past a sequence's pages) maps sequence b's 16-token block i to a
+    page, the pages being a seeded random permutation of the pool (so a
+    sequence's pages are scattered).  Position p of sequence b lives in page
+    page_table[b][p // 16], token p % 16."""
+    lengths = [int(x) for x in lengths]
+    need = [(x + 15) // 16 for x in lengths]
+    num_pages = sum(need) + spare_pages
+    pps = max(1, max(need) if need else 1)
+    order = np.argsort(uniform01(seed, 7_000_001, num_pages), kind="stable").astype(np.int32)
+    table = np.full((len(lengths), pps), -1, np.int32)
+    k = 0
+    for b, m in enumerate(need):
+        table[b, :m] = order[k:k + m]
+        k += m
+    pool = normal(seed, 7_000_002, std, (num_pages, 2, hkv, 16, hd), "bf16")
+    return pool, table

@@ -50,6 +50,9 @@ def test_full_size_batch16_per_layer_against_oracle():
         eng.prefill(b, p, N, W)
     prm = step_params(cfg["lam"], cfg["tau"], False, cfg["logit_scale"])
     eng.stream_step_async(prm, 3)
+    plans = {k: (eng.gemm_plan(k, B * W), eng.gemm_schedule(k, B * W))
+             for k in ("gemm_qkv", "gemm_o", "gemm_gate_up", "gemm_down", "gemm_lm_head")}
+    print("tuned GEMM plans at", B * W, "rows:", plans)
     b = int(np.argmin([len(p) for p in prompts]))
     f0, t0 = eng.get_window(b)
     gen = eng.read_generated(b)
@@ -105,15 +108,22 @@ def test_full_size_batch16_per_layer_against_oracle():
     if comparable(Ht, cfg["tau"], False):
         assert np.nonzero(fl[:n])[0].tolist() == fills
 
-    # end to end, for the record: exact oracle from scratch vs the GPU
-    ofull = O.KVCache.empty(m)
-    _, ck, cv = O.forward_window(m, ofull, seq, np.arange(S))
-    ofull.append(ck, cv)
-    h_e2e, _, _ = O.forward_window(m, ofull, toks, pos)
-    e2e = 0.0
-    for r in range(nf, n):
-        ref = O.lm_logits(m, h_e2e[r:r + 1], 1.0)[0]
-        e2e = max(e2e, float(np.abs(z[r] - ref).max() / np.abs(ref).max()))
+    # end to end (no teacher forcing): the oracle recomputes the sequence from
+    # scratch, exactly and with the R18 bf16 rounding points; the GPU's logits
+    # are compared with both
+    e2e = {}
+    m18 = O.Model(dims, synth.model_weights(dims, seed=0, dtype="bf16"), cache_fp64=False, act_round=O.round_bf16)
+    for name, mm in (("exact", m), ("r18", m18)):
+        ofull = O.KVCache.empty(mm)
+        _, ck, cv = O.forward_window(mm, ofull, seq, np.arange(S))
+        ofull.append(ck, cv)
+        h_e2e, _, _ = O.forward_window(mm, ofull, toks, pos)
+        worst_e = 0.0
+        for r in range(nf, n):
+            ref = O.lm_logits(mm, h_e2e[r:r + 1], 1.0)[0]
+            worst_e = max(worst_e, float(np.abs(z[r] - ref).max() / np.abs(ref).max()))
+        e2e[name] = worst_e
     print(f"full-size sampled: sequence {b} (P={len(prompts[b])}, S={S}), {n - nf} masked rows; "
-          f"end-to-end logits max-rel vs the exact oracle {e2e:.3e}")
-    assert e2e < 0.1
+          f"end-to-end logits max-rel vs the exact oracle {e2e['exact']:.3e}, vs the R18 oracle {e2e['r18']:.3e}")
+    # gross-error guards; the measured values are recorded with the design notes
+    assert e2e["exact"] < 0.1 and e2e["r18"] < 0.1
