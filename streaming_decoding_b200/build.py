@@ -31,8 +31,7 @@ def nvcc() -> str:
 def _flags(verbose_ptxas: bool):
     # -dlcm=cg: plain global loads bypass L1.  Kernels of a step start early
     # (programmatic dependent launch) and read slot state, row metadata and
-    # activations that the kernel just before them writes, and a context's
-    # buffers may reuse addresses another context freed; an L1 line filled
+    # activations that the kernel just before them writes; an L1 line filled
     # before such a write could otherwise be read stale (common.cuh).
     f = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-Xptxas", "-dlcm=cg",
          "-I" + os.path.join(ROOT, "include")] + ARCH

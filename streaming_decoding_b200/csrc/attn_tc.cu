@@ -61,7 +61,7 @@ constexpr int NTHREADS = 224;
 constexpr int CTAS_PER_SM = 2;                      // two independent item streams per SM
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;  // S buffer b at 64 b, O at 128
 constexpr int MAX_SPLITS = 32;  // key chunks per row tile
-constexpr int kMB = 8;          // merge: chunk partials in flight per lane and batch
+constexpr int kMR = 4, kMS = 2;  // merge: rows x chunk partials in flight per lane
 constexpr int XCH_FLOATS = 32 * 64 + 2 * 64;        // DUAL exchange: 32 dims x 64 rows, then (m, l)
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + Q_BYTES;
@@ -718,46 +718,72 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
                 if (is_last) {
                     __threadfence();
                     const int nsplit = item.nsplit;
-                    // a warp per row, a lane per 4 dims; lane s also holds chunk s's
-                    // (m, l), shared with the warp by shuffles; the chunk partials of
-                    // a row are read kMB at a time, all in flight together
+                    // a warp takes kMR rows at a time (rows warp, warp + 4, ...), a lane
+                    // 4 dims; lane s holds chunk s's weight 2^(m_s - M) / L of each of
+                    // those rows (shuffles), and kMR rows x kMS chunk partials are in
+                    // flight together
 #pragma unroll 1
-                    for (int row = warp; row < qrows; row += 4) {
-                        if (item.r0 + row / g >= item.n) continue;
-                        const int64_t pb = ((int64_t)(item.entry * p.stride + item.r0 + row / g) * p.hq +
-                                            item.kvh * g + row % g) * p.max_splits;
-                        const float2 ml = lane < nsplit ? __ldcg(&p.part_ml[pb + lane]) : make_float2(-INFINITY, 0.f);
-                        float M = ml.x;
+                    for (int row0 = warp; row0 < qrows; row0 += 4 * kMR) {
+                        int64_t pbr[kMR];
+                        bool okr[kMR];
+                        float wl[kMR];
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-                        const float w = (ml.x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml.x - M);
-                        float L = w * ml.y;
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-                        const float wn = L > 0.f ? w / L : 0.f;
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-                        for (int s0 = 0; s0 < nsplit; s0 += kMB) {
-                            float4 v[kMB];
-#pragma unroll
-                            for (int q = 0; q < kMB; ++q)
-                                v[q] = s0 + q < nsplit
-                                           ? __ldcg(reinterpret_cast<const float4*>(p.part_o + (pb + s0 + q) * HD) + lane)
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                            for (int q = 0; q < kMB; ++q) {
-                                const float wq = __shfl_sync(0xffffffffu, wn, (s0 + q) & 31);
-                                acc.x += wq * v[q].x;
-                                acc.y += wq * v[q].y;
-                                acc.z += wq * v[q].z;
-                                acc.w += wq * v[q].w;
-                            }
+                        for (int u = 0; u < kMR; ++u) {
+                            const int row = row0 + 4 * u;
+                            okr[u] = row < qrows && item.r0 + row / g < item.n;
+                            pbr[u] = ((int64_t)(item.entry * p.stride + item.r0 + row / g) * p.hq + item.kvh * g +
+                                      row % g) * p.max_splits;
                         }
-                        uint2 o2;
-                        o2.x = pack_bf16(acc.x, acc.y);
-                        o2.y = pack_bf16(acc.z, acc.w);
-                        *reinterpret_cast<uint2*>(p.out + ((int64_t)(item.entry * p.stride + item.r0 + row / g) * p.hq +
-                                                           item.kvh * g + row % g) * HD + lane * 4) = o2;
+                        float2 ml[kMR];
+#pragma unroll
+                        for (int u = 0; u < kMR; ++u)
+                            ml[u] = (okr[u] && lane < nsplit) ? __ldcg(&p.part_ml[pbr[u] + lane])
+                                                              : make_float2(-INFINITY, 0.f);
+#pragma unroll
+                        for (int u = 0; u < kMR; ++u) {
+                            float M = ml[u].x;
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+                            const float w = (ml[u].x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml[u].x - M);
+                            float L = w * ml[u].y;
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+                            wl[u] = L > 0.f ? w / L : 0.f;
+                        }
+                        float4 acc[kMR];
+#pragma unroll
+                        for (int u = 0; u < kMR; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+                        for (int s0 = 0; s0 < nsplit; s0 += kMS) {
+                            float4 v[kMR][kMS];
+#pragma unroll
+                            for (int u = 0; u < kMR; ++u)
+#pragma unroll
+                                for (int q = 0; q < kMS; ++q)
+                                    v[u][q] = (okr[u] && s0 + q < nsplit)
+                                                  ? __ldcg(reinterpret_cast<const float4*>(p.part_o + (pbr[u] + s0 + q) * HD) + lane)
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int u = 0; u < kMR; ++u)
+#pragma unroll
+                                for (int q = 0; q < kMS; ++q) {
+                                    const float w = __shfl_sync(0xffffffffu, wl[u], (s0 + q) & 31);
+                                    acc[u].x += w * v[u][q].x;
+                                    acc[u].y += w * v[u][q].y;
+                                    acc[u].z += w * v[u][q].z;
+                                    acc[u].w += w * v[u][q].w;
+                                }
+                        }
+#pragma unroll
+                        for (int u = 0; u < kMR; ++u) {
+                            if (!okr[u]) continue;
+                            const int row = row0 + 4 * u;
+                            uint2 o2;
+                            o2.x = pack_bf16(acc[u].x, acc[u].y);
+                            o2.y = pack_bf16(acc[u].z, acc[u].w);
+                            *reinterpret_cast<uint2*>(p.out + ((int64_t)(item.entry * p.stride + item.r0 + row / g) * p.hq +
+                                                               item.kvh * g + row % g) * HD + lane * 4) = o2;
+                        }
                     }
                 }
             }

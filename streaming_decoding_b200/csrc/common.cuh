@@ -40,12 +40,12 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 // Global memory is never read through the non-coherent read-only path (no
-// __ldg, no const __restrict__ kernel parameters): a context's buffers may
-// reuse the addresses of buffers another context freed earlier in the
-// process, and kernels started early by programmatic dependent launch do not
-// begin from clean caches, so a stale line of the old contents could be
-// returned.  Plain loads are compiled to bypass L1 (-dlcm=cg, see build.py)
-// and are served coherently from L2; bulk data moves by TMA, also through L2.
+// __ldg, no const __restrict__ kernel parameters): kernels started early by
+// programmatic dependent launch read data that the kernel just before them
+// wrote, and the read-only path is only guaranteed coherent for data that no
+// one writes while the kernel runs.  Plain loads are compiled to bypass L1
+// (-dlcm=cg, see build.py) and are served from L2; bulk data moves by TMA,
+// also through L2.
 
 // Device error word codes (mirrors of the wedlm_status values they map to).
 constexpr int kErrBounds = 1;     // a bounds check refused an access

@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(256) entropy_scan_kernel(const float* logits, 
 #pragma unroll
         for (int k = 0; k < kScanVec; ++k) {
             const int i = b + threadIdx.x + k * 256;
-            v[k] = i < nvec ? __ldcs(z4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[k] = i < nvec ? __ldcg(z4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         float m = -INFINITY;
         int a = INT_MAX;
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(256) entropy_partial_kernel(const float* logit
         const int nvec = (v1 - v0) >> 2;
         const float4* z4 = reinterpret_cast<const float4*>(zr + v0);
         for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-            const float4 z = __ldcs(z4 + i);
+            const float4 z = __ldcg(z4 + i);
             const int id = v0 + 4 * i;
             if (id != mask_id) push(z.x, id);
             if (id + 1 != mask_id) push(z.y, id + 1);

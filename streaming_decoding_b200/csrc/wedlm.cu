@@ -44,7 +44,11 @@ struct Arena {
     size_t size = 0, used = 0;
     std::vector<std::pair<void**, size_t>> plan;
     void add(void** p, size_t bytes) { plan.emplace_back(p, align_up(bytes ? bytes : 1, 256)); }
-    cudaError_t commit() {
+    // Zeroed on the context's stream: work the context enqueues later on that
+    // stream (the RoPE table, the first prefill) is ordered after the zeroing,
+    // which it would not be on the legacy default stream when the context's
+    // stream is a non-blocking one.
+    cudaError_t commit(cudaStream_t st) {
         size = 0;
         for (auto& e : plan) size += e.second;
         cudaError_t err = cudaMalloc(&base, size);
@@ -54,7 +58,7 @@ struct Arena {
             *e.first = base + off;
             off += e.second;
         }
-        return cudaMemsetAsync(base, 0, size, 0);
+        return cudaMemsetAsync(base, 0, size, st);
     }
     void release() {
         if (base) cudaFree(base);
@@ -906,7 +910,7 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         wa.add(&ctx->wgu[l], (size_t)2 * F * d * elt);
         wa.add(&ctx->wd[l], (size_t)d * F * elt);
     }
-    if (wa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+    if (wa.commit(ctx->stream) != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
     ctx->loaded.assign(3 + 9 * L, 0);
 
     // KV pool, rope table, slot and row state, step-result block.
@@ -954,7 +958,7 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         ctx->n_attn_tickets = (size_t)B * tiles * ctx->hkv;
         sa.add((void**)&ctx->attn_tickets, ctx->n_attn_tickets * sizeof(int));
     }
-    if (sa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+    if (sa.commit(ctx->stream) != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
     ss.out_count = ctx->res_dev;
     ss.S = ctx->res_dev + B;
     ss.out_tokens = ctx->res_dev + 2 * B;
@@ -1007,7 +1011,7 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         xa.add((void**)&ctx->attn_po, pairs * ctx->hd * 4);
         xa.add((void**)&ctx->attn_pml, pairs * sizeof(float2));
     }
-    if (xa.commit() != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
+    if (xa.commit(ctx->stream) != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
     if (ctx->bf16 && !(make_q_tmap(&ctx->tm_q, (const bf16*)ctx->q, Mmax, ctx->hq, ctx->hkv, false) &&
                        make_q_tmap(&ctx->tm_q_dual, (const bf16*)ctx->q, Mmax, ctx->hq, ctx->hkv, true)))
         return bail(WEDLM_ERR_CUDA);
@@ -1022,12 +1026,16 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
         std::memcpy(&no_id_bits, &no_id, 4);
         const float4 empty = make_float4(-INFINITY, 0.f, 0.f, no_id_bits);
         std::vector<float4> fill((size_t)ctx->Mdec * ctx->lm_npart, empty);
-        if (cudaMemcpy(ctx->lm_part, fill.data(), fill.size() * sizeof(float4), cudaMemcpyHostToDevice) != cudaSuccess)
+        if (cudaMemcpyAsync(ctx->lm_part, fill.data(), fill.size() * sizeof(float4), cudaMemcpyHostToDevice,
+                            ctx->stream) != cudaSuccess ||
+            cudaStreamSynchronize(ctx->stream) != cudaSuccess)
             return bail(WEDLM_ERR_CUDA);
     }
     std::vector<int32_t> pt((size_t)B * ctx->pages_per_seq, -1);
-    if (cudaMemcpy(ss.page_table, pt.data(), pt.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+    if (cudaMemcpyAsync(ss.page_table, pt.data(), pt.size() * 4, cudaMemcpyHostToDevice, ctx->stream) != cudaSuccess ||
+        cudaStreamSynchronize(ctx->stream) != cudaSuccess)
         return bail(WEDLM_ERR_CUDA);
+    if (cudaGetLastError() != cudaSuccess) return bail(WEDLM_ERR_CUDA);  // e.g. the RoPE table launch
     if (cudaDeviceSynchronize() != cudaSuccess) return bail(WEDLM_ERR_CUDA);
     ctx->h_W.assign(B, 0);
     ctx->h_S.assign(B, 0);
@@ -1541,7 +1549,8 @@ wedlm_status wedlm_debug_capture(wedlm_ctx* ctx, int32_t enable) {
             ctx->dbg_resid = nullptr;
             return fail(ctx, WEDLM_ERR_OOM_DEVICE, "residual capture buffer");
         }
-        CK(cudaMemset(ctx->dbg_resid, 0, bytes));
+        CK(cudaMemsetAsync(ctx->dbg_resid, 0, bytes, ctx->stream));
+        CK(cudaStreamSynchronize(ctx->stream));
         drop_graph(ctx);
     } else if (!enable && ctx->dbg_resid) {
         cudaFree(ctx->dbg_resid);
