@@ -459,12 +459,13 @@ wedlm_status wedlm_entropy_select_async(const float* logits, int32_t vocab, int3
  * n_heads % n_kv_heads == 0; stride <= 1024.
  * workspace: at least wedlm_attention_workspace_bytes(...) bytes; its first
  * int32 is a device error word (1: a page id outside [0, num_pages) or more
- * keys than max_ctx allows; 2: a bounded wait gave up).  The workspace must
- * be zeroed (e.g. cudaMemsetAsync) before its first use; each call leaves it
- * reusable as long as the error word stays 0.  After a nonzero error word,
- * zero the whole workspace again.  Asynchronous: the call enqueues the kernel
- * on `stream` and returns; out and the error word are valid once the stream
- * has been synchronised.  WEDLM_ERR_INVALID_ARG for bad sizes, pointers or a
+ * keys than max_ctx allows; 2: a bounded wait gave up), the rest holds the
+ * key chunks' partial results.  The error word must be zero before a call
+ * (zeroing the whole workspace once, e.g. with cudaMemsetAsync, is enough;
+ * calls leave it as they found it while no error occurs).  Asynchronous: the
+ * call enqueues the attention kernel (and, when a window's keys are split
+ * into chunks, the kernel that combines them) on `stream` and returns; out
+ * and the error word are valid once the stream has been synchronised.  WEDLM_ERR_INVALID_ARG for bad sizes, pointers or a
  * too small workspace, WEDLM_ERR_CUDA if the launch fails. */
 wedlm_status wedlm_attention_workspace_bytes(int32_t n_seq, int32_t stride, int32_t n_heads, int32_t n_kv_heads,
                                              int32_t max_ctx, int64_t* bytes);

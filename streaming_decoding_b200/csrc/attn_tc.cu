@@ -18,29 +18,37 @@
 // key rows of 128 bytes with the 128-byte swizzle: the K-major operand form
 // for K and the MN-major (dims contiguous) form for V.
 //
-// The kernel is persistent: one CTA per SM walks its share of the items (the
-// non-empty items of the launch, numbered in (entry, tile, KV head, chunk)
-// order, dealt round-robin), and its K and V rings, Q buffers, S buffers and O
-// accumulators run continuously across items, so the loads of the next item
-// stream in while the current one finishes.  Keys below a sequence's committed
-// length were written by earlier kernels, so the loaders start on them before
-// waiting for the previous kernel (the QKV projection that writes q and the
-// window's K/V).
+// Persistent, two CTAs per SM: each CTA walks its share of the launch's
+// non-empty items (numbered in (entry, tile, KV head, chunk) order, dealt
+// round-robin) with every stage of its pipeline running ahead of the next:
+// K and V rings of two 64-key blocks each (16 KB per block), a Q buffer, two S
+// buffers and an O accumulator in TMEM (256 columns: S buffer s at 64 s, O at
+// 128; P overwrites the first 32 columns of its S buffer as packed bf16).  The
+// MMA thread issues S = Q K^T a block ahead of the softmax and O += P V as
+// soon as a block's P is written; an item's output is read out by separate
+// epilogue warps while the softmax moves on to the next item.  Two CTAs per SM
+// because TMA loads of 2 KB page boxes are limited per CTA: one CTA per SM
+// streamed random pages at about 3.8 TB/s whatever its ring depth, two CTAs
+// at the HBM peak (measured on this hardware).  Keys below a sequence's
+// committed length were written by earlier kernels, so the loaders start on
+// them before waiting for the previous kernel (the QKV projection that writes
+// q and the window's K/V).
 //
-// TMEM (512 columns): two S buffers of 64 columns (P overwrites the first 32
-// columns of its own S buffer as packed bf16) and two O accumulators of 128.
-// Warp roles (224 threads):
-//   warps 0-3  softmax: thread i owns query row i (TMEM lane i); causal and
-//              chunk masks, running max m and sum l (exp2 domain); O is
-//              rescaled in TMEM only when a row's max grows by more than 2^8
-//              (otherwise P stays relative to the older max, exactly); at the
-//              end of an item O is normalised and stored, or (keys split over
-//              chunks) stored unnormalised with (m, l), and the last chunk of
-//              the (entry, tile, KV head) to finish merges the partials,
-//   warp 4     allocates TMEM; one thread issues the MMAs,
-//   warp 5     TMA loads of Q (two 3-D boxes of 64 dims x g heads x rows, into
-//              one of two Q buffers) and of K blocks into a 4-stage ring,
-//   warp 6     TMA loads of V blocks into a 4-stage ring.
+// Warp roles (352 threads):
+//   warps 0-3  softmax: thread i owns query row i (TMEM lane i), reading its
+//              scores 32 columns at a time; causal and chunk masks on the
+//              blocks that reach the window or the chunk end, running max m
+//              and sum l; O is rescaled in TMEM only when a
+//              row's max grows by more than 2^8 in the exp2 domain (otherwise
+//              P stays relative to the older max, exactly); at the end of an
+//              item (m, l) go to the epilogue warps through shared memory,
+//   warps 4-7  epilogue: O of a finished item out of TMEM, normalised to bf16
+//              (a single key chunk) or stored unnormalised with (m, l) as the
+//              chunk's partial, which attn_merge_kernel combines,
+//   warp 8     allocates TMEM; one thread issues the MMAs,
+//   warp 9     TMA loads of Q (two 3-D boxes of 64 dims x g heads x rows) and
+//              of the K blocks,
+//   warp 10    TMA loads of the V blocks.
 // All waits are bounded; a timeout sets the device error word.
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
@@ -53,23 +61,34 @@ constexpr int KBLK = 64;
 constexpr int QROWS = 128;
 constexpr int NK = 2;                               // K ring stages
 constexpr int NV = 2;                               // V ring stages
+constexpr int NQ = 1;                               // Q buffers
+constexpr int NSB = 2;                              // S buffers in TMEM
+constexpr int NO = 1;                               // O accumulators in TMEM
+constexpr int CTAS_PER_SM = 2;
 constexpr int Q_BYTES = QROWS * HD * 2;             // two 64-dim halves of 16 KB
 constexpr int HALF_BYTES = KBLK * 128;              // 64 keys x 64 dims
 constexpr int BLK_BYTES = 2 * HALF_BYTES;           // one K or V block: 16 KB
 constexpr int BOX_BYTES = kPage * 128;              // one page, one half: 2 KB
-constexpr int NTHREADS = 224;
-constexpr int CTAS_PER_SM = 2;                      // two independent item streams per SM
-constexpr uint32_t TM_S = 0, TM_O = 128, TM_COLS = 256;  // S buffer b at 64 b, O at 128
+constexpr int NTHREADS = 352;
+constexpr int WARP_EPI = 4, WARP_MMA = 8, WARP_KLOAD = 9, WARP_VLOAD = 10;
+constexpr uint32_t TM_S = 0, TM_O = NSB * 64, TM_COLS = 256;
 constexpr int MAX_SPLITS = 32;  // key chunks per row tile
-constexpr int kMR = 4, kMS = 2;  // merge: rows x chunk partials in flight per lane
-constexpr int XCH_FLOATS = 32 * 64 + 2 * 64;        // DUAL exchange: 32 dims x 64 rows, then (m, l)
+constexpr int XCH_FLOATS = 32 * 64;                 // DUAL exchange: 32 dims x 64 rows
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + Q_BYTES;
+constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
 constexpr int OFF_V = OFF_K + NK * BLK_BYTES;
 constexpr int OFF_X = OFF_V + NV * BLK_BYTES;                    // DUAL exchange
-constexpr int OFF_BAR = OFF_X + XCH_FLOATS * 4;
-constexpr int BAR_BYTES = 512;                                    // barriers and flags
+constexpr int OFF_ML = OFF_X + XCH_FLOATS * 4;                   // (m, l) per O buffer and row
+constexpr int ENT_CAP = 256;                                     // entries whose (n, S) are cached
+constexpr int GRP_CAP = 512;                                     // (entry, tile) groups with item prefix sums
+constexpr int OFF_ENT = OFF_ML + NO * QROWS * 8;                  // (n, S) of the launch's entries
+constexpr int OFF_GRP = OFF_ENT + ENT_CAP * 8;                    // items in groups 0..g, per group g
+constexpr int OFF_BAR = OFF_GRP + GRP_CAP * 4;
+constexpr int BAR_BYTES = 512;                                    // barriers
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024 /*align*/;
+static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 228 * 1024, "attention shared memory: two CTAs per SM");
+// Row max growth (exp2 domain) tolerated before O is rescaled.
+constexpr float kRescaleLog2 = 8.0f;
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -81,11 +100,28 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// Non-blocking probe: has the phase of parity `parity` completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
 // One box of the pool's tensor map (x = dim offset, y = pool row) into shared memory.
 __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// A 3-D box of q: 64 dims x g heads x rt rows (one 64-dim half of a tile).
+__device__ __forceinline__ void tma_box3(uint32_t dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
         : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -156,29 +192,39 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-// Barrier among the 128 softmax threads only (named barrier 1).
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier among the 128 epilogue threads only (named barrier 1).
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The same barrier, returning whether `v` holds in every epilogue thread: the
+// DUAL exchange (which synchronises the four warps) is entered by all of them
+// or by none, also when a bounded wait gave up in one warp only.
+__device__ __forceinline__ bool epi_all(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+
+// 2^x on the special-function unit (PTX ex2.approx, flush-to-zero): about 2
+// ulp, ex2(-inf) = +0.  The softmax weights are rounded to bf16 right after.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// A 3-D box of q: 64 dims x g heads x rt rows (one 64-dim half of a tile).
-__device__ __forceinline__ void tma_box3(uint32_t dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-        : "memory");
-}
-
 struct AttnParams {
     KVLayout kvl;
     int layer, hq, hkv;
     bf16* out;
-    float* part_o;
-    float2* part_ml;
-    int* tickets;  // [entries][hkv][tiles], zero between launches
+    float* part_o;    // [rows][hq][max_splits][128] unnormalised chunk outputs
+    float2* part_ml;  // [rows][hq][max_splits] (max in the exp2 domain, sum)
     int n_entries, stride, kv_chunk, max_splits, rt, tiles;
     SlotState ss;
     RowMap rm;
@@ -195,9 +241,15 @@ struct Item {
 // over (entry, tile) groups -- group size hkv * nsplit, KV head then chunk
 // within a group -- and CTA c takes numbers c, c + G, c + 2G, ...  Every role
 // of the CTA runs its own copy and sees the same sequence (the sizes it reads
-// do not change during the launch).  S and n are read through L2: the kernel
-// may start before the previous kernel of the stream has finished.
+// do not change during the launch).  Each entry's (n, S) is read from global
+// memory once per CTA, at kernel start, into shared memory (the first
+// ENT_CAP entries; any beyond are read through L2 as they come): walking
+// from one of the CTA's items to the next passes several groups, and a
+// dependent L2 round trip per group would dominate short items.  The kernel
+// may start before the previous kernel of the stream has finished; n and S
+// are not written by it.
 struct ItemIter {
+    int g = 0;                 // current group (prefix-sum search)
     int e = 0, t = 0;          // current group
     int base = 0;              // number of the group's first item
     int next = 0;              // next number this CTA takes
@@ -205,42 +257,79 @@ struct ItemIter {
     int S = 0, n = 0, nsplit = 0;
 };
 
-__device__ __forceinline__ bool next_item(ItemIter& it, const AttnParams& p, Item& o) {
-    while (it.e < p.n_entries) {
-        if (it.cnt < 0) {
-            const int slot = p.rm.slot_base + it.e;
-            it.n = __ldcg(p.rm.n + slot);
-            it.S = __ldcg(p.ss.S + slot);
-            const int r0 = it.t * p.rt;
-            if (r0 >= it.n) {
-                it.cnt = 0;
-            } else {
-                const int kend = it.S + min(r0 + p.rt, it.n);
-                it.nsplit = (kend + p.kv_chunk - 1) / p.kv_chunk;
-                it.cnt = p.hkv * it.nsplit;
-                if (it.nsplit > p.max_splits || it.S < 0) {  // more keys than the launch has room for
-                    set_error(p.err, kErrBounds);
-                    it.cnt = 0;
-                }
-            }
+// Key chunks of row tile t of a window with n rows over committed length S.
+__device__ __forceinline__ int tile_splits(int S, int n, int t, int rt, int kv_chunk) {
+    const int kend = S + min((t + 1) * rt, n);
+    return (kend + kv_chunk - 1) / kv_chunk;
+}
+
+// (n, S) of entry e: shared memory for the first ENT_CAP entries, else L2.
+__device__ __forceinline__ int2 entry_ns(const AttnParams& p, const int2* ent, int e) {
+    if (e < ENT_CAP) return ent[e];
+    const int slot = p.rm.slot_base + e;
+    return make_int2(__ldcg(p.rm.n + slot), __ldcg(p.ss.S + slot));
+}
+
+// Items of group g = (entry g / tiles, tile g % tiles): hkv * nsplit, 0 for an
+// empty tile or (bounds error) a tile with more chunks than the launch allows.
+__device__ __forceinline__ int group_items(const AttnParams& p, const int2* ent, int g, int& S, int& n, int& nsplit) {
+    const int e = g / p.tiles, t = g - e * p.tiles;
+    const int2 v = entry_ns(p, ent, e);
+    n = v.x;
+    S = v.y;
+    if (t * p.rt >= n) return 0;
+    nsplit = tile_splits(S, n, t, p.rt, p.kv_chunk);
+    if (nsplit > p.max_splits || S < 0) {  // more keys than the launch has room for
+        set_error(p.err, kErrBounds);
+        return 0;
+    }
+    return p.hkv * nsplit;
+}
+
+__device__ __forceinline__ void fill_item(const AttnParams& p, int g, int local, int S, int n, int nsplit, Item& o) {
+    o.entry = g / p.tiles;
+    o.tile = g - o.entry * p.tiles;
+    o.kvh = local / nsplit;
+    o.sp = local % nsplit;
+    o.slot = p.rm.slot_base + o.entry;
+    o.S = S;
+    o.n = n;
+    o.nsplit = nsplit;
+    o.r0 = o.tile * p.rt;
+    o.r_last = min(o.r0 + p.rt, n) - 1;
+    const int kend = S + o.r_last + 1;
+    o.ks = o.sp * p.kv_chunk;
+    o.ke = min(kend, o.ks + p.kv_chunk);
+    o.nblk = (o.ke - o.ks + KBLK - 1) / KBLK;
+}
+
+// The CTA's next item.  With at most GRP_CAP groups the item number is looked
+// up by bisection in the per-group prefix sums `gend` (built once per CTA);
+// otherwise the groups are walked one by one.
+__device__ __forceinline__ bool next_item(ItemIter& it, const AttnParams& p, const int2* ent, const int* gend,
+                                          Item& o) {
+    const int G = p.n_entries * p.tiles;
+    if (G <= GRP_CAP) {
+        if (G == 0 || it.next >= gend[G - 1]) return false;
+        int lo = it.g, hi = G - 1;  // the group holding item it.next: first g with gend[g] > it.next
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (gend[mid] > it.next) hi = mid;
+            else lo = mid + 1;
         }
+        it.g = lo;
+        int S, n, nsplit;
+        group_items(p, ent, lo, S, n, nsplit);
+        fill_item(p, lo, it.next - (lo ? gend[lo - 1] : 0), S, n, nsplit, o);
+        it.next += gridDim.x;
+        return true;
+    }
+    while (it.e < p.n_entries) {
+        const int g = it.e * p.tiles + it.t;
+        if (it.cnt < 0) it.cnt = group_items(p, ent, g, it.S, it.n, it.nsplit);
         if (it.next < it.base + it.cnt) {
-            const int local = it.next - it.base;
+            fill_item(p, g, it.next - it.base, it.S, it.n, it.nsplit, o);
             it.next += gridDim.x;
-            o.entry = it.e;
-            o.tile = it.t;
-            o.kvh = local / it.nsplit;
-            o.sp = local % it.nsplit;
-            o.slot = p.rm.slot_base + it.e;
-            o.S = it.S;
-            o.n = it.n;
-            o.nsplit = it.nsplit;
-            o.r0 = it.t * p.rt;
-            o.r_last = min(o.r0 + p.rt, it.n) - 1;
-            const int kend = it.S + o.r_last + 1;
-            o.ks = o.sp * p.kv_chunk;
-            o.ke = min(kend, o.ks + p.kv_chunk);
-            o.nblk = (o.ke - o.ks + KBLK - 1) / KBLK;
             return true;
         }
         it.base += it.cnt;
@@ -260,50 +349,62 @@ __device__ __forceinline__ bool next_item(ItemIter& it, const AttnParams& p, Ite
 // is zeroed at creation and only ever holds finite K/V, so P = 0 times V stays
 // 0.  Blocks that reach the window rows (keys >= S) wait for the previous
 // kernel first; with `with_q` the warp also loads each item's Q (after that
-// wait) into its Q buffer.  Returns false after a failed wait.
-template <bool DUAL, int NST>
-__device__ __forceinline__ bool kv_loader(const AttnParams& p, const CUtensorMap* tm_kv, const CUtensorMap* tm_q,
-                                          int kv, uint8_t* ring, uint64_t* full, uint64_t* empty, bool with_q,
+// wait) into Q buffer (item index mod NQ).  Returns false after a failed wait.
+template <bool DUAL>
+__device__ __forceinline__ bool kv_loader(const AttnParams& p, const int2* ent, const int* gend,
+                                          const CUtensorMap* tm_kv,
+                                          const CUtensorMap* tm_q, int kv, uint8_t* ring, uint64_t* full, uint64_t* empty, bool with_q,
                                           uint8_t* sQ, uint64_t* q_full, uint64_t* q_empty, int lane, bool& waited,
                                           uint32_t& issued, uint32_t& q_issued) {
+    constexpr int NST = NK;
+    static_assert(NK == NV, "one loader body serves both rings");
     int* err = p.err;
     const int g = p.hq / p.hkv;
+    const int64_t page_rows = (int64_t)2 * p.kvl.hkv * kPage;  // pool rows per page step
+    // Page ids of one item's pages [page_first + 128 b, +128): lane l holds
+    // pages +l, +32+l, +64+l, +96+l (-1 past the chunk end or out of range).
+    auto page_batch = [&](const Item& itm, int b, int (&out)[4]) {
+        const int32_t* pt = p.ss.page_table + (int64_t)itm.slot * p.ss.pages_per_seq;
+        const int page_first = itm.ks / kPage, page_end = (itm.ke + kPage - 1) / kPage;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int pi = page_first + b * 128 + i * 32 + lane;
+            int pg = -1;
+            if (pi < page_end) {
+                pg = pi < p.ss.pages_per_seq ? __ldcg(pt + pi) : -1;
+                if (pg < 0 || pg >= p.kvl.num_pages) {
+                    set_error(err, kErrBounds);
+                    pg = -1;
+                }
+            }
+            out[i] = pg;
+        }
+    };
     ItemIter it;
     it.next = blockIdx.x;
-    Item item;
+    Item item, nitem;
+    bool has = next_item(it, p, ent, gend, item);
+    int preg[4] = {-1, -1, -1, -1}, pnext[4] = {-1, -1, -1, -1};
+    if (has) page_batch(item, 0, preg);
     uint32_t gb = 0;
     int li = 0;
     bool ok = true;
-    while (ok && next_item(it, p, item)) {
-        const int32_t* pt = p.ss.page_table + (int64_t)item.slot * p.ss.pages_per_seq;
+    while (ok && has) {
+        // the next item's first page ids are fetched now, while this one streams
+        const bool nhas = next_item(it, p, ent, gend, nitem);
+        if (nhas) page_batch(nitem, 0, pnext);
         const int64_t row0 = p.kvl.page_base(p.layer, 0, kv, item.kvh) / HD;  // pool row of (page 0, kv, head, 0)
-        const int64_t page_rows = (int64_t)2 * p.kvl.hkv * kPage;            // pool rows per page step
-        const int page_first = item.ks / kPage, page_end = (item.ke + kPage - 1) / kPage;
-        int batch = -1;
-        int preg[4];
+        int batch = 0;
         auto load_batch = [&](int b) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int pi = page_first + b * 128 + i * 32 + lane;
-                int pg = -1;
-                if (pi < page_end) {
-                    pg = pi < p.ss.pages_per_seq ? __ldcg(pt + pi) : -1;
-                    if (pg < 0 || pg >= p.kvl.num_pages) {
-                        set_error(err, kErrBounds);
-                        pg = -1;
-                    }
-                }
-                preg[i] = pg;
-            }
+            page_batch(item, b, preg);
             batch = b;
         };
-        load_batch(0);
         int fallback = __shfl_sync(0xffffffffu, preg[0], 0);
         if (fallback < 0) fallback = 0;
         // Q of this item (q comes from the previous kernel).  The first item's Q
         // is deferred until a block needs that kernel anyway, or the ring is
         // full (the MMAs that free it need Q): cache blocks go out first.
-        const int qb = 0;  // one Q buffer: item li's load waits for item li-1's last S
+        const int qb = li % NQ;
         bool q_pending = with_q;
         auto issue_q = [&]() -> bool {
             if (!waited) {
@@ -311,7 +412,7 @@ __device__ __forceinline__ bool kv_loader(const AttnParams& p, const CUtensorMap
                 waited = true;
             }
             bool qok = true;
-            if (lane == 0) qok = mbar_wait_bounded(smem_u32(&q_empty[qb]), (li & 1) ^ 1, err);
+            if (lane == 0) qok = mbar_wait_bounded(smem_u32(&q_empty[qb]), ((li / NQ) & 1) ^ 1, err);
             qok = __shfl_sync(0xffffffffu, qok, 0);
             if (qok) q_issued = (uint32_t)li + 1;
             if (qok && lane == 0) {
@@ -361,6 +462,10 @@ __device__ __forceinline__ bool kv_loader(const AttnParams& p, const CUtensorMap
         }
         if (ok && q_pending) ok = issue_q();
         ++li;
+        item = nitem;
+        has = nhas;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) preg[i] = pnext[i];
     }
     return ok;
 }
@@ -368,34 +473,38 @@ __device__ __forceinline__ bool kv_loader(const AttnParams& p, const CUtensorMap
 // DUAL (valid query rows <= 64): rows 64..127 repeat rows 0..63, and the
 // thread of row i + 64 takes keys 32..63 of every block while the thread of
 // row i takes keys 0..31, each writing zeros into the other half of its P
-// row; the two share the running max through shared memory, so O rows i and
-// i + 64 hold the two halves of one result (summed at the end).  This halves
-// the per-thread softmax work when a tile has 64 or fewer query rows.
+// row; each half keeps its own running max and sum, so O rows i and i + 64
+// hold the two halves of one result, which the epilogue combines.  This
+// halves the per-thread softmax work when a tile has 64 or fewer query rows.
 template <bool DUAL>
 __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kv,
                                                               const __grid_constant__ CUtensorMap tm_q,
                                                               const AttnParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem + OFF_Q;  // Q buffer
+    uint8_t* sQ = smem + OFF_Q;  // [NQ] Q buffers
     uint8_t* sK = smem + OFF_K;  // [NK] K blocks
     uint8_t* sV = smem + OFF_V;  // [NV] V blocks
-    float* xch = reinterpret_cast<float*>(smem + OFF_X);  // DUAL exchange
+    float* xch = reinterpret_cast<float*>(smem + OFF_X);     // DUAL exchange
+    float2* sml = reinterpret_cast<float2*>(smem + OFF_ML);  // [NO][128] (m, l) per row
+    int2* ent = reinterpret_cast<int2*>(smem + OFF_ENT);      // [ENT_CAP] (n, S) per entry
+    int* gend = reinterpret_cast<int*>(smem + OFF_GRP);       // [GRP_CAP] items in groups 0..g
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* q_full = bars + 0;    // [1]
-    uint64_t* q_empty = bars + 1;   // [1]
-    uint64_t* k_full = bars + 2;    // [NK]
-    uint64_t* k_empty = bars + 4;   // [NK]
-    uint64_t* v_full = bars + 6;    // [NV]
-    uint64_t* v_empty = bars + 8;   // [NV]
-    uint64_t* s_full = bars + 10;   // [2] per S buffer
-    uint64_t* p_full = bars + 12;   // [2] per S buffer
-    uint64_t* o_done = bars + 14;   // one completion per P V
-    uint64_t* o_full = bars + 15;   // the item's last P V done
-    uint64_t* o_free = bars + 16;   // O read out by the softmax warps
-    uint64_t* drain = bars + 17;    // the MMA thread's last MMAs (error exit)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
-    int* last_flag = reinterpret_cast<int*>(bars + 19);
+    uint64_t* q_full = bars;              // [NQ]
+    uint64_t* q_empty = q_full + NQ;      // [NQ]
+    uint64_t* k_full = q_empty + NQ;      // [NK]
+    uint64_t* k_empty = k_full + NK;      // [NK]
+    uint64_t* v_full = k_empty + NK;      // [NV]
+    uint64_t* v_empty = v_full + NV;      // [NV]
+    uint64_t* s_full = v_empty + NV;      // [NSB] S = Q K^T of the buffer's block done
+    uint64_t* p_full = s_full + NSB;      // [NSB] its P written (the 4 softmax warps)
+    uint64_t* s_free = p_full + NSB;      // [NSB] its P V done: the buffer may take the next S
+    uint64_t* o_full = s_free + NSB;      // [NO] an item's last P V into the accumulator done
+    uint64_t* o_free = o_full + NO;       // [NO] accumulator read out (the 4 epilogue warps)
+    uint64_t* ml_full = o_free + NO;      // [NO] the item's (m, l) written (softmax warps)
+    uint64_t* ml_free = ml_full + NO;     // [NO] (m, l) read (epilogue warps)
+    uint64_t* drain = ml_free + NO;       // the MMA thread's last MMAs (error exit)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.hq / p.hkv;
@@ -404,13 +513,9 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
     if (threadIdx.x == 0) {
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_kv)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_q)) : "memory");
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
-        mbar_init(o_full, 1);
-        mbar_init(o_free, 4);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 4);
+        for (int s = 0; s < NQ; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
         }
         for (int s = 0; s < NK; ++s) {
             mbar_init(&k_full[s], 1);
@@ -420,12 +525,43 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        mbar_init(o_done, 1);
+        for (int s = 0; s < NSB; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], 4);
+            mbar_init(&s_free[s], 1);
+        }
+        for (int s = 0; s < NO; ++s) {
+            mbar_init(&o_full[s], 1);
+            mbar_init(&o_free[s], 4);
+            mbar_init(&ml_full[s], 4);
+            mbar_init(&ml_free[s], 4);
+        }
         mbar_init(drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 4) {
+    for (int e = threadIdx.x; e < min(p.n_entries, ENT_CAP); e += NTHREADS) {
+        const int slot = p.rm.slot_base + e;
+        ent[e] = make_int2(__ldcg(p.rm.n + slot), __ldcg(p.ss.S + slot));
+    }
+    __syncthreads();
+    if (warp == 0 && p.n_entries * p.tiles <= GRP_CAP) {
+        // items per group, then an inclusive prefix sum over the groups
+        const int G = p.n_entries * p.tiles;
+        int carry = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            int S, n, nsplit, v = 0;
+            if (g0 + lane < G) v = group_items(p, ent, g0 + lane, S, n, nsplit);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (g0 + lane < G) gend[g0 + lane] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    if (warp == WARP_MMA) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(TM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -435,29 +571,31 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     int* err = p.err;
+    const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(head_dim)
 
-    if (warp == 5 || warp == 6) {
+    if (warp == WARP_KLOAD || warp == WARP_VLOAD) {
         // ---------------------------------------------------------- loaders
         bool waited = false;
         uint32_t issued = 0, q_issued = 0;
-        if (warp == 5)
-            kv_loader<DUAL, NK>(p, &tm_kv, &tm_q, 0, sK, k_full, k_empty, true, sQ, q_full, q_empty, lane, waited,
-                                issued, q_issued);
+        const bool kw = warp == WARP_KLOAD;
+        if (kw)
+            kv_loader<DUAL>(p, ent, gend, &tm_kv, &tm_q, 0, sK, k_full, k_empty, true, sQ, q_full, q_empty, lane, waited, issued,
+                            q_issued);
         else
-            kv_loader<DUAL, NV>(p, &tm_kv, &tm_q, 1, sV, v_full, v_empty, false, sQ, q_full, q_empty, lane, waited,
-                                issued, q_issued);
+            kv_loader<DUAL>(p, ent, gend, &tm_kv, &tm_q, 1, sV, v_full, v_empty, false, sQ, q_full, q_empty, lane, waited,
+                            issued, q_issued);
         if (!waited) griddep_wait();
         griddep_launch();
         // Copies still in flight (only after an error) must land before the CTA
         // exits: wait, bounded, for the last blocks issued to each stage.
         if (lane == 0) {
-            uint64_t* full = warp == 5 ? k_full : v_full;
-            const uint32_t nst = warp == 5 ? NK : NV;
-            for (uint32_t j = issued > nst ? issued - nst : 0u; j < issued; ++j)
-                mbar_wait_bounded(smem_u32(&full[j % nst]), (j / nst) & 1, nullptr, 200000000LL);
-            if (q_issued > 0) mbar_wait_bounded(smem_u32(q_full), (q_issued - 1) & 1, nullptr, 200000000LL);
+            uint64_t* full = kw ? k_full : v_full;
+            for (uint32_t j = issued > (uint32_t)NK ? issued - NK : 0u; j < issued; ++j)
+                mbar_wait_bounded(smem_u32(&full[j % NK]), (j / NK) & 1, nullptr, 200000000LL);
+            for (uint32_t j = q_issued > (uint32_t)NQ ? q_issued - NQ : 0u; j < q_issued; ++j)
+                mbar_wait_bounded(smem_u32(&q_full[j % NQ]), (j / NQ) & 1, nullptr, 200000000LL);
         }
-    } else if (warp == 4) {
+    } else if (warp == WARP_MMA) {
         // -------------------------------------------------------------- MMA
         griddep_wait();
         griddep_launch();
@@ -465,82 +603,103 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
             constexpr uint32_t idS = idesc_bf16(128, KBLK);
             constexpr uint32_t idO = idesc_bf16(128, HD) | (1u << 16);  // B (V) MN-major
             // Two cursors over this CTA's blocks (in item order): `sc` issues
-            // S = Q K^T two blocks ahead of `pv`, which issues O += P V.
+            // S = Q K^T into S buffer (block mod NSB) as soon as the block's K,
+            // the item's Q and the buffer are there (up to NSB blocks ahead);
+            // `pv` issues O += P V once the softmax has written the block's P.
             struct Cursor {
                 ItemIter it;
                 Item item;
-                int li = -1, j = 0;
+                int li = 0, j = 0;
                 uint32_t gb = 0;
                 bool valid = false;
             };
             auto start = [&](Cursor& c) {
                 c.it.next = blockIdx.x;
-                c.valid = next_item(c.it, p, c.item);
-                c.li = 0;
-                c.j = 0;
-                c.gb = 0;
+                c.valid = next_item(c.it, p, ent, gend, c.item);
             };
             auto advance = [&](Cursor& c) {
                 ++c.gb;
                 if (++c.j == c.item.nblk) {
                     c.j = 0;
                     ++c.li;
-                    c.valid = next_item(c.it, p, c.item);
+                    c.valid = next_item(c.it, p, ent, gend, c.item);
                 }
             };
-            auto issue_s = [&](const Cursor& c) -> bool {
+            // 1: S of c's block may be issued; 0: not yet (probe only); -1: a wait failed.
+            auto s_ready = [&](const Cursor& c, bool block) -> int {
                 const uint32_t b = c.gb;
-                const int qb = 0;
-                if (c.j == 0 && !mbar_wait_bounded(smem_u32(q_full), c.li & 1, err)) return false;
-                if (!mbar_wait_bounded(smem_u32(&k_full[b % NK]), (b / NK) & 1, err)) return false;
+                const int qb = c.li % NQ;
+                const uint32_t qpar = (c.li / NQ) & 1, fpar = ((b / NSB) & 1) ^ 1, kpar = (b / NK) & 1;
+                if (block) {
+                    if (c.j == 0 && !mbar_wait_bounded(smem_u32(&q_full[qb]), qpar, err)) return -1;
+                    if (b >= (uint32_t)NSB && !mbar_wait_bounded(smem_u32(&s_free[b % NSB]), fpar, err)) return -1;
+                    if (!mbar_wait_bounded(smem_u32(&k_full[b % NK]), kpar, err)) return -1;
+                    return 1;
+                }
+                if (c.j == 0 && !mbar_test(&q_full[qb], qpar)) return 0;
+                if (b >= (uint32_t)NSB && !mbar_test(&s_free[b % NSB], fpar)) return 0;
+                return mbar_test(&k_full[b % NK], kpar) ? 1 : 0;
+            };
+            auto issue_s = [&](const Cursor& c) {
+                const uint32_t b = c.gb;
+                const int qb = c.li % NQ;
                 tc_fence_after();
                 const uint32_t qa = smem_u32(sQ + qb * Q_BYTES);
                 const uint32_t kb = smem_u32(sK + (b % NK) * BLK_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk)
-                    mma_ss(tmem + TM_S + (b & 1) * 64, sdesc(qa + (kk >> 2) * (QROWS * 128) + (kk & 3) * 32),
+                    mma_ss(tmem + TM_S + (b % NSB) * 64, sdesc(qa + (kk >> 2) * (QROWS * 128) + (kk & 3) * 32),
                            sdesc(kb + (kk >> 2) * HALF_BYTES + (kk & 3) * 32), idS, kk > 0 ? 1u : 0u);
                 umma_commit(&k_empty[b % NK]);
-                umma_commit(&s_full[b & 1]);
+                umma_commit(&s_full[b % NSB]);
                 if (c.j == c.item.nblk - 1) umma_commit(&q_empty[qb]);
+            };
+            auto issue_pv = [&](const Cursor& c) -> bool {
+                const uint32_t b = c.gb;
+                const int sb = b % NSB, ob = c.li % NO;
+                if (!mbar_wait_bounded(smem_u32(&p_full[sb]), (b / NSB) & 1, err)) return false;
+                if (c.j == 0 && !mbar_wait_bounded(smem_u32(&o_free[ob]), ((c.li / NO) & 1) ^ 1, err)) return false;
+                if (!mbar_wait_bounded(smem_u32(&v_full[b % NV]), (b / NV) & 1, err)) return false;
+                tc_fence_after();
+                const uint32_t vb = smem_u32(sV + (b % NV) * BLK_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < KBLK / 16; ++kk)
+                    mma_ts(tmem + TM_O + ob * 128, tmem + TM_S + sb * 64 + kk * 8, sdesc_mn(vb + kk * 2048), idO,
+                           (c.j > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&v_empty[b % NV]);
+                umma_commit(&s_free[sb]);
+                if (c.j == c.item.nblk - 1) umma_commit(&o_full[ob]);
                 return true;
             };
             Cursor sc, pv;
             start(sc);
             start(pv);
             bool ok = true;
-            for (int a = 0; a < 2 && sc.valid && ok; ++a) {
-                ok = issue_s(sc);
-                advance(sc);
-            }
             while (pv.valid && ok) {
-                const uint32_t b = pv.gb;
-                const int ob = 0;
-                if (!(ok = mbar_wait_bounded(smem_u32(&p_full[b & 1]), (b >> 1) & 1, err))) break;
-                if (pv.j == 0 && !(ok = mbar_wait_bounded(smem_u32(o_free), (pv.li & 1) ^ 1, err))) break;
-                if (!(ok = mbar_wait_bounded(smem_u32(&v_full[b % NV]), (b / NV) & 1, err))) break;
-                tc_fence_after();
-                const uint32_t vb = smem_u32(sV + (b % NV) * BLK_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < KBLK / 16; ++kk)
-                    mma_ts(tmem + TM_O + ob * 128, tmem + TM_S + (b & 1) * 64 + kk * 8, sdesc_mn(vb + kk * 2048), idO,
-                           (pv.j > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&v_empty[b % NV]);
-                umma_commit(o_done);
-                if (pv.j == pv.item.nblk - 1) umma_commit(o_full);
-                advance(pv);
-                if (sc.valid) {
-                    // S buffer b & 1 is read by this P V: wait for it before S(b + 2) overwrites it
-                    if (!(ok = mbar_wait_bounded(smem_u32(o_done), b & 1, err))) break;
-                    ok = issue_s(sc);
+                // the softmax needs S of pv's block: issue up to it, waiting if need be
+                while (sc.valid && sc.gb <= pv.gb) {
+                    const int r = s_ready(sc, true);
+                    if (r < 0) {
+                        ok = false;
+                        break;
+                    }
+                    issue_s(sc);
                     advance(sc);
                 }
+                if (!ok) break;
+                // further S blocks whose inputs are already there
+                while (sc.valid && sc.gb < pv.gb + NSB && s_ready(sc, false) > 0) {
+                    issue_s(sc);
+                    advance(sc);
+                }
+                if (!(ok = issue_pv(pv))) break;
+                advance(pv);
             }
             // every MMA issued has completed before TMEM may be released
             umma_commit(drain);
             mbar_wait_bounded(smem_u32(drain), 0, nullptr, 200000000LL);
         }
-    } else if (warp < 4) {
+    } else if (warp < WARP_EPI) {
         // ---------------------------------------------------------- softmax
         griddep_wait();
         griddep_launch();
@@ -548,119 +707,166 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const int qi = DUAL ? (tid & 63) : tid;     // query row this thread works for
         const int half = DUAL ? (tid >> 6) : 0;     // DUAL: key half of every block
-        const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
-        constexpr int NC = DUAL ? 32 : 64;          // score columns per thread and block
+        const float thr = kRescaleLog2 / sl2;       // rescale threshold in raw score units
         ItemIter it;
         it.next = blockIdx.x;
         Item item;
         uint32_t gb = 0;
         int li = 0;
         bool ok = true;
-        while (ok && next_item(it, p, item)) {
+        while (ok && next_item(it, p, ent, gend, item)) {
+            const int ob = li % NO;
             const int rr = item.r0 + qi / g;
             const bool qok = qi < qrows && rr < item.n;
             const int lim = item.S + (qok ? rr : item.r_last);  // last visible key
-            // running max (exp2 domain) and sum of this thread's keys; in DUAL
-            // mode each key half keeps its own and the two merge at the end
-            float m_ref = -INFINITY, l = 0.f;
+            const int kfree = min(item.ke, item.S);             // keys below: visible to every row
+            // running max (raw scores) and sum of this thread's keys; in DUAL
+            // mode each key half keeps its own and the epilogue merges them
+            float m = -INFINITY, l = 0.f;
             for (int j = 0; j < item.nblk && ok; ++j, ++gb) {
-                const int b = gb & 1;
-                const int kb0 = item.ks + j * KBLK + half * 32;
-                const uint32_t tS = tmem + lane_base + TM_S + b * 64;
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&s_full[b]), (gb >> 1) & 1, err));
+                const int sb = gb % NSB;
+                const uint32_t tS = tmem + lane_base + TM_S + sb * 64;
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&s_full[sb]), (gb / NSB) & 1, err));
                 if (!ok) break;
                 tc_fence_after();
                 uint32_t r[32];
-                float s[NC];
-#pragma unroll
-                for (int h = 0; h < NC / 32; ++h) {
-                    tmem_ld32(tS + (DUAL ? half * 32 : h * 32), r);
+                const int kb0 = item.ks + j * KBLK + half * 32;
+                // the block reaches the window or the chunk end: mask by key position
+                const bool edge = item.ks + (j + 1) * KBLK > kfree;
+                // scores of columns [c0, c0 + 32) of this thread's block, masked
+                auto load_scores = [&](int c0, float (&sv)[32]) {
+                    tmem_ld32(tS + c0, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int t = kb0 + h * 32 + c;
-                        s[h * 32 + c] = (t < item.ke && t <= lim) ? __uint_as_float(r[c]) * sl2 : -INFINITY;
-                    }
-                }
-                float bmax = -INFINITY;
+                    for (int c = 0; c < 32; ++c) sv[c] = __uint_as_float(r[c]);
+                    if (edge) {
+                        const int t0 = kb0 + (DUAL ? 0 : c0);
 #pragma unroll
-                for (int c = 0; c < NC; ++c) bmax = fmaxf(bmax, s[c]);
-                const bool need = bmax > m_ref + 8.0f;
+                        for (int c = 0; c < 32; ++c)
+                            if (!(t0 + c < item.ke && t0 + c <= lim)) sv[c] = -INFINITY;
+                    }
+                };
+                float sv[32];
+                float bmax = -INFINITY;
+                load_scores(DUAL ? half * 32 : 0, sv);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) bmax = fmaxf(bmax, sv[c]);
+                if (!DUAL) {
+                    // the second half's max first; its scores are loaded again below
+                    float sv2[32];
+                    load_scores(32, sv2);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) bmax = fmaxf(bmax, sv2[c]);
+                }
+                const bool need = bmax > m + thr;
                 if (j > 0 && __any_sync(0xffffffffu, need)) {
                     // P V of the previous block must be done before O is rescaled
-                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(o_done), (gb - 1) & 1, err));
+                    const uint32_t pb = gb - 1;
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&s_free[pb % NSB]), (pb / NSB) & 1, err));
                     if (!ok) break;
                     tc_fence_after();
-                    const float f = need ? exp2f(m_ref - bmax) : 1.0f;
+                    const float f = need ? fast_exp2((m - bmax) * sl2) : 1.0f;
+                    const uint32_t tO = tmem + lane_base + TM_O + ob * 128;
 #pragma unroll 1
                     for (int c = 0; c < HD; c += 32) {
-                        tmem_ld32(tmem + lane_base + TM_O + c, r);
+                        tmem_ld32(tO + c, r);
                         tmem_wait_ld();
 #pragma unroll
                         for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * f);
-                        tmem_st32(tmem + lane_base + TM_O + c, r);
+                        tmem_st32(tO + c, r);
                     }
                     l *= f;
                 }
-                if (need) m_ref = bmax;
-                const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
+                if (need) m = bmax;
+                const float neg = (m == -INFINITY) ? 0.f : -m * sl2;
                 float psum = 0.f;
+                uint32_t pk[32];
                 if constexpr (DUAL) {
-                    uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float a = exp2f(s[2 * c] - ref), bb = exp2f(s[2 * c + 1] - ref);
+                        const float a = fast_exp2(fmaf(sv[2 * c], sl2, neg));
+                        const float bb = fast_exp2(fmaf(sv[2 * c + 1], sl2, neg));
                         psum += a + bb;
-                        pk[c] = pack_bf16(a, bb);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        r[c] = half ? 0u : pk[c];
-                        r[16 + c] = half ? pk[c] : 0u;
+                        const uint32_t v = pack_bf16(a, bb);
+                        pk[c] = half ? 0u : v;
+                        pk[16 + c] = half ? v : 0u;
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float a = exp2f(s[2 * c] - ref), bb = exp2f(s[2 * c + 1] - ref);
+                    for (int c = 0; c < 16; ++c) {
+                        const float a = fast_exp2(fmaf(sv[2 * c], sl2, neg));
+                        const float bb = fast_exp2(fmaf(sv[2 * c + 1], sl2, neg));
                         psum += a + bb;
-                        r[c] = pack_bf16(a, bb);
+                        pk[c] = pack_bf16(a, bb);
+                    }
+                    load_scores(32, sv);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const float a = fast_exp2(fmaf(sv[2 * c], sl2, neg));
+                        const float bb = fast_exp2(fmaf(sv[2 * c + 1], sl2, neg));
+                        psum += a + bb;
+                        pk[16 + c] = pack_bf16(a, bb);
                     }
                 }
                 l += psum;
-                tmem_st32(tS, r);
+                tmem_st32(tS, pk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[b]);
+                if (lane == 0) mbar_arrive(&p_full[sb]);
             }
             if (!ok) break;
-            // ---- item epilogue: O of this item is complete once its last P V is
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(o_full), li & 1, err));
+            // (m, l) of this item to the epilogue warps, m in the exp2 domain
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&ml_free[ob]), ((li / NO) & 1) ^ 1, err));
+            if (!ok) break;
+            sml[ob * QROWS + tid] = make_float2(m == -INFINITY ? -INFINITY : m * sl2, l);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ml_full[ob]);
+            ++li;
+        }
+    } else if (warp < WARP_MMA) {
+        // --------------------------------------------------------- epilogue
+        griddep_wait();
+        griddep_launch();
+        const int e = threadIdx.x - WARP_EPI * 32;  // TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp - WARP_EPI) * 32) << 16;
+        const int qi = DUAL ? (e & 63) : e;
+        const int half = DUAL ? (e >> 6) : 0;
+        ItemIter it;
+        it.next = blockIdx.x;
+        Item item;
+        int li = 0;
+        bool ok = true;
+        while (ok && next_item(it, p, ent, gend, item)) {
+            const int ob = li % NO;
+            const int rr = item.r0 + qi / g;
+            const bool qok = qi < qrows && rr < item.n;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&ml_full[ob]), (li / NO) & 1, err));
+            float2 own = make_float2(-INFINITY, 0.f), oth = own;
+            if (ok) {
+                own = sml[ob * QROWS + e];
+                if (DUAL) oth = sml[ob * QROWS + (e ^ 64)];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ml_free[ob]);
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(smem_u32(&o_full[ob]), (li / NO) & 1, err));
+            }
+            if (DUAL) ok = epi_all(ok);
             if (!ok) break;
             tc_fence_after();
+            // DUAL: the two key halves of row qi (rows qi and qi + 64 of O) merge:
+            // O = 2^(m0 - M) O0 + 2^(m1 - M) O1, l likewise, M = max(m0, m1)
+            float m = own.x, l = own.y, a_own = 1.f, a_other = 0.f;
+            if (DUAL) {
+                const float M = fmaxf(own.x, oth.x);
+                a_own = M == -INFINITY ? 0.f : fast_exp2(own.x - M);
+                a_other = M == -INFINITY ? 0.f : fast_exp2(oth.x - M);
+                l = a_own * own.y + a_other * oth.y;
+                m = M;
+            }
             const int qrow = item.entry * p.stride + (qok ? rr : item.r_last);
             const int qhead = item.kvh * g + qi % g;
             const int64_t pbase = ((int64_t)qrow * p.hq + qhead) * p.max_splits;
-            const uint32_t tO = tmem + lane_base + TM_O;
-            // DUAL: the two key halves of row qi (rows qi and qi + 64 of O) merge:
-            // O = 2^(m0 - M) O0 + 2^(m1 - M) O1, l likewise, M = max(m0, m1)
-            float a_own = 1.f, a_other = 0.f;
-            if (DUAL) {
-                softmax_sync();  // the exchange buffer is free (previous item)
-                if (half) {
-                    xch[32 * 64 + qi] = m_ref;
-                    xch[32 * 64 + 64 + qi] = l;
-                }
-                softmax_sync();
-                if (!half) {
-                    const float m1 = xch[32 * 64 + qi], l1 = xch[32 * 64 + 64 + qi];
-                    const float M = fmaxf(m_ref, m1);
-                    a_own = (M == -INFINITY) ? 0.f : exp2f(m_ref - M);
-                    a_other = (M == -INFINITY) ? 0.f : exp2f(m1 - M);
-                    l = a_own * l + a_other * l1;
-                    m_ref = M;
-                }
-            }
+            const uint32_t tO = tmem + lane_base + TM_O + ob * 128;
             const float inv = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll 1
             for (int c = 0; c < HD; c += 32) {
@@ -669,12 +875,12 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
                 tmem_wait_ld();
                 if (DUAL) {
                     // the other key half of row qi, through shared memory
-                    softmax_sync();
+                    epi_sync();
                     if (half) {
 #pragma unroll
                         for (int x = 0; x < 32; ++x) xch[x * 64 + qi] = __uint_as_float(r[x]);
                     }
-                    softmax_sync();
+                    epi_sync();
                     if (half) continue;
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
@@ -695,111 +901,78 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
                                             __uint_as_float(r[4 * x + 2]), __uint_as_float(r[4 * x + 3]));
                 }
             }
-            // O is read out: the MMA may accumulate the next item into it
+            // O is read out: the MMA may accumulate a later item into it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(o_free);
-            if (qok && item.nsplit > 1 && !(DUAL && half)) p.part_ml[pbase + item.sp] = make_float2(m_ref, l);
-            if (item.nsplit > 1) {
-                // The last chunk of this (entry, tile, KV head) to finish merges all
-                // chunks' partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-                __threadfence();
-                softmax_sync();
-                if (tid == 0) {
-                    int* ticket = p.tickets + ((int64_t)item.entry * p.hkv + item.kvh) * p.tiles + item.tile;
-                    const int prev = atomicAdd(ticket, 1);
-                    const int last = prev == item.nsplit - 1;
-                    if (last) *ticket = 0;
-                    *last_flag = last;
-                }
-                softmax_sync();
-                const int is_last = *last_flag;
-                softmax_sync();  // every thread has read the flag before the next item may rewrite it
-                if (is_last) {
-                    __threadfence();
-                    const int nsplit = item.nsplit;
-                    // a warp takes kMR rows at a time (rows warp, warp + 4, ...), a lane
-                    // 4 dims; lane s holds chunk s's weight 2^(m_s - M) / L of each of
-                    // those rows (shuffles), and kMR rows x kMS chunk partials are in
-                    // flight together
-#pragma unroll 1
-                    for (int row0 = warp; row0 < qrows; row0 += 4 * kMR) {
-                        int64_t pbr[kMR];
-                        bool okr[kMR];
-                        float wl[kMR];
-#pragma unroll
-                        for (int u = 0; u < kMR; ++u) {
-                            const int row = row0 + 4 * u;
-                            okr[u] = row < qrows && item.r0 + row / g < item.n;
-                            pbr[u] = ((int64_t)(item.entry * p.stride + item.r0 + row / g) * p.hq + item.kvh * g +
-                                      row % g) * p.max_splits;
-                        }
-                        float2 ml[kMR];
-#pragma unroll
-                        for (int u = 0; u < kMR; ++u)
-                            ml[u] = (okr[u] && lane < nsplit) ? __ldcg(&p.part_ml[pbr[u] + lane])
-                                                              : make_float2(-INFINITY, 0.f);
-#pragma unroll
-                        for (int u = 0; u < kMR; ++u) {
-                            float M = ml[u].x;
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-                            const float w = (ml[u].x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml[u].x - M);
-                            float L = w * ml[u].y;
-#pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-                            wl[u] = L > 0.f ? w / L : 0.f;
-                        }
-                        float4 acc[kMR];
-#pragma unroll
-                        for (int u = 0; u < kMR; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-                        for (int s0 = 0; s0 < nsplit; s0 += kMS) {
-                            float4 v[kMR][kMS];
-#pragma unroll
-                            for (int u = 0; u < kMR; ++u)
-#pragma unroll
-                                for (int q = 0; q < kMS; ++q)
-                                    v[u][q] = (okr[u] && s0 + q < nsplit)
-                                                  ? __ldcg(reinterpret_cast<const float4*>(p.part_o + (pbr[u] + s0 + q) * HD) + lane)
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                            for (int u = 0; u < kMR; ++u)
-#pragma unroll
-                                for (int q = 0; q < kMS; ++q) {
-                                    const float w = __shfl_sync(0xffffffffu, wl[u], (s0 + q) & 31);
-                                    acc[u].x += w * v[u][q].x;
-                                    acc[u].y += w * v[u][q].y;
-                                    acc[u].z += w * v[u][q].z;
-                                    acc[u].w += w * v[u][q].w;
-                                }
-                        }
-#pragma unroll
-                        for (int u = 0; u < kMR; ++u) {
-                            if (!okr[u]) continue;
-                            const int row = row0 + 4 * u;
-                            uint2 o2;
-                            o2.x = pack_bf16(acc[u].x, acc[u].y);
-                            o2.y = pack_bf16(acc[u].z, acc[u].w);
-                            *reinterpret_cast<uint2*>(p.out + ((int64_t)(item.entry * p.stride + item.r0 + row / g) * p.hq +
-                                                               item.kvh * g + row % g) * HD + lane * 4) = o2;
-                        }
-                    }
-                }
-            }
+            if (lane == 0) mbar_arrive(&o_free[ob]);
+            if (qok && item.nsplit > 1 && !(DUAL && half)) p.part_ml[pbase + item.sp] = make_float2(m, l);
             ++li;
         }
-    } else {
-        griddep_wait();
-        griddep_launch();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == WARP_MMA) {
         __syncwarp();
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TM_COLS) : "memory");
     }
+}
+
+// Combine the key chunks of every (row, query head) whose row tile was split:
+// O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.  One warp
+// per (row, head), a lane per 4 dims; lane s holds chunk s's (m, l), and all
+// of a pair's chunk partials are in flight together.  Rows whose tile had one
+// chunk were written by the attention kernel itself and are left alone.
+struct MergeParams {
+    const float* part_o;
+    const float2* part_ml;
+    bf16* out;
+    int n_entries, stride, hq, rt, kv_chunk, max_splits;
+    SlotState ss;
+    RowMap rm;
+};
+
+__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+    griddep_wait();
+    griddep_launch();
+    const int lane = threadIdx.x & 31;
+    const int64_t pair = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (pair >= (int64_t)p.n_entries * p.stride * p.hq) return;
+    const int row = (int)(pair / p.hq), h = (int)(pair % p.hq);
+    const int e = row / p.stride, r = row - e * p.stride;
+    const int slot = p.rm.slot_base + e;
+    const int n = __ldcg(p.rm.n + slot);
+    if (r >= n) return;
+    const int S = __ldcg(p.ss.S + slot);
+    const int nsplit = tile_splits(S, n, r / p.rt, p.rt, p.kv_chunk);
+    if (nsplit <= 1 || nsplit > p.max_splits) return;
+    const int64_t pb = ((int64_t)row * p.hq + h) * p.max_splits;
+    const float2 ml = lane < nsplit ? __ldcg(p.part_ml + pb + lane) : make_float2(-INFINITY, 0.f);
+    const float M = warp_max(ml.x);
+    const float w = (ml.x == -INFINITY || M == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
+    const float L = warp_sum(w * ml.y);
+    const float wl = L > 0.f ? w / L : 0.f;
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + pb * HD) + lane;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int s0 = 0; s0 < nsplit; s0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            v[q] = s0 + q < nsplit ? __ldcg(po + (int64_t)(s0 + q) * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float wq = __shfl_sync(0xffffffffu, wl, (s0 + q) & 31);
+            acc.x += wq * v[q].x;
+            acc.y += wq * v[q].y;
+            acc.z += wq * v[q].z;
+            acc.w += wq * v[q].w;
+        }
+    }
+    uint2 o2;
+    o2.x = pack_bf16(acc.x, acc.y);
+    o2.y = pack_bf16(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(p.out + ((int64_t)row * p.hq + h) * HD + lane * 4) = o2;
 }
 
 }  // namespace
@@ -810,16 +983,18 @@ int attn_max_splits() { return MAX_SPLITS; }
 
 int attn_kv_chunk_for(int max_batch, int max_window, int hq, int hkv, int max_ctx, int num_sms) {
     // Fixed per context (a sequence's result does not depend on its batch
-    // neighbours): a full batch at half the context length makes about two
-    // items per SM; at least four 64-key blocks per chunk (below that the item
-    // setup and the merge of many partials outweigh the extra parallelism), at
-    // most 32 blocks, and at most attn_max_splits() chunks per row tile.
+    // neighbours): a full batch at half the context length makes about one
+    // item per CTA (two CTAs per SM; every further item of a CTA waits for its
+    // Q to load, the CTA's one Q buffer being busy until the item before has
+    // issued its last S); at least four 64-key blocks per chunk, at most 32
+    // blocks, and at most attn_max_splits() chunks per row tile.
     const int g = hq / hkv;
     const int rt = attn_rows_per_tile(g);
     const long long tiles = (max_window + rt - 1) / rt;
     const long long pairs = (long long)max_batch * tiles * hkv;
     const long long blocks = pairs * std::max(1, (max_ctx / 2 + 63) / 64);
-    long long cb = (blocks + 2LL * num_sms - 1) / (2LL * num_sms);
+    const long long ctas = (long long)CTAS_PER_SM * num_sms;
+    long long cb = (blocks + ctas - 1) / ctas;
     cb = std::max(4LL, std::min(cb, 32LL));
     cb = std::max(cb, ((long long)max_ctx + 64LL * MAX_SPLITS - 1) / (64LL * MAX_SPLITS));
     return (int)(cb * 64);
@@ -841,17 +1016,17 @@ bool make_q_tmap(CUtensorMap* tm, const bf16* q, int rows, int hq, int hkv, bool
 
 cudaError_t launch_attn_bf16(const CUtensorMap& tm_kv, const CUtensorMap& tm_q, const CUtensorMap& tm_q_dual,
                              KVLayout kvl, int layer, int hq, int hkv, bf16* out, float* part_o, float2* part_ml,
-                             int* tickets, int n_entries, int stride, int kv_chunk, int max_splits, SlotState ss,
-                             RowMap rm, int* err, cudaStream_t st) {
+                             int n_entries, int stride, int kv_chunk, int max_splits, SlotState ss, RowMap rm,
+                             int* err, cudaStream_t st) {
     if (hq % hkv || hq / hkv > QROWS || max_splits < 1 || max_splits > MAX_SPLITS || kv_chunk < KBLK ||
-        kv_chunk % KBLK || n_entries < 1 || stride < 1)
+        kv_chunk % KBLK || n_entries < 1 || stride < 1 || (max_splits > 1 && (!part_o || !part_ml)))
         return cudaErrorInvalidValue;
     const int g = hq / hkv;
     // DUAL when every query row of a window fits in 64 (one tile of 64 / g rows)
     const bool dual = stride * g <= 64;
     const int rt = dual ? attn_dual_rows_per_tile(g) : attn_rows_per_tile(g);
     const int tiles = (stride + rt - 1) / rt;
-    AttnParams p{kvl, layer, hq, hkv, out, part_o, part_ml, tickets, n_entries, stride, kv_chunk, max_splits, rt, tiles,
+    AttnParams p{kvl, layer, hq, hkv, out, part_o, part_ml, n_entries, stride, kv_chunk, max_splits, rt, tiles,
                  ss, rm, err};
     static int attr_dev = -1;
     static int num_sms = 148;
@@ -869,8 +1044,13 @@ cudaError_t launch_attn_bf16(const CUtensorMap& tm_kv, const CUtensorMap& tm_q, 
     // two persistent CTAs per SM, fewer when the launch has fewer items
     const long long items_max = (long long)n_entries * tiles * hkv * max_splits;
     const int grid = (int)std::max(1LL, std::min<long long>(items_max, (long long)CTAS_PER_SM * num_sms));
-    if (dual) return launch_pdl(attn_tc_kernel<true>, dim3(grid), dim3(NTHREADS), SMEM_BYTES, st, tm_kv, tm_q_dual, p);
-    return launch_pdl(attn_tc_kernel<false>, dim3(grid), dim3(NTHREADS), SMEM_BYTES, st, tm_kv, tm_q, p);
+    cudaError_t e = dual ? launch_pdl(attn_tc_kernel<true>, dim3(grid), dim3(NTHREADS), SMEM_BYTES, st, tm_kv,
+                                      tm_q_dual, p)
+                         : launch_pdl(attn_tc_kernel<false>, dim3(grid), dim3(NTHREADS), SMEM_BYTES, st, tm_kv, tm_q, p);
+    if (e != cudaSuccess || max_splits == 1) return e;
+    MergeParams mp{part_o, part_ml, out, n_entries, stride, hq, rt, kv_chunk, max_splits, ss, rm};
+    const long long pairs = (long long)n_entries * stride * hq;
+    return launch_pdl(attn_merge_kernel, dim3((unsigned)((pairs + 7) / 8)), dim3(256), 0, st, mp);
 }
 
 }  // namespace wedlm

@@ -167,13 +167,26 @@ __device__ __forceinline__ bool stalled(int* err) {
     return err && *reinterpret_cast<volatile int*>(err) == kErrTimeout;
 }
 
+// The same probe, but a thread whose phase is not complete is suspended until
+// it completes or about `ns` nanoseconds have passed, instead of returning at
+// once: waiting warps then take no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* err,
                                                   long long limit_cycles = 2000000000LL) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 1023u) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((it & 15u) == 0) {
             if (stalled(err)) return false;
             if (clock64() - t0 > limit_cycles) {
                 set_error(err, kErrTimeout);

@@ -113,17 +113,17 @@ bool make_kv_tmap(CUtensorMap* tm, const bf16* kv_pool, const KVLayout& kvl, int
 // Tensor map over q [rows][hq][128] with boxes of 64 dims x g heads x the
 // attention's rows per tile (dual: the tile of windows with <= 64 query rows).
 bool make_q_tmap(CUtensorMap* tm, const bf16* q, int rows, int hq, int hkv, bool dual);
-// Decode/prefill attention (persistent: one CTA per SM).  With more than one
-// key chunk per row tile (kv_chunk < keys), partials go to part_o [rows][hq]
-// [max_splits][128] / part_ml [rows][hq][max_splits] and the last chunk of
-// each (entry, KV head, tile) to finish merges them; `tickets` holds
-// entries * hkv * tiles ints that are zero between launches; max_splits <=
-// attn_max_splits(), and every sequence's S + n must fit in max_splits chunks
-// (otherwise the bounds check fires).  kv_chunk is a multiple of 64.
+// Decode/prefill attention (persistent: two CTAs per SM).  With more than one
+// key chunk per row tile (kv_chunk < keys), chunk partials go to part_o
+// [rows][hq][max_splits][128] / part_ml [rows][hq][max_splits] and a second
+// kernel, launched behind the attention on the same stream, combines them
+// into `out`; max_splits <= attn_max_splits(), and every sequence's S + n must
+// fit in max_splits chunks (otherwise the bounds check fires).  kv_chunk is a
+// multiple of 64.
 cudaError_t launch_attn_bf16(const CUtensorMap& tm_kv, const CUtensorMap& tm_q, const CUtensorMap& tm_q_dual,
                              KVLayout kvl, int layer, int hq, int hkv, bf16* out, float* part_o, float2* part_ml,
-                             int* tickets, int n_entries, int stride, int kv_chunk, int max_splits, SlotState ss,
-                             RowMap rm, int* err, cudaStream_t st);
+                             int n_entries, int stride, int kv_chunk, int max_splits, SlotState ss, RowMap rm,
+                             int* err, cudaStream_t st);
 // Keys per chunk of the decode attention for a context's capacity (fixed per
 // context, so a sequence's result does not depend on its batch neighbours).
 int attn_kv_chunk_for(int max_batch, int max_window, int hq, int hkv, int max_ctx, int num_sms);

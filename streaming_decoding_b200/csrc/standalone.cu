@@ -107,11 +107,11 @@ wedlm_status wedlm_entropy_select_async(const float* logits, int32_t vocab, int3
 }
 
 // Workspace of the stand-alone attention: [0, 256) the device error word;
-// then the merge tickets, the (m, l) partials and the O partials of the key
-// chunks, each piece 256-byte aligned.
+// then the (m, l) partials and the O partials of the key chunks, each piece
+// 256-byte aligned.
 struct AttnWs {
-    int kv_chunk = 0, max_splits = 0, tiles = 0;
-    size_t off_tickets = 0, off_ml = 0, off_o = 0, bytes = 0;
+    int kv_chunk = 0, max_splits = 0;
+    size_t off_ml = 0, off_o = 0, bytes = 0;
 };
 
 static size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -123,15 +123,11 @@ static bool attn_ws_layout(int n_seq, int stride, int hq, int hkv, int max_ctx, 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int g = hq / hkv;
     w->kv_chunk = attn_kv_chunk_for(n_seq, stride, hq, hkv, max_ctx, sms);
     w->max_splits = (max_ctx + w->kv_chunk - 1) / w->kv_chunk;
     if (w->max_splits > attn_max_splits()) return false;
-    const int rt = attn_rows_per_tile(g);
-    w->tiles = (stride + rt - 1) / rt;
     const size_t rows = (size_t)n_seq * stride;
-    w->off_tickets = 256;
-    w->off_ml = w->off_tickets + round256((size_t)n_seq * hkv * std::max(w->tiles, 1) * sizeof(int));
+    w->off_ml = 256;
     const size_t parts = w->max_splits > 1 ? rows * hq * w->max_splits : 0;
     w->off_o = w->off_ml + round256(parts * sizeof(float2));
     w->bytes = w->off_o + round256(parts * 128 * sizeof(float));
@@ -178,7 +174,7 @@ wedlm_status wedlm_attention_bf16(const void* q, const void* kv_pool, int32_t nu
     cudaStream_t st = (cudaStream_t)stream;
     const cudaError_t e =
         launch_attn_bf16(tm_kv, tm_q, tm_qd, kvl, 0, hq, hkv, (bf16*)out, (float*)(ws + w.off_o),
-                         (float2*)(ws + w.off_ml), (int*)(ws + w.off_tickets), n_seq, stride, w.kv_chunk,
+                         (float2*)(ws + w.off_ml), n_seq, stride, w.kv_chunk,
                          w.max_splits, ss, rm, (int*)ws, st);
     return e == cudaSuccess ? WEDLM_OK : WEDLM_ERR_CUDA;
 }

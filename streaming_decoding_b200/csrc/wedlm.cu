@@ -158,8 +158,6 @@ struct wedlm_ctx {
     bool capturing = false;           // a step is being captured into a CUDA graph: no timing runs
     float* attn_po = nullptr;
     float2* attn_pml = nullptr;
-    int* attn_tickets = nullptr;   // [maxB][hkv][tiles] merge tickets of the key-chunked attention
-    size_t n_attn_tickets = 0;
     CUtensorMap tm_kv{};
     CUtensorMap tm_q{}, tm_q_dual{};
     int attn_kv_chunk = 1 << 30, attn_max_splits = 1;
@@ -447,8 +445,6 @@ wedlm_status check_device_error(wedlm_ctx* ctx, int code) {
     // a GEMM that gave up may leave split-K tickets behind
     if (ctx->tile_counters)
         CK(cudaMemsetAsync(ctx->tile_counters, 0, ctx->n_tile_counters * sizeof(int), ctx->stream));
-    if (ctx->attn_tickets)
-        CK(cudaMemsetAsync(ctx->attn_tickets, 0, ctx->n_attn_tickets * sizeof(int), ctx->stream));
     if (code == kErrTimeout) return fail(ctx, WEDLM_ERR_TIMEOUT, "a bounded device wait timed out");
     if (code == kErrNonFinite)
         return fail(ctx, WEDLM_ERR_NONFINITE, "a masked slot's logits held a NaN or an infinity (slot not filled)");
@@ -552,7 +548,7 @@ wedlm_status forward_bf16(wedlm_ctx* ctx, int slot_base, int n_entries, int stri
             ProfScope ps(ctx, WEDLM_PROF_ATTENTION);
             const cudaError_t ae =
                 launch_attn_bf16(ctx->tm_kv, ctx->tm_q, ctx->tm_q_dual, ctx->kvl, l, ctx->hq, ctx->hkv, ao,
-                                 ctx->attn_po, ctx->attn_pml, ctx->attn_tickets, n_entries, stride, kc, ms, ctx->ss, rm,
+                                 ctx->attn_po, ctx->attn_pml, n_entries, stride, kc, ms, ctx->ss, rm,
                                  ctx->err, ctx->stream);
             if (ae != cudaSuccess)
                 return fail(ctx, WEDLM_ERR_CUDA, std::string("attention launch: ") + cudaGetErrorString(ae));
@@ -950,13 +946,8 @@ wedlm_status wedlm_create(const wedlm_model_cfg* cfg, void* cuda_stream, wedlm_c
     // Attention key chunks for decode: fixed per context (a sequence's result
     // does not depend on its batch neighbours).
     if (ctx->bf16) {
-        const int g = ctx->hq / ctx->hkv;
-        const int rt = attn_rows_per_tile(g);
-        const int tiles = (maxW + rt - 1) / rt;
         ctx->attn_kv_chunk = attn_kv_chunk_for(B, maxW, ctx->hq, ctx->hkv, ctx->max_ctx, ctx->num_sms);
         ctx->attn_max_splits = (ctx->max_ctx + ctx->attn_kv_chunk - 1) / ctx->attn_kv_chunk;
-        ctx->n_attn_tickets = (size_t)B * tiles * ctx->hkv;
-        sa.add((void**)&ctx->attn_tickets, ctx->n_attn_tickets * sizeof(int));
     }
     if (sa.commit(ctx->stream) != cudaSuccess) return bail(WEDLM_ERR_OOM_DEVICE);
     ss.out_count = ctx->res_dev;
