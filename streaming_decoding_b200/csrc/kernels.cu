@@ -516,6 +516,11 @@ __device__ __forceinline__ SampAcc samp_merge(SampAcc x, SampAcc y) {
 // A NaN or an infinity among z leaves a NaN in s or t (R22: the row is then
 // reported invalid by the selection).
 constexpr int kScanVec = 10;
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __global__ void __launch_bounds__(256) entropy_scan_kernel(const float* logits, int64_t ld, int V,
                                                            int mask_id, float scale,
                                                            const uint8_t* rowmask, int chunks,
@@ -530,48 +535,68 @@ __global__ void __launch_bounds__(256) entropy_scan_kernel(const float* logits, 
     const float4* z4 = reinterpret_cast<const float4*>(logits + (int64_t)row * ld + v0);
     constexpr float kLog2e = 1.4426950408889634f;
     EntAcc acc{-INFINITY, 0.f, 0.f, INT_MAX};
+    // The mask id and ids past the chunk end read -FLT_MAX: never a maximum
+    // (ties do not replace), weight 2^(-288) = 0 below.  Non-finite logits are
+    // caught by chk = sum z * 0 (NaN as soon as one z is a NaN or an
+    // infinity), which makes the partial's sums NaN (the row is then invalid).
+    float chk = 0.f;
     for (int b = 0; b < nvec; b += 256 * kScanVec) {
         float4 v[kScanVec];
+        // all loads of the block first, in flight together
 #pragma unroll
         for (int k = 0; k < kScanVec; ++k) {
             const int i = b + threadIdx.x + k * 256;
-            v[k] = i < nvec ? __ldcg(z4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[k] = i < nvec ? __ldcg(z4 + i) : make_float4(-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX);
         }
-        float m = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kScanVec; ++k) {
+            const unsigned off = (unsigned)(mask_id - (v0 + 4 * (b + threadIdx.x + k * 256)));
+            if (off < 4u) {
+                if (off == 0) v[k].x = -FLT_MAX;
+                else if (off == 1) v[k].y = -FLT_MAX;
+                else if (off == 2) v[k].z = -FLT_MAX;
+                else v[k].w = -FLT_MAX;
+            }
+        }
+        // maximum and its first index, compared on the raw logits (scale > 0
+        // keeps their order)
+        float zm = -FLT_MAX;
         int a = INT_MAX;
+        float c4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < kScanVec; ++k) {
-            const int i = b + threadIdx.x + k * 256;
+            const int id = v0 + 4 * (b + threadIdx.x + k * 256);
+            if (v[k].x > zm) { zm = v[k].x; a = id; }
+            if (v[k].y > zm) { zm = v[k].y; a = id + 1; }
+            if (v[k].z > zm) { zm = v[k].z; a = id + 2; }
+            if (v[k].w > zm) { zm = v[k].w; a = id + 3; }
+            c4[0] = fmaf(v[k].x, 0.f, c4[0]);
+            c4[1] = fmaf(v[k].y, 0.f, c4[1]);
+            c4[2] = fmaf(v[k].z, 0.f, c4[2]);
+            c4[3] = fmaf(v[k].w, 0.f, c4[3]);
+        }
+        chk += (c4[0] + c4[1]) + (c4[2] + c4[3]);
+        if (a == INT_MAX) continue;  // nothing but the mask id and padding
+        // e = 2^(d log2 e), d = scale z - m (clamped at -200: e is 0 there);
+        // four independent partial sums per thread
+        const float m = scale * zm;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f}, tw[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < kScanVec; ++k) {
             const float zz[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int id = v0 + 4 * i + q;
-                const float z = scale * zz[q];
-                if (i < nvec && id != mask_id && z > m) {
-                    m = z;
-                    a = id;
-                }
+                const float d = fmaxf(fmaf(scale, zz[q], -m), -200.f);
+                const float e = ex2_ftz(d * kLog2e);
+                sum[q] += e;
+                tw[q] = fmaf(e, d, tw[q]);
             }
         }
-        float sum = 0.f, tw = 0.f;
-        bool any = false;
-#pragma unroll
-        for (int k = 0; k < kScanVec; ++k) {
-            const int i = b + threadIdx.x + k * 256;
-            const float zz[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int id = v0 + 4 * i + q;
-                if (i < nvec && id != mask_id) {
-                    const float d = scale * zz[q] - m;
-                    const float e = exp2f(d * kLog2e);
-                    sum += e;
-                    tw += e * d;
-                    any = true;
-                }
-            }
-        }
-        if (any) acc = ent_merge(acc, EntAcc{m, sum, tw, a});
+        acc = ent_merge(acc, EntAcc{m, (sum[0] + sum[1]) + (sum[2] + sum[3]), (tw[0] + tw[1]) + (tw[2] + tw[3]), a});
+    }
+    if (chk != 0.f) {  // a NaN or an infinity among this thread's logits
+        acc.s = __int_as_float(0x7fc00000);
+        acc.t = acc.s;
     }
     // the chunk's last (v1 - v0) % 4 ids
     for (int id = v0 + 4 * nvec + threadIdx.x; id < v1; id += blockDim.x)

@@ -20,7 +20,10 @@ it and the GPU's own committed cache of that layer:
 End to end (no teacher forcing) bf16 arithmetic itself drifts with depth on
 this random-init model: the exact oracle and an oracle that rounds at the bf16
 mode's points differ by about 5e-2 in the logits.  The GPU's own end-to-end
-deviation is printed and only guarded against gross error."""
+deviation is printed and bounded by what it measures with margin: about 5e-2
+against the exact oracle and 4e-2 against the oracle with the bf16 rounding
+points (runs differ by a few thousandths with the tuned GEMM launch shapes),
+guarded at 8e-2 and 6e-2."""
 import numpy as np
 import pytest
 
@@ -125,5 +128,5 @@ def test_full_size_batch16_per_layer_against_oracle():
         e2e[name] = worst_e
     print(f"full-size sampled: sequence {b} (P={len(prompts[b])}, S={S}), {n - nf} masked rows; "
           f"end-to-end logits max-rel vs the exact oracle {e2e['exact']:.3e}, vs the R18 oracle {e2e['r18']:.3e}")
-    # gross-error guards; the measured values are recorded with the design notes
-    assert e2e["exact"] < 0.1 and e2e["r18"] < 0.1
+    # measured about 5.0e-2 / 3.8e-2; guarded with about 1.5x margin
+    assert e2e["exact"] < 0.08 and e2e["r18"] < 0.06, e2e
