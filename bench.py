@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--micro-cell", default=None,
                     help="attn_micro: run one cell 'S,B' (attention, then the entropy pass at s=4) and exit "
                          "(single-kernel captures)")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="kernel case: activation rows of the projection (0 = the batch-16 step's 256; 16 = batch 1)")
     ap.add_argument("--kernel-case", default=None,
                     help="run one projection of the batch-16 step (gemm_qkv|gemm_o|gemm_gate_up|gemm_down|"
                          "gemm_lm_head) three times through wedlm_linear_bf16, or 'attention' (3 decode steps of "
@@ -659,14 +661,14 @@ def attention_case(steps: int = 3):
                       "prefill_attention_launches": cfg["B"] * 2}))
 
 
-def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False):
+def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False, rows: int = 0):
     import torch
     from streaming_decoding_b200 import linear_bf16
     if name == "attention":
         return attention_case()
     cfg = synth.CONFIGS["qwen3_8b_b16"]
     dims = cfg["model"]
-    L, M, N, K = gemm_shapes(dims, cfg["B"] * cfg["W"])[name]
+    L, M, N, K = gemm_shapes(dims, rows if rows > 0 else cfg["B"] * cfg["W"])[name]
     g = torch.Generator(device="cuda").manual_seed(0)
     X = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
@@ -680,7 +682,7 @@ def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False):
 if __name__ == "__main__":
     args = parse()
     if args.kernel_case:
-        kernel_case(args.kernel_case, args.tile_n, args.cta_pair)
+        kernel_case(args.kernel_case, args.tile_n, args.cta_pair, args.rows)
     elif args.workload == "attn_micro" and args.impl == "ours":
         run_micro(args)
     elif args.impl == "reference":
