@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--micro-cell", default=None,
                     help="attn_micro: run one cell 'S,B' (attention, then the entropy pass at s=4) and exit "
                          "(single-kernel captures)")
+    ap.add_argument("--k-splits", type=int, default=0, help="kernel case: pin the GEMM K slices (0 = automatic)")
     ap.add_argument("--rows", type=int, default=0,
                     help="kernel case: activation rows of the projection (0 = the batch-16 step's 256; 16 = batch 1)")
     ap.add_argument("--kernel-case", default=None,
@@ -661,7 +662,7 @@ def attention_case(steps: int = 3):
                       "prefill_attention_launches": cfg["B"] * 2}))
 
 
-def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False, rows: int = 0):
+def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False, rows: int = 0, k_splits: int = 0):
     import torch
     from streaming_decoding_b200 import linear_bf16
     if name == "attention":
@@ -673,16 +674,16 @@ def kernel_case(name: str, tile_n: int = 0, cta_pair: bool = False, rows: int = 
     X = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
     W = (torch.randn(N, K, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
     for _ in range(3):
-        linear_bf16(X, W, tile_n=tile_n, cta_pair=cta_pair)
+        linear_bf16(X, W, tile_n=tile_n, k_splits=k_splits, cta_pair=cta_pair)
     torch.cuda.synchronize()
     print(json.dumps({"kernel_case": name, "M": M, "N": N, "K": K, "weight_bytes": 2 * N * K, "tile_n": tile_n,
-                      "cta_pair": cta_pair}))
+                      "k_splits": k_splits, "cta_pair": cta_pair}))
 
 
 if __name__ == "__main__":
     args = parse()
     if args.kernel_case:
-        kernel_case(args.kernel_case, args.tile_n, args.cta_pair, args.rows)
+        kernel_case(args.kernel_case, args.tile_n, args.cta_pair, args.rows, args.k_splits)
     elif args.workload == "attn_micro" and args.impl == "ours":
         run_micro(args)
     elif args.impl == "reference":
