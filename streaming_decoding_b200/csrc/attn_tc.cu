@@ -82,8 +82,8 @@ constexpr int OFF_ML = OFF_X + XCH_FLOATS * 4;                   // (m, l) per O
 constexpr int ENT_CAP = 256;                                     // entries whose (n, S) are cached
 constexpr int GRP_CAP = 512;                                     // (entry, tile) groups with item prefix sums
 constexpr int OFF_ENT = OFF_ML + NO * QROWS * 8;                  // (n, S) of the launch's entries
-constexpr int OFF_GRP = OFF_ENT + ENT_CAP * 8;                    // items in groups 0..g, per group g
-constexpr int OFF_BAR = OFF_GRP + GRP_CAP * 4;
+constexpr int OFF_GRP = OFF_ENT + ENT_CAP * 8;                    // item prefix sums per group (two)
+constexpr int OFF_BAR = OFF_GRP + 2 * GRP_CAP * 4;
 constexpr int BAR_BYTES = 512;                                    // barriers
 constexpr int SMEM_BYTES = OFF_BAR + BAR_BYTES + 1024 /*align*/;
 static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 228 * 1024, "attention shared memory: two CTAs per SM");
@@ -249,7 +249,7 @@ struct Item {
 // may start before the previous kernel of the stream has finished; n and S
 // are not written by it.
 struct ItemIter {
-    int g = 0;                 // current group (prefix-sum search)
+    int g = 0, g2 = 0;         // current group of the full-chunk / last-chunk items (bisection)
     int e = 0, t = 0;          // current group
     int base = 0;              // number of the group's first item
     int next = 0;              // next number this CTA takes
@@ -286,11 +286,12 @@ __device__ __forceinline__ int group_items(const AttnParams& p, const int2* ent,
     return p.hkv * nsplit;
 }
 
-__device__ __forceinline__ void fill_item(const AttnParams& p, int g, int local, int S, int n, int nsplit, Item& o) {
+__device__ __forceinline__ void fill_item(const AttnParams& p, int g, int kvh, int sp, int S, int n, int nsplit,
+                                          Item& o) {
     o.entry = g / p.tiles;
     o.tile = g - o.entry * p.tiles;
-    o.kvh = local / nsplit;
-    o.sp = local % nsplit;
+    o.kvh = kvh;
+    o.sp = sp;
     o.slot = p.rm.slot_base + o.entry;
     o.S = S;
     o.n = n;
@@ -303,24 +304,48 @@ __device__ __forceinline__ void fill_item(const AttnParams& p, int g, int local,
     o.nblk = (o.ke - o.ks + KBLK - 1) / KBLK;
 }
 
-// The CTA's next item.  With at most GRP_CAP groups the item number is looked
-// up by bisection in the per-group prefix sums `gend` (built once per CTA);
-// otherwise the groups are walked one by one.
+// First g in [lo, G) with a[g] > x (a non-decreasing, a[G - 1] > x).
+__device__ __forceinline__ int bisect(const int* a, int lo, int G, int x) {
+    int hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (a[mid] > x) hi = mid;
+        else lo = mid + 1;
+    }
+    return lo;
+}
+
+// The CTA's next item.  With at most GRP_CAP groups the items are numbered
+// full chunks first -- (group, KV head, chunk) for every chunk but a group's
+// last -- then every group's last chunk (KV head order), and the number is
+// looked up by bisection in per-group prefix sums built once per CTA (gend:
+// full-chunk items, gend + GRP_CAP: last-chunk items).  Dealt round-robin,
+// this puts a short tail chunk beside a full chunk on an SM's two CTAs, where
+// the plain (group, head, chunk) order alternated them so that the two CTAs of
+// an SM often both drew full chunks.  Otherwise the groups are walked one by
+// one in (group, head, chunk) order.
 __device__ __forceinline__ bool next_item(ItemIter& it, const AttnParams& p, const int2* ent, const int* gend,
                                           Item& o) {
     const int G = p.n_entries * p.tiles;
     if (G <= GRP_CAP) {
-        if (G == 0 || it.next >= gend[G - 1]) return false;
-        int lo = it.g, hi = G - 1;  // the group holding item it.next: first g with gend[g] > it.next
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (gend[mid] > it.next) hi = mid;
-            else lo = mid + 1;
-        }
-        it.g = lo;
+        if (G == 0) return false;
+        const int* glast = gend + GRP_CAP;
+        const int nfull = gend[G - 1];
+        if (it.next >= nfull + glast[G - 1]) return false;
         int S, n, nsplit;
-        group_items(p, ent, lo, S, n, nsplit);
-        fill_item(p, lo, it.next - (lo ? gend[lo - 1] : 0), S, n, nsplit, o);
+        if (it.next < nfull) {
+            const int g = bisect(gend, it.g, G, it.next);
+            it.g = g;
+            group_items(p, ent, g, S, n, nsplit);
+            const int local = it.next - (g ? gend[g - 1] : 0);
+            fill_item(p, g, local / (nsplit - 1), local % (nsplit - 1), S, n, nsplit, o);
+        } else {
+            const int x = it.next - nfull;
+            const int g = bisect(glast, it.g2, G, x);
+            it.g2 = g;
+            group_items(p, ent, g, S, n, nsplit);
+            fill_item(p, g, x - (g ? glast[g - 1] : 0), nsplit - 1, S, n, nsplit, o);
+        }
         it.next += gridDim.x;
         return true;
     }
@@ -328,7 +353,8 @@ __device__ __forceinline__ bool next_item(ItemIter& it, const AttnParams& p, con
         const int g = it.e * p.tiles + it.t;
         if (it.cnt < 0) it.cnt = group_items(p, ent, g, it.S, it.n, it.nsplit);
         if (it.next < it.base + it.cnt) {
-            fill_item(p, g, it.next - it.base, it.S, it.n, it.nsplit, o);
+            const int local = it.next - it.base;
+            fill_item(p, g, local / it.nsplit, local % it.nsplit, it.S, it.n, it.nsplit, o);
             it.next += gridDim.x;
             return true;
         }
@@ -488,7 +514,7 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
     float* xch = reinterpret_cast<float*>(smem + OFF_X);     // DUAL exchange
     float2* sml = reinterpret_cast<float2*>(smem + OFF_ML);  // [NO][128] (m, l) per row
     int2* ent = reinterpret_cast<int2*>(smem + OFF_ENT);      // [ENT_CAP] (n, S) per entry
-    int* gend = reinterpret_cast<int*>(smem + OFF_GRP);       // [GRP_CAP] items in groups 0..g
+    int* gend = reinterpret_cast<int*>(smem + OFF_GRP);       // [2][GRP_CAP] item prefix sums per group
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* q_full = bars;              // [NQ]
     uint64_t* q_empty = q_full + NQ;      // [NQ]
@@ -546,19 +572,30 @@ __global__ void __launch_bounds__(NTHREADS, CTAS_PER_SM) attn_tc_kernel(const __
     }
     __syncthreads();
     if (warp == 0 && p.n_entries * p.tiles <= GRP_CAP) {
-        // items per group, then an inclusive prefix sum over the groups
+        // full-chunk and last-chunk items per group, then inclusive prefix sums
         const int G = p.n_entries * p.tiles;
-        int carry = 0;
+        int carry = 0, carry2 = 0;
         for (int g0 = 0; g0 < G; g0 += 32) {
-            int S, n, nsplit, v = 0;
-            if (g0 + lane < G) v = group_items(p, ent, g0 + lane, S, n, nsplit);
+            int S, n, nsplit, v = 0, v2 = 0;
+            if (g0 + lane < G && group_items(p, ent, g0 + lane, S, n, nsplit) > 0) {
+                v = p.hkv * (nsplit - 1);
+                v2 = p.hkv;
+            }
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
+                const int u2 = __shfl_up_sync(0xffffffffu, v2, o);
+                if (lane >= o) {
+                    v += u;
+                    v2 += u2;
+                }
             }
-            if (g0 + lane < G) gend[g0 + lane] = carry + v;
+            if (g0 + lane < G) {
+                gend[g0 + lane] = carry + v;
+                gend[GRP_CAP + g0 + lane] = carry2 + v2;
+            }
             carry += __shfl_sync(0xffffffffu, v, 31);
+            carry2 += __shfl_sync(0xffffffffu, v2, 31);
         }
     }
     if (warp == WARP_MMA) {
