@@ -970,33 +970,39 @@ struct MergeParams {
 };
 
 __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
-    griddep_wait();
-    griddep_launch();
     const int lane = threadIdx.x & 31;
     const int64_t pair = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (pair >= (int64_t)p.n_entries * p.stride * p.hq) return;
-    const int row = (int)(pair / p.hq), h = (int)(pair % p.hq);
+    const bool have = pair < (int64_t)p.n_entries * p.stride * p.hq;
+    const int row = have ? (int)(pair / p.hq) : 0, h = have ? (int)(pair % p.hq) : 0;
     const int e = row / p.stride, r = row - e * p.stride;
     const int slot = p.rm.slot_base + e;
-    const int n = __ldcg(p.rm.n + slot);
-    if (r >= n) return;
-    const int S = __ldcg(p.ss.S + slot);
+    // n and S are not written by the attention kernel: read before the wait
+    const int n = have ? __ldcg(p.rm.n + slot) : 0;
+    const int S = have ? __ldcg(p.ss.S + slot) : 0;
+    griddep_wait();
+    griddep_launch();
+    if (!have || r >= n) return;
     const int nsplit = tile_splits(S, n, r / p.rt, p.rt, p.kv_chunk);
     if (nsplit <= 1 || nsplit > p.max_splits) return;
     const int64_t pb = ((int64_t)row * p.hq + h) * p.max_splits;
+    // the (m, l) of every chunk and the first 8 chunk outputs, all in flight
     const float2 ml = lane < nsplit ? __ldcg(p.part_ml + pb + lane) : make_float2(-INFINITY, 0.f);
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + pb * HD) + lane;
+    float4 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = q < nsplit ? __ldcg(po + (int64_t)q * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
     const float M = warp_max(ml.x);
     const float w = (ml.x == -INFINITY || M == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
     const float L = warp_sum(w * ml.y);
     const float wl = L > 0.f ? w / L : 0.f;
-    const float4* po = reinterpret_cast<const float4*>(p.part_o + pb * HD) + lane;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
     for (int s0 = 0; s0 < nsplit; s0 += 8) {
-        float4 v[8];
+        if (s0 > 0) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            v[q] = s0 + q < nsplit ? __ldcg(po + (int64_t)(s0 + q) * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < 8; ++q)
+                v[q] = s0 + q < nsplit ? __ldcg(po + (int64_t)(s0 + q) * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const float wq = __shfl_sync(0xffffffffu, wl, (s0 + q) & 31);

@@ -145,9 +145,13 @@ def test_fused_lm_head_entropy_matches_two_pass():
     """Greedy bf16 steps reduce the vocabulary in the LM head's epilogue (per-32-id
     partials, merged) instead of writing logits and scanning them: every step's
     H~, fills, commits and the token streams equal those of the two-pass path
-    run on the same inputs (H~ within the decision margin)."""
+    run on the same inputs (H~ within the decision margin).  The two runs see
+    the same inputs at every step (equal streams), so the fused H~ and argmax
+    are also checked against the oracle's entropy and argmax of the two-pass
+    run's logits, and its fills against the oracle's rule where comparable."""
     from streaming_decoding_b200 import step_params
     N, W = 24, 16
+    lam, tau, scale = 0.05, 6.0, 16.0
     prompts = _prompts()
     runs = []
     for keep in (False, True):
@@ -156,20 +160,40 @@ def test_fused_lm_head_entropy_matches_two_pass():
         eng.keep_logits(keep)
         for b, p in prompts.items():
             eng.prefill(b, p, N, W)
-        prm = step_params(0.05, 6.0, False, 16.0)
+        prm = step_params(lam, tau, False, scale)
         trace, active = [], 3
         while active:
             _, _, active = eng.stream_step(prm)
+            rows = None
+            if keep:
+                stride, nrows = eng.last_rows()
+                rows = (eng.debug_read("PERM", nrows, np.int32).reshape(-1, stride).copy(),
+                        eng.debug_read("LOGITS", (nrows, MID["V"]), np.float32).reshape(-1, stride, MID["V"]).copy())
             trace.append((eng.debug_read("KN", (3, 3), np.int32).copy(),
                           eng.debug_read("HTILDE", (3, 16), np.float32).copy(),
                           eng.debug_read("FILL", (3, 16), np.uint8).copy(),
-                          eng.debug_read("ARGMAX", (3, 16), np.int32).copy()))
+                          eng.debug_read("ARGMAX", (3, 16), np.int32).copy(), rows))
         runs.append((trace, [eng.read_generated(b) for b in prompts]))
         eng.close()
     (tf, gf), (tt, gt) = runs
     assert gf == gt and len(tf) == len(tt)
-    for (kf, hf, ff, af), (kt, ht, ft, at) in zip(tf, tt):
+    checked = 0
+    for (kf, hf, ff, af, _), (kt, ht, ft, at, rows) in zip(tf, tt):
         assert (kf == kt).all() and (ff == ft).all() and (af == at).all()
         ok = ~np.isnan(ht)
         assert (np.isnan(hf) == ~ok).all()
         assert np.abs(hf[ok] - ht[ok]).max(initial=0.0) < MARGIN
+        perm, z = rows
+        for b in range(3):
+            k, n, nf = (int(v) for v in kt[b])
+            if n == 0 or nf == n:
+                continue
+            by_slot = {int(perm[b, r]): z[b, r] for r in range(nf, n)}
+            Ho, amo, fills = oracle_select(by_slot, MID["mask_id"], lam, tau, False, scale)
+            for j, h in Ho.items():
+                assert abs(float(hf[b, j]) - h) < MARGIN, (b, j, float(hf[b, j]), h)
+                assert int(af[b, j]) == amo[j]
+            if comparable(Ho, tau, False):
+                assert np.nonzero(ff[b, :n])[0].tolist() == sorted(fills)
+            checked += 1
+    assert checked > 0
