@@ -4,10 +4,11 @@
 // weighted sum, argmax) partials it needs from cudaMallocAsync.  Some callers
 // cannot allow that: a runtime that has already reserved the whole device for
 // its own pool (so any further cudaMalloc fails or fragments what it
-// manages), or a latency-critical host thread that must not risk the implicit
-// device synchronisation an allocation can cause.  This file gives them the
-// same computation with its scratch in a fixed device array owned by the
-// library image instead.
+// manages), or a host thread that must not take the allocator's locks or risk
+// the device-wide synchronisation an allocation can cause (the call still waits
+// for the one stream it is given, as wedlm_entropy_select does).  This file
+// gives them the same computation with its scratch in a fixed device array
+// owned by the library image instead.
 //
 // The array lives in every GPU that loads the library until the process
 // exits.  In host code its name is only a host-side stand-in for the symbol,
