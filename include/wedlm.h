@@ -465,8 +465,9 @@ wedlm_status wedlm_entropy_select_async(const float* logits, int32_t vocab, int3
  * calls leave it as they found it while no error occurs).  Asynchronous: the
  * call enqueues the attention kernel (and, when a window's keys are split
  * into chunks, the kernel that combines them) on `stream` and returns; out
- * and the error word are valid once the stream has been synchronised.  WEDLM_ERR_INVALID_ARG for bad sizes, pointers or a
- * too small workspace, WEDLM_ERR_CUDA if the launch fails. */
+ * and the error word are valid once the stream has been synchronised.
+ * WEDLM_ERR_INVALID_ARG for bad sizes, pointers or a too small workspace,
+ * WEDLM_ERR_CUDA if the launch fails. */
 wedlm_status wedlm_attention_workspace_bytes(int32_t n_seq, int32_t stride, int32_t n_heads, int32_t n_kv_heads,
                                              int32_t max_ctx, int64_t* bytes);
 wedlm_status wedlm_attention_bf16(const void* q, const void* kv_pool, int32_t num_pages, int32_t n_heads,
